@@ -1,0 +1,169 @@
+"""Float64 CPU oracle for attention with a KV cache and fused RoPE.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package; the product path
+(``rotary_embedding_b200``) never does, and the two share no code.
+
+The arithmetic lives in ``oracle.c`` (plain C, double precision, built with
+gcc into ``liboracle.so`` beside it).  This module only builds that library
+and marshals numpy arrays into it.  ``brute.py`` holds a second, pure-Python
+statement of the same definitions for tiny shapes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+FMT_NONE, FMT_FP16, FMT_BF16 = 0, 1, 2
+_FMT = {None: FMT_NONE, "none": FMT_NONE, "fp16": FMT_FP16, "bf16": FMT_BF16,
+        "float16": FMT_FP16, "bfloat16": FMT_BF16}
+
+
+def build(force: bool = False, extra_flags: tuple = (), out_path: str | None = None) -> str:
+    """Compile oracle.c with gcc (-O2, no fast-math) into a shared library."""
+    out = out_path or _LIB_PATH
+    if (not force and out_path is None and os.path.exists(out)
+            and os.path.getmtime(out) >= os.path.getmtime(_SRC)):
+        return out
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+           "-ffp-contract=off", *extra_flags, _SRC, "-o", out, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _bind(lib):
+    d, i64, i32 = ctypes.c_double, ctypes.c_int64, ctypes.c_int
+    P = ctypes.c_void_p
+    lib.oracle_round_one.argtypes = [d, i32]
+    lib.oracle_round_one.restype = d
+    lib.oracle_round.argtypes = [P, i64, i32]
+    lib.oracle_round.restype = None
+    lib.oracle_rope.argtypes = [P, P, i64, i32, P, P, P, i64, i32, i32]
+    lib.oracle_rope.restype = i32
+    lib.oracle_kvcache_fwd.argtypes = [i64, i64, i64, i64, i64, i32, i32, i64,
+                                       P, P, P, P, P, P, P, i64, i32, i32, P,
+                                       i32, d, i32, P, P]
+    lib.oracle_kvcache_fwd.restype = i32
+    lib.oracle_fwd.argtypes = [i64, i64, i64, i64, i64, i32, i32, P, P, P, i32, d, P, P]
+    lib.oracle_fwd.restype = i32
+    return lib
+
+
+def load(path: str | None = None):
+    """Load (building if needed) the oracle library; `path` loads a variant build."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    with _lock:
+        if _lib is None:
+            _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def round_to(x, fmt):
+    """Round float64 values to the nearest fp16/bf16 value (ties to even)."""
+    a = _f64(x).copy()
+    load().oracle_round(_ptr(a), a.size, _FMT[fmt])
+    return a
+
+
+def rope(x, pos, cos_tab, sin_tab, rotary_dim, interleaved, lib=None):
+    """RoPE of rows x[..., d] at table rows pos[...]; returns float64."""
+    lib = lib or load()
+    x = _f64(x)
+    d = x.shape[-1]
+    rows = x.size // d if d else 0
+    pos = np.asarray(pos, dtype=np.int64)
+    if x.ndim == 1:
+        pos = pos.reshape(())
+    pos = np.ascontiguousarray(np.broadcast_to(pos, x.shape[:-1]))
+    cos_tab = _f64(cos_tab)
+    sin_tab = _f64(sin_tab)
+    y = np.empty_like(x)
+    tab_rows = cos_tab.shape[0] if cos_tab.ndim == 2 else 0
+    rc = lib.oracle_rope(_ptr(x), _ptr(y), rows, d, _ptr(pos), _ptr(cos_tab), _ptr(sin_tab),
+                         tab_rows, int(rotary_dim), int(bool(interleaved)))
+    if rc != 0:
+        raise ValueError("position outside the rotary table")
+    return y
+
+
+def kvcache_fwd(q, k_cache, v_cache, k_new, v_new, cos_tab, sin_tab, cache_seqlens,
+                rotary_dim=0, interleaved=False, causal=False, scale=None, fmt=None,
+                lib=None):
+    """The whole attn_with_kvcache path in float64.
+
+    Arrays are [batch, seq, heads, dim] (any float dtype; upconverted exactly).
+    `cache_seqlens` is an int or a per-batch int array.  Returns
+    (out [b, s_q, h_q, d_v], lse [b, h_q, s_q], k_cache', v_cache') with the
+    caches updated copies; the inputs are not modified.
+    """
+    lib = lib or load()
+    q = _f64(q)
+    kc = _f64(k_cache).copy()
+    vc = _f64(v_cache).copy()
+    b, s_q, h_q, d_qk = q.shape
+    _, cap, h_kv, _ = kc.shape
+    d_v = vc.shape[3]
+    if k_new is None:
+        kn = np.zeros((b, 0, h_kv, d_qk))
+        vn = np.zeros((b, 0, h_kv, d_v))
+    else:
+        kn, vn = _f64(k_new), _f64(v_new)
+    s_new = kn.shape[1]
+    seql = np.ascontiguousarray(np.broadcast_to(np.asarray(cache_seqlens, dtype=np.int32), (b,)))
+    r = int(rotary_dim)
+    if r > 0:
+        ct, st = _f64(cos_tab), _f64(sin_tab)
+        tab_rows = ct.shape[0]
+    else:
+        ct = st = np.zeros((1, 1))
+        tab_rows = 0
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(d_qk)
+    out = np.zeros((b, s_q, h_q, d_v))
+    lse = np.zeros((b, h_q, s_q))
+    rc = lib.oracle_kvcache_fwd(b, s_q, s_new, h_q, h_kv, d_qk, d_v, cap,
+                                _ptr(q), _ptr(kc), _ptr(vc), _ptr(kn), _ptr(vn),
+                                _ptr(ct), _ptr(st), tab_rows, r, int(bool(interleaved)),
+                                _ptr(seql), int(bool(causal)), float(scale), _FMT[fmt],
+                                _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle_kvcache_fwd rejected its arguments (code {rc})")
+    return out, lse, kc, vc
+
+
+def fwd(q, k, v, causal=False, scale=None, lib=None):
+    """Cache-less attention in float64: returns (out [b,s_q,h_q,d_v], lse [b,h_q,s_q])."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    b, s_q, h_q, d_qk = q.shape
+    s_k, h_kv = k.shape[1], k.shape[2]
+    d_v = v.shape[3]
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(d_qk)
+    out = np.zeros((b, s_q, h_q, d_v))
+    lse = np.zeros((b, h_q, s_q))
+    rc = lib.oracle_fwd(b, s_q, s_k, h_q, h_kv, d_qk, d_v, _ptr(q), _ptr(k), _ptr(v),
+                        int(bool(causal)), float(scale), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle_fwd rejected its arguments (code {rc})")
+    return out, lse

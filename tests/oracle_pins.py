@@ -1,0 +1,394 @@
+"""Pins for the float64 oracle: facts fixed by the pages or by mathematics.
+
+Each ``pin_*`` function takes a loaded oracle library and raises
+AssertionError if the oracle disagrees with the fact.  test_oracle.py runs
+them against the real oracle (all must hold) and against builds with a
+planted mistake (each mistake must break at least one pin).
+
+Nothing here restates the oracle's formulas: the expected values come from
+closed forms (rotation by a right angle, rotation by zero), invariants
+(norms, relative position, softmax rows summing to one), special cases that
+reduce to a library routine (scipy softmax / logsumexp, numpy float16
+rounding), the pure-Python brute force in oracle/brute.py, and the printed
+outcomes of the flash-attention issue #1402 reproducers.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+from scipy.special import logsumexp, softmax
+
+import oracle
+from oracle import brute
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _tables(rows, r, base=10000.0):
+    j = np.arange(r // 2, dtype=np.float64)
+    ang = np.outer(np.arange(rows, dtype=np.float64), base ** (-2.0 * j / r))
+    return np.cos(ang), np.sin(ang), ang
+
+
+def _const_tables(rows, r, angle):
+    shape = (rows, r // 2)
+    return np.full(shape, math.cos(angle)), np.full(shape, math.sin(angle))
+
+
+# ---------------------------------------------------------------- rounding
+def pin_round_fp16_matches_numpy(lib):
+    rng = np.random.default_rng(1)
+    x = np.concatenate([
+        rng.standard_normal(4000) * 10.0 ** rng.integers(-8, 5, 4000),
+        np.array([65504.0, 65519.99, 65520.0, 1e-8, 2.0 ** -24, 3 * 2.0 ** -25,
+                  1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, -0.0, 5.9604644775390625e-08]),
+    ])
+    got = oracle.round_to(x, "fp16")
+    with np.errstate(over="ignore"):
+        want = x.astype(np.float16).astype(np.float64)
+    assert np.array_equal(got, want), "fp16 rounding differs from numpy's correctly rounded cast"
+
+
+def pin_round_bf16_ties_to_even(lib):
+    # exact bf16 neighbours of 1.0 are 1.0 and 1 + 2^-7; the midpoint ties to the even one
+    cases = {1.0 + 2.0 ** -8: 1.0, 1.0 + 3 * 2.0 ** -8: 1.0 + 2.0 ** -6,
+             1.0 + 2.0 ** -8 + 2.0 ** -30: 1.0 + 2.0 ** -7, -3.0: -3.0,
+             2.0 ** -130: 2.0 ** -130, 3.3895313892515355e38: 3.3895313892515355e38}
+    for x, want in cases.items():
+        assert oracle.round_to(np.array([x]), "bf16")[0] == want, x
+
+
+# ---------------------------------------------------------------- RoPE
+def pin_rope_right_angle_is_rotate_half(lib):
+    """Angle pi/2 (cos 0, sin 1): the RoPE reproducer of issue #1402 gives
+    q*cos + rotate_half(q)*sin = rotate_half(q) = cat(-x2, x1) (half-split);
+    interleaved pairs (a, b) -> (-b, a)."""
+    x = np.arange(1.0, 9.0)[None, :]
+    c, s = _const_tables(1, 8, math.pi / 2)
+    c[:] = 0.0
+    s[:] = 1.0
+    y = oracle.rope(x, [0], c, s, 8, False, lib=lib)
+    assert np.array_equal(y[0], [-5.0, -6.0, -7.0, -8.0, 1.0, 2.0, 3.0, 4.0]), y
+    y = oracle.rope(x, [0], c, s, 8, True, lib=lib)
+    assert np.array_equal(y[0], [-2.0, 1.0, -4.0, 3.0, -6.0, 5.0, -8.0, 7.0]), y
+
+
+def pin_rope_partial_right_angle(lib):
+    """rotary_dim 4 of head_dim 8 (rotary_fraction 0.5 of PR #99): half-split
+    pairs (0,2),(1,3); dims 4..7 unchanged."""
+    x = np.arange(1.0, 9.0)[None, :]
+    c = np.zeros((1, 2))
+    s = np.ones((1, 2))
+    y = oracle.rope(x, [0], c, s, 4, False, lib=lib)
+    assert np.array_equal(y[0], [-3.0, -4.0, 1.0, 2.0, 5.0, 6.0, 7.0, 8.0]), y
+    y = oracle.rope(x, [0], c, s, 4, True, lib=lib)
+    assert np.array_equal(y[0], [-2.0, 1.0, -4.0, 3.0, 5.0, 6.0, 7.0, 8.0]), y
+
+
+def pin_rope_position_zero_and_r_zero_identity(lib):
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((5, 16))
+    c, s, _ = _tables(8, 16)
+    for inter in (False, True):
+        y = oracle.rope(x, [0] * 5, c, s, 16, inter, lib=lib)
+        assert np.array_equal(y, x)
+    y = oracle.rope(x, [3] * 5, c, s, 0, False, lib=lib)
+    assert np.array_equal(y, x)
+
+
+def pin_rope_norm_and_relative_position(lib):
+    """Rotation preserves norms; (R_m q).(R_n k) depends only on m - n."""
+    rng = np.random.default_rng(3)
+    d = r = 32
+    c, s, _ = _tables(64, r)
+    q = rng.standard_normal((1, d))
+    k = rng.standard_normal((1, d))
+    for inter in (False, True):
+        for m in (0, 5, 17, 40):
+            y = oracle.rope(q, [m], c, s, r, inter, lib=lib)
+            assert abs(np.linalg.norm(y) - np.linalg.norm(q)) < 1e-12
+        dots = []
+        for m, n in ((7, 3), (11, 7), (50, 46), (4, 0)):
+            dots.append(float(oracle.rope(q, [m], c, s, r, inter, lib=lib)[0]
+                              @ oracle.rope(k, [n], c, s, r, inter, lib=lib)[0]))
+        assert max(dots) - min(dots) < 1e-10, dots
+        # and it does change with the distance
+        far = float(oracle.rope(q, [20], c, s, r, inter, lib=lib)[0]
+                    @ oracle.rope(k, [0], c, s, r, inter, lib=lib)[0])
+        assert abs(far - dots[0]) > 1e-3
+
+
+def pin_rope_angle_sign(lib):
+    """Counter-clockwise rotation: e_a at angle t maps to (cos t, sin t) on the
+    (a, b) plane, matching the page's q*cos + rotate_half(q)*sin."""
+    t = 0.3
+    c = np.full((1, 1), math.cos(t))
+    s = np.full((1, 1), math.sin(t))
+    y = oracle.rope(np.array([[1.0, 0.0]]), [0], c, s, 2, False, lib=lib)
+    assert np.allclose(y[0], [math.cos(t), math.sin(t)], atol=1e-15)
+    y = oracle.rope(np.array([[0.0, 1.0]]), [0], c, s, 2, True, lib=lib)
+    assert np.allclose(y[0], [-math.sin(t), math.cos(t)], atol=1e-15)
+
+
+def pin_rope_pairings_are_permutations(lib):
+    """Half-split and interleaved differ only by the pairing: permuting dims
+    (j, j+r/2) <-> (2j, 2j+1) maps one onto the other."""
+    rng = np.random.default_rng(4)
+    d, r = 24, 16
+    c, s, _ = _tables(20, r)
+    x = rng.standard_normal((6, d))
+    pos = [0, 1, 5, 9, 13, 19]
+    perm = np.arange(d)
+    for j in range(r // 2):
+        perm[2 * j] = j
+        perm[2 * j + 1] = j + r // 2
+    y_half = oracle.rope(x, pos, c, s, r, False, lib=lib)
+    y_int = oracle.rope(x[:, perm], pos, c, s, r, True, lib=lib)
+    assert np.allclose(y_int, y_half[:, perm], atol=0, rtol=0)
+
+
+def pin_rope_matches_complex_form(lib):
+    rng = np.random.default_rng(5)
+    d, r = 12, 8
+    c, s, ang = _tables(30, r)
+    x = rng.standard_normal((4, d))
+    pos = [0, 3, 17, 29]
+    for inter in (False, True):
+        y = oracle.rope(x, pos, c, s, r, inter, lib=lib)
+        for i, p in enumerate(pos):
+            want = brute.rope_row(list(x[i]), list(ang[p]), r, inter)
+            assert np.allclose(y[i], want, atol=1e-13), (inter, i)
+
+
+# ---------------------------------------------------------------- attention
+def pin_single_key_gives_v(lib):
+    """One key: softmax weight 1, out = v exactly, lse = scale*q.k (issue
+    #1402: every backend agrees at seqlen 1)."""
+    rng = np.random.default_rng(6)
+    q = rng.standard_normal((2, 1, 3, 8))
+    k = rng.standard_normal((2, 1, 3, 8))
+    v = rng.standard_normal((2, 1, 3, 5))
+    for causal in (False, True):
+        out, lse = oracle.fwd(q, k, v, causal=causal, scale=0.7, lib=lib)
+        assert np.array_equal(out, v)
+        want = 0.7 * np.einsum("bshd,bshd->bhs", q, k)
+        assert np.allclose(lse, want, atol=1e-14)
+
+
+def pin_equal_keys_average_values(lib):
+    rng = np.random.default_rng(7)
+    n = 6
+    q = rng.standard_normal((1, 1, 1, 4))
+    k = np.repeat(rng.standard_normal((1, 1, 1, 4)), n, axis=1)
+    v = rng.standard_normal((1, n, 1, 3))
+    out, lse = oracle.fwd(q, k, v, causal=False, scale=1.0, lib=lib)
+    assert np.allclose(out[0, 0, 0], v[0, :, 0].mean(axis=0), atol=1e-14)
+    assert abs(lse[0, 0, 0] - (float(q[0, 0, 0] @ k[0, 0, 0]) + math.log(n))) < 1e-13
+
+
+def pin_probabilities_rows_and_bottom_right_mask(lib):
+    """With V = identity the output rows are the attention weights: each row
+    is a probability vector, zero exactly on the masked keys.  Causal is
+    aligned bottom-right: query i of s_q sees keys j <= i + N - s_q."""
+    rng = np.random.default_rng(8)
+    for s_q, n in ((3, 7), (7, 7), (1, 5), (4, 4)):
+        q = rng.standard_normal((1, s_q, 1, 4))
+        k = rng.standard_normal((1, n, 1, 4))
+        v = np.eye(n)[None, :, None, :]
+        out, _ = oracle.fwd(q, k, v, causal=True, scale=0.5, lib=lib)
+        p = out[0, :, 0, :]
+        assert np.allclose(p.sum(axis=1), 1.0, atol=1e-14)
+        for i in range(s_q):
+            for j in range(n):
+                if j <= i + n - s_q:
+                    assert p[i, j] > 0.0
+                else:
+                    assert p[i, j] == 0.0
+
+
+def pin_matches_textbook_softmax(lib):
+    """scipy softmax(scale q k^T + mask) v and logsumexp, causal and not, with
+    s_q == N (lower-triangular mask) and s_q < N (bottom-right)."""
+    rng = np.random.default_rng(9)
+    for s_q, n, causal in ((5, 5, True), (5, 5, False), (3, 9, True), (2, 6, False)):
+        q = rng.standard_normal((1, s_q, 1, 6))
+        k = rng.standard_normal((1, n, 1, 6))
+        v = rng.standard_normal((1, n, 1, 4))
+        out, lse = oracle.fwd(q, k, v, causal=causal, scale=0.3, lib=lib)
+        sc = 0.3 * q[0, :, 0] @ k[0, :, 0].T
+        if causal:
+            sc = np.where(np.triu(np.ones((s_q, n), bool), k=n - s_q + 1), -np.inf, sc)
+        assert np.allclose(out[0, :, 0], softmax(sc, axis=1) @ v[0, :, 0], atol=1e-13)
+        assert np.allclose(lse[0, 0], logsumexp(sc, axis=1), atol=1e-13)
+
+
+def pin_default_scale(lib):
+    """softmax_scale=None means 1/sqrt(d) ("optimizing-attention-flash", Workflow 2)."""
+    rng = np.random.default_rng(10)
+    q = rng.standard_normal((1, 2, 1, 16))
+    k = rng.standard_normal((1, 3, 1, 16))
+    v = rng.standard_normal((1, 3, 1, 2))
+    a = oracle.fwd(q, k, v, scale=None, lib=lib)
+    b = oracle.fwd(q, k, v, scale=0.25, lib=lib)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def pin_gqa_equals_repeated_heads(lib):
+    """Fewer KV heads ("optimizing-attention-flash", Workflow 2 Step 3): query
+    head h uses kv head h // (h_q/h_kv); equal to MHA with each kv head
+    repeated for its group."""
+    rng = np.random.default_rng(11)
+    h_q, h_kv = 6, 2
+    q = rng.standard_normal((2, 3, h_q, 4))
+    k = rng.standard_normal((2, 5, h_kv, 4))
+    v = rng.standard_normal((2, 5, h_kv, 3))
+    a = oracle.fwd(q, k, v, causal=True, lib=lib)
+    b = oracle.fwd(q, np.repeat(k, 3, axis=2), np.repeat(v, 3, axis=2), causal=True, lib=lib)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    # through the cache path as well
+    kc = rng.standard_normal((2, 8, h_kv, 4))
+    vc = rng.standard_normal((2, 8, h_kv, 3))
+    a = oracle.kvcache_fwd(q, kc, vc, k[:, :3], v[:, :3], None, None, [2, 4], causal=True, lib=lib)
+    b = oracle.kvcache_fwd(q, np.repeat(kc, 3, axis=2), np.repeat(vc, 3, axis=2),
+                           np.repeat(k[:, :3], 3, axis=2), np.repeat(v[:, :3], 3, axis=2),
+                           None, None, [2, 4], causal=True, lib=lib)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+# ---------------------------------------------------------------- whole path
+def _tiny_case(rng, b, s_new, h_q, h_kv, d_qk, d_v, cap, seqlens, r):
+    q = rng.standard_normal((b, s_new, h_q, d_qk))
+    kc = rng.standard_normal((b, cap, h_kv, d_qk))
+    vc = rng.standard_normal((b, cap, h_kv, d_v))
+    kn = rng.standard_normal((b, s_new, h_kv, d_qk))
+    vn = rng.standard_normal((b, s_new, h_kv, d_v))
+    return q, kc, vc, kn, vn
+
+
+def pin_brute_force_whole_path(lib):
+    """The pure-Python enumeration agrees on tiny shapes: RoPE (both pairings,
+    partial), append at per-batch offsets, GQA, bottom-right causal, fp16
+    rounding of the rotated rows (numpy's cast as the rounding routine)."""
+    rng = np.random.default_rng(12)
+    for (b, s_new, h_q, h_kv, d, dv, cap, seql, r, inter, causal) in (
+            (2, 3, 4, 2, 8, 6, 8, [1, 4], 8, False, True),
+            (2, 2, 2, 1, 8, 4, 6, [0, 3], 4, True, True),
+            (1, 1, 3, 3, 6, 6, 5, [4], 6, False, False),
+            (2, 4, 2, 2, 4, 4, 9, [5, 0], 0, False, True)):
+        q, kc, vc, kn, vn = _tiny_case(rng, b, s_new, h_q, h_kv, d, dv, cap, seql, r)
+        c, s, ang = _tables(cap, max(r, 2))
+        out, lse, kc2, vc2 = oracle.kvcache_fwd(q, kc, vc, kn, vn, c, s, seql, rotary_dim=r,
+                                                interleaved=inter, causal=causal, scale=0.4,
+                                                fmt="fp16", lib=lib)
+        bo, bl, bkc, bvc = brute.kvcache_fwd(
+            q.tolist(), kc.tolist(), vc.tolist(), kn.tolist(), vn.tolist(),
+            lambda p: list(ang[p]), seql, r, inter, causal, 0.4,
+            round_fn=lambda t: float(np.float16(t)))
+        assert np.allclose(out, np.array(bo), atol=1e-12)
+        assert np.allclose(lse, np.array(bl), atol=1e-12)
+        assert np.array_equal(kc2, np.array(bkc)) and np.array_equal(vc2, np.array(bvc))
+
+
+def pin_append_rows_and_canaries(lib):
+    """Cache append: rows L_b .. L_b+s_new-1 get rope(k_new) rounded and the raw
+    v_new bits; every other row is untouched (flash_attn_with_kvcache usage of
+    issue #1402, cache_seqlens offsets)."""
+    rng = np.random.default_rng(13)
+    b, s_new, h, d, cap, r = 3, 2, 2, 8, 10, 8
+    q, kc, vc, kn, vn = _tiny_case(rng, b, s_new, h, h, d, d, cap, None, r)
+    kc = oracle.round_to(kc, "bf16")
+    vc = oracle.round_to(vc, "bf16")
+    c, s, _ = _tables(cap, r)
+    seql = [0, 3, 8]
+    _, _, kc2, vc2 = oracle.kvcache_fwd(q, kc, vc, kn, vn, c, s, seql, rotary_dim=r,
+                                        causal=True, fmt="bf16", lib=lib)
+    for bi, L in enumerate(seql):
+        for row in range(cap):
+            if L <= row < L + s_new:
+                i = row - L
+                want_k = oracle.round_to(oracle.rope(kn[bi, i], [row] * h, c, s, r, False,
+                                                     lib=lib), "bf16")
+                assert np.array_equal(kc2[bi, row], want_k)
+                assert np.array_equal(vc2[bi, row], vn[bi, i])
+            else:
+                assert np.array_equal(kc2[bi, row], kc[bi, row])
+                assert np.array_equal(vc2[bi, row], vc[bi, row])
+
+
+def pin_query_rotation_positions(lib):
+    """The rotated query used by attention is q rotated at row L_b + i: with a
+    single cached key at position p and its own rotation built in, the score
+    of query i equals (R_{L+i} q_i).(R_p k)."""
+    rng = np.random.default_rng(15)
+    d = 8
+    c, s, _ = _tables(32, d)
+    L, s_new = 5, 3
+    q = rng.standard_normal((1, s_new, 1, d))
+    kc = np.zeros((1, 12, 1, d))
+    vc = np.zeros((1, 12, 1, 1))
+    kn = rng.standard_normal((1, s_new, 1, d))
+    vn = np.zeros((1, s_new, 1, 1))
+    # v = 1 on key 0 only, so out = weight of key 0
+    vc[0, 0, 0, 0] = 1.0
+    kc[0, 0, 0] = rng.standard_normal(d)
+    out, lse, kc2, _ = oracle.kvcache_fwd(q, kc, vc, kn, vn, c, s, [L], rotary_dim=d,
+                                          causal=True, scale=1.0, lib=lib)
+    for i in range(s_new):
+        qi = oracle.rope(q[0, i, 0], [L + i], c, s, d, False, lib=lib)
+        scores = np.array([qi @ kc2[0, j, 0] for j in range(L + i + 1)])
+        assert abs(out[0, i, 0, 0] - softmax(scores)[0]) < 1e-12
+        assert abs(lse[0, 0, i] - logsumexp(scores)) < 1e-12
+
+
+def pin_issue_1402_no_rope(lib):
+    """The no-RoPE reproducer of issue #1402: q = k = v ~ U[0,1) fp16, zero
+    cache, cache_seqlens=0, non-causal.  Seqlen 1: the output is v exactly
+    (all backends agree to 1e-5).  Seqlen 2: the textbook softmax."""
+    rng = np.random.default_rng(16)
+    for seqlen in (1, 2):
+        x = oracle.round_to(rng.random((4, seqlen, 16, 16)), "fp16")
+        zero = np.zeros((4, seqlen, 16, 16))
+        out, lse, _, _ = oracle.kvcache_fwd(x, zero, zero, x, x, None, None, 0,
+                                            causal=False, fmt="fp16", lib=lib)
+        if seqlen == 1:
+            assert np.array_equal(out, x)
+        for bi in range(4):
+            for h in range(16):
+                qh = x[bi, :, h]
+                sc = 0.25 * qh @ qh.T
+                assert np.allclose(out[bi, :, h], softmax(sc, axis=1) @ qh, atol=1e-13)
+
+
+def pin_issue_1402_double_rotation(lib):
+    """The RoPE reproducer of issue #1402 rotates q/k itself and then passes the
+    rotated tensors with rotary_cos/sin again.  At seqlen 1 (position 0,
+    cos=1, sin=0) the double rotation is invisible; at seqlen 2 it is not
+    (FLASHCACHE differs from SDPA at atol 1e-3).  Rotating once matches the
+    unrotated-input path with kernel RoPE."""
+    with open(os.path.join(GOLDEN, "issue1402_rope_outcomes.json")) as f:
+        printed = json.load(f)
+    rng = np.random.default_rng(17)
+    c, s, _ = _tables(512, 16)
+    c16, s16 = oracle.round_to(c, "fp16"), oracle.round_to(s, "fp16")
+    for seqlen in (1, 2):
+        x = oracle.round_to(rng.random((2, seqlen, 16, 16)), "fp16")
+        zero = np.zeros((2, seqlen, 16, 16))
+        pos = np.arange(seqlen)[None, :, None]
+        xr = oracle.round_to(oracle.rope(x, np.broadcast_to(pos, x.shape[:3]), c16, s16, 16,
+                                         False, lib=lib), "fp16")
+        # SDPA on the rotated tensors, value = unrotated query (the script's value = query)
+        sdpa, _, _, _ = oracle.kvcache_fwd(xr, zero, zero, xr, x, None, None, 0,
+                                           causal=False, fmt="fp16", lib=lib)
+        once, _, _, _ = oracle.kvcache_fwd(x, zero, zero, x, x, c16, s16, 0, rotary_dim=16,
+                                           causal=False, fmt="fp16", lib=lib)
+        twice, _, _, _ = oracle.kvcache_fwd(xr, zero, zero, xr, x, c16, s16, 0, rotary_dim=16,
+                                            causal=False, fmt="fp16", lib=lib)
+        agree_twice = bool(np.allclose(sdpa, twice, atol=1e-3, rtol=0))
+        assert agree_twice == printed[str(seqlen)]["FLASHCACHE_matches_SDPA_atol_1e-3"]
+        assert np.allclose(sdpa, once, atol=1e-3, rtol=0)
+
+
+PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
