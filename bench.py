@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""Benchmark of the attention-with-KV-cache hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one fa_kvcache_fwd (or fa_fwd) call over one batch of seeded
+synthetic input resident in HBM: RoPE of q and the new k rows, cache
+append, and attention over cache + new rows.  The default workload is the
+GQA decode with RoPE (bf16, batch 8, 32 query / 8 kv heads, head dim 128,
+cache capacity 8192, cache_seqlens ~ U{1024..8000}, rotary_dim 64
+half-split); --config picks another.  Decode workloads report HBM GB/s of
+algorithmic bytes, prefill/dense workloads TFLOP/s of algorithmic FLOPs.
+
+Timing: W untimed warm-up steps, then K steps, each timed with CUDA events on
+the launching stream; the L2 is flushed (a 512 MiB write) before every timed
+step, outside the events.  Multi-GPU runs (torchrun, one rank per GPU) give
+every rank its own full copy of the workload (weak scaling, no collective on
+the data path) and report the max over ranks.
+
+--impl reference times the float64 CPU oracle (the correctness reference of
+the tests, not tuned for speed) on a bounded sample of the same workload, on
+rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from rotary_embedding_b200 import workloads as W  # noqa: E402
+
+METRIC = "prefill attention TFLOP/s and decode KV-cache GB/s on 1 B200, % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DEFAULT_CONFIG = "gqa-decode"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(W.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU time budget of the oracle sample (cpu_baseline / reference arm)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+def is_decode(w: W.Workload) -> bool:
+    return w.mode == "kvcache" and w.s_q <= 8
+
+
+def work_units(w: W.Workload, seqlens):
+    """(algorithmic amount per step, unit, bound) for the workload."""
+    if is_decode(w):
+        return W.kvcache_bytes(w, seqlens) / 1e9, "GB/s", "hbm"
+    return W.flops(w, seqlens) / 1e12, "TFLOP/s", "tensor"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- traffic record
+def traffic_record(kernel_tag: str):
+    """DRAM traffic per launch from the committed ncu summary of this kernel, if
+    it was taken on the current kernel source (its sha256 prefix must match)."""
+    src = {"decode": "decode.cu", "prefill": "prefill_sm100.cu"}.get(kernel_tag)
+    summ = os.path.join(ROOT, "profiles", f"traffic_{kernel_tag}.md")
+    if not src or not os.path.exists(summ):
+        return None
+    path = os.path.join(ROOT, "rotary_embedding_b200", "csrc", src)
+    if not os.path.exists(path):
+        return None
+    sha = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    text = open(summ).read()
+    m = re.search(r"source_sha256_16:\s*([0-9a-f]{16}).*?traffic_bytes_per_launch_full_size:\s*([0-9.eE+]+)",
+                  text, re.S)
+    if not m or m.group(1) != sha:
+        return None
+    return float(m.group(2))
+
+
+# ----------------------------------------------------------------------------- our arm
+def make_step(w, inp_dev, fa):
+    if w.mode == "dense":
+        q, k, v = inp_dev["q"], inp_dev["k"], inp_dev["v"]
+        out = torch.empty(q.shape[:3] + (w.d_v,), dtype=q.dtype, device=q.device)
+        lse = torch.empty((w.batch, w.h_q, w.s_q), dtype=torch.float32, device=q.device)
+
+        def step():
+            fa.fa_fwd(q, k, v, causal=w.causal, softmax_scale=w.scale or None, out=out, lse=lse)
+        plan = fa.fa_fwd_plan(q, k, v)
+        return step, plan, (out, lse)
+    d = inp_dev
+    out = torch.empty((w.batch, w.s_q, w.h_q, w.d_v), dtype=d["q"].dtype, device=d["q"].device)
+    lse = torch.empty((w.batch, w.h_q, w.s_q), dtype=torch.float32, device=d["q"].device)
+    ws_bytes = fa.fa_kvcache_workspace_size(d["q"], d["k_cache"], d["v_cache"], d["k_new"], w.rotary_dim)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=d["q"].device)
+    seq = d["cache_seqlens"] if not w.seqlens_scalar else int(d["cache_seqlens"][0].item())
+
+    def step():
+        fa.fa_kvcache_fwd(d["q"], d["k_cache"], d["v_cache"], d["k_new"], d["v_new"], d.get("cos"),
+                          d.get("sin"), cache_seqlens=seq, rotary_dim=w.rotary_dim or None,
+                          rotary_interleaved=w.interleaved, causal=w.causal,
+                          softmax_scale=w.scale or None, out=out, lse=lse, workspace=ws)
+    plan = fa.fa_kvcache_plan(d["q"], d["k_cache"], d["v_cache"], d["k_new"], w.rotary_dim)
+    return step, plan, (out, lse)
+
+
+def time_steps(step, steps, warmup, stream, flush_buf, barrier):
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        flush_buf.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+def time_e2e(w, inp_host, inp_dev, step_fn_factory, steps, warmup, stream, flush_buf, barrier):
+    """End-to-end through the public API: per step, copy the step's inputs from
+    pinned host memory, run the call, read out + lse back to pinned host memory."""
+    names = ["q", "k", "v"] if w.mode == "dense" else ["q", "k_new", "v_new", "cache_seqlens"]
+    pinned = {n: inp_host[n].pin_memory() for n in names}
+    step, _, (out, lse) = step_fn_factory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+
+    def e2e_step():
+        for n in names:
+            inp_dev[n].copy_(pinned[n], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+    times = time_steps(e2e_step, steps, warmup, stream, flush_buf, barrier)
+    return times, h2d, d2h
+
+
+def cpu_sample(w, inp, budget_s):
+    """Time the float64 oracle on successive batch entries of the workload until
+    the budget is spent; returns (amount processed in the metric's unit numerator,
+    seconds, description)."""
+    import oracle
+    t_total, amount, done = 0.0, 0.0, []
+    b = 0
+    while not done or (t_total < budget_s and len(done) < 4 * w.batch):
+        bi = b % w.batch
+        if w.mode == "dense":
+            # one (batch, head) pair, every query row
+            h = (b // w.batch) % w.h_q
+            q = inp["q"][bi:bi + 1, :, h:h + 1].double().numpy()
+            hk = h // (w.h_q // w.h_kv)
+            k = inp["k"][bi:bi + 1, :, hk:hk + 1].double().numpy()
+            v = inp["v"][bi:bi + 1, :, hk:hk + 1].double().numpy()
+            t0 = time.perf_counter()
+            oracle.fwd(q, k, v, causal=w.causal, scale=w.softmax_scale())
+            dt = time.perf_counter() - t0
+            sub = w.scaled(batch=1, h_q=1, h_kv=1)
+            amount += W.flops(sub) / 1e12
+            done.append(f"b{bi}h{h}")
+        else:
+            L = int(inp["cache_seqlens"][bi])
+            n = L + w.s_q
+            args = [inp["q"][bi:bi + 1], inp["k_cache"][bi:bi + 1, :n], inp["v_cache"][bi:bi + 1, :n],
+                    inp["k_new"][bi:bi + 1], inp["v_new"][bi:bi + 1]]
+            args = [a.double().numpy() for a in args]
+            cs = inp["cos"].double().numpy() if "cos" in inp else None
+            sn = inp["sin"].double().numpy() if "sin" in inp else None
+            t0 = time.perf_counter()
+            oracle.kvcache_fwd(*args, cs, sn, [L], rotary_dim=w.rotary_dim, interleaved=w.interleaved,
+                               causal=w.causal, scale=w.softmax_scale(), fmt=w.dtype)
+            dt = time.perf_counter() - t0
+            sub = w.scaled(batch=1)
+            amount += (W.kvcache_bytes(sub, [L]) / 1e9 if is_decode(w) else W.flops(sub, [L]) / 1e12)
+            done.append(f"b{bi}")
+        t_total += dt
+        b += 1
+    desc = (f"float64 oracle, single thread, on {len(done)} "
+            f"{'(batch, head) pairs' if w.mode == 'dense' else 'batch entries'} of the workload "
+            f"({', '.join(done[:8])}{'...' if len(done) > 8 else ''}); inputs converted to float64 "
+            f"outside the timed region")
+    return amount, t_total, desc
+
+
+def run_ours(args):
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    barrier = (lambda: dist.barrier()) if world > 1 else (lambda: None)
+
+    import rotary_embedding_b200 as fa
+    w = W.CONFIGS[args.config]
+    inp = W.make_inputs(w, seed=0)
+    inp_dev = {k: v.to(device) for k, v in inp.items()}
+    seqlens = inp["cache_seqlens"].tolist() if w.mode == "kvcache" else None
+    amount, unit, bound = work_units(w, seqlens)
+    stream = torch.cuda.current_stream(device)
+    flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
+
+    step, plan, _ = make_step(w, inp_dev, fa)
+    with ClockSampler(local) as clk:
+        times = time_steps(step, args.steps, max(args.warmup, 3), stream, flush_buf, barrier)
+    ms = sum(times) / len(times)
+    t = torch.tensor([ms], device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    value = world * amount / (ms_max / 1e3)
+
+    e2e_times, h2d, d2h = time_e2e(w, inp, inp_dev, lambda: make_step(w, inp_dev, fa), args.steps,
+                                   max(args.warmup, 3), stream, flush_buf, barrier)
+    e_ms = sum(e2e_times) / len(e2e_times)
+    t = torch.tensor([e_ms], device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_value = world * amount / (float(t.item()) / 1e3)
+
+    peaks, peaks_src = load_peaks()
+    if bound == "hbm":
+        peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    else:
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = amount / (ms / 1e3)   # this rank, per launch of the call
+    kernel_tag = "decode" if plan["path"] == fa.FA_PATH_DECODE else "prefill"
+    traffic = traffic_record(kernel_tag)
+    result = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": unit,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": round(ms_max, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded, N(0,1)/U[0,1) as the workload states)",
+        "config": {"workload": w.name, "batch": w.batch, "h_q": w.h_q, "h_kv": w.h_kv,
+                   "d_qk": w.d_qk, "d_v": w.d_v, "s_q": w.s_q,
+                   "cap_or_s_k": w.cap if w.mode == "kvcache" else w.s_k, "causal": w.causal,
+                   "rotary_dim": w.rotary_dim, "interleaved": w.interleaved,
+                   "l2": "flushed before every timed step (512 MiB write, untimed)",
+                   "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU",
+                   "plan": plan},
+        "roofline": {"bound": bound, "achieved": round(achieved, 3), "peak": peak,
+                     "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_source": f"{peaks_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
+                     "kernel": ("decode_kernel (+combine_kernel in the same timed call)"
+                                if kernel_tag == "decode" else "whole call"),
+                     "amount_per_launch": amount},
+        "e2e": {"value": round(e2e_value, 3), "unit": unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(plan["launches"]) * args.steps,
+    }
+    clocks = clk.summary()
+    if clocks:
+        result["clocks"] = clocks
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        amt, secs, desc = cpu_sample(w, inp, args.cpu_seconds)
+        result["cpu_baseline"] = {"value": round(amt / secs, 6), "unit": unit, "cores": 1,
+                                  "kind": "oracle", "sample": desc, "seconds": round(secs, 2)}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = W.CONFIGS[args.config]
+    inp = W.make_inputs(w, seed=0)
+    seqlens = inp["cache_seqlens"].tolist() if w.mode == "kvcache" else None
+    _, unit, _ = work_units(w, seqlens)
+    # each step is one bounded sample; the whole run stays within a few minutes
+    per_step = max(0.2, min(5.0, 60.0 / max(args.steps, 1)))
+    for _ in range(max(args.warmup, 0)):
+        cpu_sample(w, inp, 0.0)
+    vals, tot_amt, tot_s, desc = [], 0.0, 0.0, ""
+    for _ in range(args.steps):
+        amt, secs, desc = cpu_sample(w, inp, per_step)
+        vals.append(amt / secs)
+        tot_amt += amt
+        tot_s += secs
+    value = tot_amt / tot_s
+    result = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit,
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": {"workload": w.name},
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,212 @@
+"""Attention with a KV cache and fused RoPE on NVIDIA B200 (sm_100a).
+
+A thin Python binding over the C ABI of ``libfa.so`` (declared in
+``include/fa.h``).  Functions carry the C names; they only marshal torch
+tensors into ``fa_tensor`` descriptors, pick the current CUDA stream, let
+torch allocate outputs and the workspace, and raise on a non-zero status.
+Every step of the computation runs in the library's CUDA kernels; there is
+no CPU or PyTorch fallback: if the library is missing, importing this
+package raises.
+
+Argument names follow flash_attn_with_kvcache as used on flash-attention
+issue #1402 (rotary_cos, rotary_sin, cache_seqlens, rotary_interleaved,
+causal, softmax_scale).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = -1
+FA_ERR_UNSUPPORTED = -2
+FA_ERR_LAYOUT = -3
+FA_ERR_WORKSPACE = -4
+FA_ERR_CUDA = -5
+FA_ERR_DEVICE_PRECONDITION = -6
+FA_ERR_DEVICE_TIMEOUT = -7
+FA_DTYPE_F16 = 1
+FA_DTYPE_BF16 = 2
+
+_DTYPES = {torch.float16: FA_DTYPE_F16, torch.bfloat16: FA_DTYPE_BF16}
+
+
+class FaTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{message} (status {status})")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m rotary_embedding_b200.build`")
+lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.POINTER(FaTensor)
+_v = ctypes.c_void_p
+_i32 = ctypes.c_int32
+lib.fa_kvcache_fwd.argtypes = [_P, _P, _P, _P, _P, _P, _P, _v, _i32, _i32, _i32, _i32, ctypes.c_float,
+                               _P, _v, _v, ctypes.c_size_t, _v]
+lib.fa_kvcache_fwd.restype = ctypes.c_int
+lib.fa_kvcache_workspace_size.argtypes = [_P, _P, _P, _P, _i32, ctypes.POINTER(ctypes.c_size_t)]
+lib.fa_kvcache_workspace_size.restype = ctypes.c_int
+lib.fa_fwd.argtypes = [_P, _P, _P, _i32, ctypes.c_float, _P, _v, _v, ctypes.c_size_t, _v]
+lib.fa_fwd.restype = ctypes.c_int
+lib.fa_fwd_workspace_size.argtypes = [_P, _P, _P, ctypes.POINTER(ctypes.c_size_t)]
+lib.fa_fwd_workspace_size.restype = ctypes.c_int
+lib.fa_device_status.argtypes = [_v, ctypes.POINTER(ctypes.c_int32)]
+lib.fa_device_status.restype = ctypes.c_int
+lib.fa_status_string.argtypes = [ctypes.c_int]
+lib.fa_status_string.restype = ctypes.c_char_p
+lib.fa_last_error.argtypes = []
+lib.fa_last_error.restype = ctypes.c_char_p
+lib.fa_version.argtypes = []
+lib.fa_version.restype = ctypes.c_int
+
+
+def describe(t: torch.Tensor | None):
+    """fa_tensor descriptor of a torch tensor (None -> NULL)."""
+    if t is None:
+        return None
+    d = FaTensor()
+    d.data = t.data_ptr()
+    d.dtype = _DTYPES.get(t.dtype, 0)
+    d.ndim = t.dim()
+    for k in range(min(t.dim(), 4)):
+        d.shape[k] = t.shape[k]
+        d.stride[k] = t.stride(k)
+    return d
+
+
+def _ref(d):
+    return ctypes.byref(d) if d is not None else None
+
+
+def _check(status: int):
+    if status != FA_OK:
+        msg = lib.fa_last_error().decode() or lib.fa_status_string(status).decode()
+        raise FaError(status, msg)
+
+
+def _stream_handle(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def fa_kvcache_workspace_size(q, k_cache, v_cache, k_new=None, rotary_dim=0) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.fa_kvcache_workspace_size(_ref(describe(q)), _ref(describe(k_cache)),
+                                         _ref(describe(v_cache)), _ref(describe(k_new)),
+                                         int(rotary_dim), ctypes.byref(n)))
+    return n.value
+
+
+def fa_fwd_workspace_size(q, k, v) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.fa_fwd_workspace_size(_ref(describe(q)), _ref(describe(k)), _ref(describe(v)),
+                                     ctypes.byref(n)))
+    return n.value
+
+
+def fa_kvcache_fwd(q, k_cache, v_cache, k_new=None, v_new=None, rotary_cos=None, rotary_sin=None,
+                   cache_seqlens=0, rotary_dim=None, rotary_interleaved=False, causal=False,
+                   softmax_scale=None, out=None, lse=None, workspace=None, return_lse=True,
+                   stream=None):
+    """RoPE of q/k_new at positions cache_seqlens[b] + i, append of the rotated
+    k and raw v into k_cache/v_cache (in place), then attention over cache and
+    new rows.  Tensors are [batch, seq, heads, dim] CUDA tensors; cache_seqlens
+    is an int or an int32 CUDA tensor [batch].  Returns (out, lse)."""
+    b, s_q, h_q, _ = q.shape
+    d_v = v_cache.shape[3]
+    if rotary_cos is not None and rotary_dim is None:
+        rotary_dim = 2 * rotary_cos.shape[1]
+    rotary_dim = int(rotary_dim or 0) if rotary_cos is not None else 0
+    if out is None:
+        out = torch.empty((b, s_q, h_q, d_v), dtype=q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
+    ws_bytes = fa_kvcache_workspace_size(q, k_cache, v_cache, k_new, rotary_dim)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    if isinstance(cache_seqlens, torch.Tensor):
+        seq_ptr, seq_scalar = ctypes.c_void_p(cache_seqlens.data_ptr()), 0
+    else:
+        seq_ptr, seq_scalar = None, int(cache_seqlens)
+    dq = describe(q)
+    _check(lib.fa_kvcache_fwd(
+        _ref(dq), _ref(describe(k_cache)), _ref(describe(v_cache)), _ref(describe(k_new)),
+        _ref(describe(v_new)), _ref(describe(rotary_cos)), _ref(describe(rotary_sin)), seq_ptr,
+        seq_scalar, rotary_dim, int(bool(rotary_interleaved)), int(bool(causal)),
+        float(softmax_scale or 0.0), _ref(describe(out)),
+        ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+        ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None,
+        workspace.numel() if workspace is not None else 0, _stream_handle(stream, q.device)))
+    return out, lse
+
+
+def fa_fwd(q, k, v, causal=False, softmax_scale=None, out=None, lse=None, workspace=None,
+           return_lse=True, stream=None):
+    """Cache-less attention: q [b, s_q, h_q, d_qk], k/v [b, s_k, h_kv, d]; returns (out, lse)."""
+    b, s_q, h_q, _ = q.shape
+    d_v = v.shape[3]
+    if out is None:
+        out = torch.empty((b, s_q, h_q, d_v), dtype=q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
+    ws_bytes = fa_fwd_workspace_size(q, k, v)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    _check(lib.fa_fwd(
+        _ref(describe(q)), _ref(describe(k)), _ref(describe(v)), int(bool(causal)),
+        float(softmax_scale or 0.0), _ref(describe(out)),
+        ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+        ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None,
+        workspace.numel() if workspace is not None else 0, _stream_handle(stream, q.device)))
+    return out, lse
+
+
+class FaPlan(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("launches", ctypes.c_int32), ("n_splits", ctypes.c_int32),
+                ("chunk", ctypes.c_int32), ("workspace_bytes", ctypes.c_size_t)]
+
+
+FA_PATH_DECODE, FA_PATH_PREFILL, FA_PATH_DENSE = 1, 2, 3
+lib.fa_kvcache_plan.argtypes = [_P, _P, _P, _P, _i32, ctypes.POINTER(FaPlan)]
+lib.fa_kvcache_plan.restype = ctypes.c_int
+lib.fa_fwd_plan.argtypes = [_P, _P, _P, ctypes.POINTER(FaPlan)]
+lib.fa_fwd_plan.restype = ctypes.c_int
+
+
+def fa_kvcache_plan(q, k_cache, v_cache, k_new=None, rotary_dim=0) -> dict:
+    p = FaPlan()
+    _check(lib.fa_kvcache_plan(_ref(describe(q)), _ref(describe(k_cache)), _ref(describe(v_cache)),
+                               _ref(describe(k_new)), int(rotary_dim), ctypes.byref(p)))
+    return {k: getattr(p, k) for k, _ in FaPlan._fields_}
+
+
+def fa_fwd_plan(q, k, v) -> dict:
+    p = FaPlan()
+    _check(lib.fa_fwd_plan(_ref(describe(q)), _ref(describe(k)), _ref(describe(v)), ctypes.byref(p)))
+    return {k: getattr(p, k) for k, _ in FaPlan._fields_}
+
+
+def fa_device_status(stream=None) -> int:
+    """Synchronise and read (then clear) the device status word."""
+    s = ctypes.c_int32(0)
+    h = ctypes.c_void_p(stream.cuda_stream) if stream is not None else None
+    _check(lib.fa_device_status(h, ctypes.byref(s)))
+    return s.value
+
+
+def fa_version() -> int:
+    return lib.fa_version()

@@ -1,0 +1,482 @@
+// decode.cu -- split-KV decode attention with fused RoPE + cache append, and
+// the LSE combine of the split partials.
+//
+// Path (decode branch of the attention-with-KV-cache call: s2.cpp PR #40's
+// single-token branch, flash-attention issue #1402's flash_attn_with_kvcache
+// with a short new chunk):
+//  * grid (split, kv head, batch).  A split owns key rows
+//    [split * chunk, min((split + 1) * chunk, N_b)) of one (batch, kv head);
+//    splits past N_b exit at once.  All g * s_q query rows that read this kv
+//    head (grouped-query heads of the "optimizing-attention-flash" page,
+//    Workflow 2 Step 3) are packed into one 16- or 32-row MMA tile, so each
+//    key/value row is read from HBM once.
+//  * warp 4 streams 64-row K and V tiles of the cache with TMA (128-byte
+//    swizzled boxes) through a ring of shared-memory stages; warps 0-3 each
+//    take 16 keys of every tile, keep their own running max / sum / output
+//    (online softmax) and meet only once at the end.
+//  * the tile that holds rows >= L_b is patched in shared memory by the warp
+//    that owns those keys: new key rows are rotated (same rotation as the
+//    append kernel) and rounded, new value rows copied, and both written to
+//    the cache (this CTA is the only one owning those rows); rows >= N_b
+//    are zeroed so garbage past the sequence cannot reach the PV product.
+//  * q rows are rotated at position L_b + i while being staged.
+//  * a split that covers all of N_b writes out / lse directly; otherwise it
+//    writes its normalised partial output and lse to the workspace and the
+//    combine kernel merges them: lse = log sum exp(lse_s),
+//    out = sum exp(lse_s - lse) * out_s.
+//
+// QK^T and PV use mma.sync m16n8k16 (fp32 accumulate): with at most 32 query
+// rows per kv head the product is far from the tensor-core roof and the
+// kernel is bound by the HBM stream of the cache.
+#include <algorithm>
+
+#include "fa_common.cuh"
+#include "fa_internal.h"
+
+namespace fa {
+
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int D_QK, int D_V, int MT>
+struct DecodeCfg {
+    static constexpr int TILE = 64;
+    static constexpr int KBYTES = TILE * D_QK * 2;
+    static constexpr int VBYTES = TILE * D_V * 2;
+    static constexpr int STAGE = KBYTES + VBYTES;
+    static constexpr int STAGES_RAW = (112 * 1024) / STAGE;
+    static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 8 ? 8 : STAGES_RAW);
+    static constexpr int QROWS = MT * 16;
+    static constexpr int QBYTES = ((QROWS * D_QK * 2 + 1023) / 1024) * 1024;
+    static constexpr int MERGE_BYTES = 4 * QROWS * (D_V + 2) * 4;
+    static constexpr int SMEM = 1024 + QBYTES + STAGES * STAGE + 2 * STAGES * 8;
+    static_assert(MERGE_BYTES <= STAGES * STAGE, "merge scratch must fit in the stage ring");
+    static_assert(D_QK % 16 == 0 && D_V % 16 == 0, "head dims are multiples of 16");
+};
+
+template <typename T, int D_QK, int D_V, int MT>
+__global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                     const __grid_constant__ CUtensorMap tmV,
+                                                     const DecodeParams p) {
+    using C = DecodeCfg<D_QK, D_V, MT>;
+    constexpr int CHK = box_cols(D_QK), RBK = box_row_bytes(D_QK);
+    constexpr int CHV = box_cols(D_V), RBV = box_row_bytes(D_V);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem;
+    uint8_t *sStage = smem + C::QBYTES;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sStage + C::STAGES * C::STAGE);
+    uint64_t *empty = full + C::STAGES;
+
+    const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int L = seqlen_of(p.seqlens, p.seqlen_scalar, b);
+    const int64_t N64 = (int64_t)L + p.s_new;
+    if (L < 0 || N64 > p.cap ||
+        (p.r > 0 && (int64_t)L + (p.s_q > p.s_new ? p.s_q : p.s_new) > p.cs_rows)) {
+        if (threadIdx.x == 0 && split == 0 && hk == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
+        return;
+    }
+    const int N = (int)N64;
+    const int row_begin = split * p.chunk;
+    if (N == 0) {
+        // no key at all (empty cache, no new rows): out = 0, lse = -inf
+        if (split == 0) {
+            for (int idx = threadIdx.x; idx < p.g * p.s_q * (D_V / 8); idx += blockDim.x) {
+                const int row = idx / (D_V / 8), c = idx % (D_V / 8);
+                const int i = row / p.g, hq = hk * p.g + row % p.g;
+                T *dst = static_cast<T *>(p.out) + b * p.os.b + i * p.os.s + hq * p.os.h;
+                reinterpret_cast<uint4 *>(dst)[c] = make_uint4(0, 0, 0, 0);
+                if (c == 0 && p.lse) p.lse[((int64_t)b * p.h_q + hq) * p.s_q + i] = -INFINITY;
+            }
+        }
+        return;
+    }
+    if (row_begin >= N) return;
+    const int row_end = min(row_begin + p.chunk, N);
+    const int n_tiles = (row_end - row_begin + C::TILE - 1) / C::TILE;
+    const int n_splits_b = (N + p.chunk - 1) / p.chunk;
+    const int M = p.g * p.s_q;
+    const int hq0 = hk * p.g;
+    const bool inter = p.interleaved != 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 4);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == 4) {
+        // ---------------- producer: TMA stream of K/V tiles ----------------
+        if (lane == 0) {
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            for (int t = 0; t < n_tiles; ++t) {
+                const int s = t % C::STAGES;
+                if (t >= C::STAGES && !mbar_wait(&empty[s], ((t / C::STAGES) - 1) & 1, p.status)) break;
+                mbar_arrive_expect_tx(&full[s], C::STAGE);
+                uint8_t *kd = sStage + s * C::STAGE;
+                uint8_t *vd = kd + C::KBYTES;
+                const int row = row_begin + t * C::TILE;
+#pragma unroll
+                for (int c = 0; c < D_QK / CHK; ++c)
+                    tma_load_4d(kd + c * C::TILE * RBK, &tmK, &full[s], c * CHK, hk, row, b);
+#pragma unroll
+                for (int c = 0; c < D_V / CHV; ++c)
+                    tma_load_4d(vd + c * C::TILE * RBV, &tmV, &full[s], c * CHV, hk, row, b);
+            }
+        }
+        return;
+    }
+
+    // ---------------- consumers: stage rotated q ----------------
+    const T *cos_t = static_cast<const T *>(p.cos);
+    const T *sin_t = static_cast<const T *>(p.sin);
+    for (int idx = threadIdx.x; idx < C::QROWS * (D_QK / 8); idx += 128) {
+        const int r = idx / (D_QK / 8), c = idx % (D_QK / 8);
+        float f[8];
+        if (r < M) {
+            const int i = r / p.g, hq = hq0 + r % p.g;
+            const T *src = static_cast<const T *>(p.q) + b * p.qs.b + i * p.qs.s + hq * p.qs.h;
+            const int64_t pos = (int64_t)L + i;
+            load_rotated_chunk<T>(src, c, p.r, inter, p.r ? cos_t + pos * p.cs_row : nullptr,
+                                  p.r ? sin_t + pos * p.cs_row : nullptr, f);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = 0.f;
+        }
+        *reinterpret_cast<uint4 *>(sQ + swz_offset<D_QK>(r, c * 8, C::QROWS)) = pack8<T>(f);
+    }
+    consumer_sync();
+
+    const uint32_t sQa = smem_addr(sQ);
+    float o[MT][D_V / 8][4];
+    float m_r[MT][2], l_r[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+        for (int n = 0; n < D_V / 8; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[mt][n][e] = 0.f;
+        m_r[mt][0] = m_r[mt][1] = -INFINITY;
+        l_r[mt][0] = l_r[mt][1] = 0.f;
+    }
+    // last visible key per owned query row (bottom-right causal)
+    int last_vis[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int r = mt * 16 + (lane >> 2) + hr * 8;
+            if (r < M) {
+                const int i = r / p.g;
+                last_vis[mt][hr] = p.causal ? min(N - 1, i + N - p.s_q) : N - 1;
+            } else {
+                last_vis[mt][hr] = -1;
+            }
+        }
+
+    constexpr int CK = D_QK / 8, CV = D_V / 8;
+    for (int t = 0; t < n_tiles; ++t) {
+        const int s = t % C::STAGES;
+        // on a timeout leave the loop (not the kernel) so every consumer warp
+        // still reaches the named barriers below
+        if (!mbar_wait(&full[s], (t / C::STAGES) & 1, p.status)) break;
+        uint8_t *sK = sStage + s * C::STAGE;
+        uint8_t *sV = sK + C::KBYTES;
+        const int tile_row0 = row_begin + t * C::TILE;
+        const int key0 = tile_row0 + warp * 16;
+
+        if (key0 + 16 > L) {
+            // patch this warp's rows >= L_b: new rows (rotated k, raw v) or zeros
+            for (int item = lane; item < 16 * (CK + CV); item += 32) {
+                const int rr = item / (CK + CV), c = item % (CK + CV);
+                const int j = key0 + rr;
+                if (j < L) continue;
+                const int tr = warp * 16 + rr;
+                if (j < N) {
+                    const int i = j - L;
+                    if (c < CK) {
+                        const T *src = static_cast<const T *>(p.k_new) + b * p.kn.b + i * p.kn.s + hk * p.kn.h;
+                        float f[8];
+                        load_rotated_chunk<T>(src, c, p.r, inter, p.r ? cos_t + (int64_t)j * p.cs_row : nullptr,
+                                              p.r ? sin_t + (int64_t)j * p.cs_row : nullptr, f);
+                        const uint4 v = pack8<T>(f);
+                        *reinterpret_cast<uint4 *>(sK + swz_offset<D_QK>(tr, c * 8, C::TILE)) = v;
+                        T *dst = static_cast<T *>(p.k_cache) + b * p.kc.b + (int64_t)j * p.kc.s + hk * p.kc.h;
+                        reinterpret_cast<uint4 *>(dst)[c] = v;
+                    } else {
+                        const int cv = c - CK;
+                        const T *src = static_cast<const T *>(p.v_new) + b * p.vn.b + i * p.vn.s + hk * p.vn.h;
+                        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(src) + cv);
+                        *reinterpret_cast<uint4 *>(sV + swz_offset<D_V>(tr, cv * 8, C::TILE)) = v;
+                        T *dst = static_cast<T *>(p.v_cache) + b * p.vc.b + (int64_t)j * p.vc.s + hk * p.vc.h;
+                        reinterpret_cast<uint4 *>(dst)[cv] = v;
+                    }
+                } else {
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    if (c < CK)
+                        *reinterpret_cast<uint4 *>(sK + swz_offset<D_QK>(tr, c * 8, C::TILE)) = z;
+                    else
+                        *reinterpret_cast<uint4 *>(sV + swz_offset<D_V>(tr, (c - CK) * 8, C::TILE)) = z;
+                }
+            }
+            fence_proxy_async();
+            __syncwarp();
+        }
+
+        // S = Q K^T over this warp's 16 keys
+        float sacc[MT][2][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sacc[mt][nt][e] = 0.f;
+        const uint32_t sKa = smem_addr(sK), sVa = smem_addr(sV);
+#pragma unroll
+        for (int kk = 0; kk < D_QK / 16; ++kk) {
+            uint32_t kb[4];
+            ldmatrix_x4(sKa + swz_offset<D_QK>(warp * 16 + (lane & 7) + ((lane >> 4) << 3),
+                                               kk * 16 + (((lane >> 3) & 1) << 3), C::TILE),
+                        kb[0], kb[1], kb[2], kb[3]);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                uint32_t a[4];
+                ldmatrix_x4(sQa + swz_offset<D_QK>(mt * 16 + (lane & 15), kk * 16 + ((lane >> 4) << 3), C::QROWS),
+                            a[0], a[1], a[2], a[3]);
+                Mma<T>::run(sacc[mt][0], a, kb[0], kb[1]);
+                Mma<T>::run(sacc[mt][1], a, kb[2], kb[3]);
+            }
+        }
+
+        // mask + online softmax (base-2, scale folded in)
+        uint32_t pa[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            float pv[2][2][2];  // [hr][nt][e]
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                float vals[2][2];
+                float mx = -INFINITY;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int j = key0 + nt * 8 + ((lane & 3) << 1) + e;
+                        float v = sacc[mt][nt][hr * 2 + e] * p.scale_log2;
+                        if (j > last_vis[mt][hr]) v = -INFINITY;
+                        vals[nt][e] = v;
+                        mx = fmaxf(mx, v);
+                    }
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float m_new = fmaxf(m_r[mt][hr], mx);
+                const float m_use = m_new == -INFINITY ? 0.f : m_new;
+                const float corr = ex2(m_r[mt][hr] - m_use);
+                float sum = 0.f;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        pv[hr][nt][e] = ex2(vals[nt][e] - m_use);
+                        sum += pv[hr][nt][e];
+                    }
+                l_r[mt][hr] = l_r[mt][hr] * corr + sum;
+                m_r[mt][hr] = m_new;
+#pragma unroll
+                for (int n = 0; n < D_V / 8; ++n) {
+                    o[mt][n][hr * 2] *= corr;
+                    o[mt][n][hr * 2 + 1] *= corr;
+                }
+            }
+            pa[mt][0] = Elem<T>::pack2(pv[0][0][0], pv[0][0][1]);
+            pa[mt][1] = Elem<T>::pack2(pv[1][0][0], pv[1][0][1]);
+            pa[mt][2] = Elem<T>::pack2(pv[0][1][0], pv[0][1][1]);
+            pa[mt][3] = Elem<T>::pack2(pv[1][1][0], pv[1][1][1]);
+        }
+
+        // O += P V over this warp's 16 keys
+#pragma unroll
+        for (int nn = 0; nn < D_V / 16; ++nn) {
+            uint32_t vb[4];
+            ldmatrix_x4_trans(sVa + swz_offset<D_V>(warp * 16 + (lane & 7) + (((lane >> 3) & 1) << 3),
+                                                    nn * 16 + ((lane >> 4) << 3), C::TILE),
+                              vb[0], vb[1], vb[2], vb[3]);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                Mma<T>::run(o[mt][2 * nn], pa[mt], vb[0], vb[1]);
+                Mma<T>::run(o[mt][2 * nn + 1], pa[mt], vb[2], vb[3]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+    }
+
+    // ---------------- merge the four warps ----------------
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            l_r[mt][hr] += __shfl_xor_sync(0xffffffffu, l_r[mt][hr], 1);
+            l_r[mt][hr] += __shfl_xor_sync(0xffffffffu, l_r[mt][hr], 2);
+        }
+    consumer_sync();  // every warp is done with the stage ring; reuse it
+    float *red_o = reinterpret_cast<float *>(sStage);
+    float *red_m = red_o + 4 * C::QROWS * D_V;
+    float *red_l = red_m + 4 * C::QROWS;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int row = mt * 16 + (lane >> 2) + hr * 8;
+            if ((lane & 3) == 0) {
+                red_m[warp * C::QROWS + row] = m_r[mt][hr];
+                red_l[warp * C::QROWS + row] = l_r[mt][hr];
+            }
+            float *dst = red_o + (warp * C::QROWS + row) * D_V + ((lane & 3) << 1);
+#pragma unroll
+            for (int n = 0; n < D_V / 8; ++n)
+                *reinterpret_cast<float2 *>(dst + n * 8) = make_float2(o[mt][n][hr * 2], o[mt][n][hr * 2 + 1]);
+        }
+    consumer_sync();
+    for (int idx = threadIdx.x; idx < M * CV; idx += 128) {
+        const int row = idx / CV, c = idx % CV;
+        float mw[4], mx = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            mw[w] = red_m[w * C::QROWS + row];
+            mx = fmaxf(mx, mw[w]);
+        }
+        const float mu = mx == -INFINITY ? 0.f : mx;
+        float ltot = 0.f, acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float sc = ex2(mw[w] - mu);
+            ltot += red_l[w * C::QROWS + row] * sc;
+            const float *src = red_o + (w * C::QROWS + row) * D_V + c * 8;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] += src[e] * sc;
+        }
+        const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] *= inv;
+        const float lse_v = ltot > 0.f ? (mx + log2f(ltot)) * kLn2 : -INFINITY;
+        const int i = row / p.g, hq = hq0 + row % p.g;
+        if (n_splits_b == 1) {
+            T *dst = static_cast<T *>(p.out) + b * p.os.b + i * p.os.s + hq * p.os.h;
+            reinterpret_cast<uint4 *>(dst)[c] = pack8<T>(acc);
+            if (c == 0 && p.lse) p.lse[((int64_t)b * p.h_q + hq) * p.s_q + i] = lse_v;
+        } else {
+            const int64_t part = (((int64_t)split * p.b + b) * p.h_q + hq) * p.s_q + i;
+            float4 *dst = reinterpret_cast<float4 *>(p.o_part + part * D_V + c * 8);
+            dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            if (c == 0) p.lse_part[part] = lse_v;
+        }
+    }
+}
+
+// One warp per (batch, query head, query row): merge the split partials.
+template <typename T>
+__global__ void __launch_bounds__(256) combine_kernel(const DecodeParams p, int d_v) {
+    const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t total = (int64_t)p.b * p.h_q * p.s_q;
+    if (w >= total) return;
+    const int i = (int)(w % p.s_q);
+    const int hq = (int)((w / p.s_q) % p.h_q);
+    const int b = (int)(w / ((int64_t)p.s_q * p.h_q));
+    const int L = seqlen_of(p.seqlens, p.seqlen_scalar, b);
+    const int64_t N64 = (int64_t)L + p.s_new;
+    if (L < 0 || N64 > p.cap ||
+        (p.r > 0 && (int64_t)L + (p.s_q > p.s_new ? p.s_q : p.s_new) > p.cs_rows))
+        return;
+    const int n = (int)((N64 + p.chunk - 1) / p.chunk);
+    if (n <= 1) return;
+    auto part = [&](int s) { return (((int64_t)s * p.b + b) * p.h_q + hq) * p.s_q + i; };
+    float mx = -INFINITY;
+    for (int s = lane; s < n; s += 32) mx = fmaxf(mx, p.lse_part[part(s)]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    T *dst = static_cast<T *>(p.out) + b * p.os.b + i * p.os.s + hq * p.os.h;
+    if (mx == -INFINITY) {
+        for (int c = lane * 2; c < d_v; c += 64) *reinterpret_cast<uint32_t *>(dst + c) = 0u;
+        if (lane == 0 && p.lse) p.lse[((int64_t)b * p.h_q + hq) * p.s_q + i] = -INFINITY;
+        return;
+    }
+    float sum = 0.f;
+    for (int s = lane; s < n; s += 32) sum += ex2((p.lse_part[part(s)] - mx) * kLog2e);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float lse = mx + logf(sum);
+    for (int c = lane * 2; c < d_v; c += 64) {
+        float a0 = 0.f, a1 = 0.f;
+        for (int s = 0; s < n; ++s) {
+            const float wgt = ex2((p.lse_part[part(s)] - lse) * kLog2e);
+            const float2 v = *reinterpret_cast<const float2 *>(p.o_part + part(s) * d_v + c);
+            a0 = fmaf(wgt, v.x, a0);
+            a1 = fmaf(wgt, v.y, a1);
+        }
+        *reinterpret_cast<uint32_t *>(dst + c) = Elem<T>::pack2(a0, a1);
+    }
+    if (lane == 0 && p.lse) p.lse[((int64_t)b * p.h_q + hq) * p.s_q + i] = lse;
+}
+
+template <typename T, int D_QK, int D_V, int MT>
+static cudaError_t run_decode(const DecodeParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                              cudaStream_t st) {
+    using C = DecodeCfg<D_QK, D_V, MT>;
+    static bool configured = false;  // per instantiation, per process
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D_QK, D_V, MT>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    dim3 grid(p.n_splits, p.h_kv, p.b);
+    decode_kernel<T, D_QK, D_V, MT><<<grid, 160, C::SMEM, st>>>(tmK, tmV, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (p.n_splits > 1) {
+        const int64_t warps = (int64_t)p.b * p.h_q * p.s_q;
+        const int64_t blocks = (warps * 32 + 255) / 256;
+        combine_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(p, D_V);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+#define FA_DECODE_DIMS(X) \
+    X(16, 16, 1) X(16, 16, 2) X(32, 32, 1) X(32, 32, 2) X(64, 64, 1) X(64, 64, 2) \
+    X(128, 128, 1) X(128, 128, 2) X(192, 128, 1) X(192, 128, 2) X(256, 256, 1)
+
+bool decode_supported(int d_qk, int d_v, int mt) {
+#define FA_CASE(DQ, DV, MT) if (d_qk == DQ && d_v == DV && mt == MT) return true;
+    FA_DECODE_DIMS(FA_CASE)
+#undef FA_CASE
+    return false;
+}
+
+cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                          int dtype, int d_qk, int d_v, int mt, cudaStream_t st) {
+#define FA_CASE(DQ, DV, MT)                                                          \
+    if (d_qk == DQ && d_v == DV && mt == MT) {                                       \
+        if (dtype == FA_DTYPE_F16) return run_decode<__half, DQ, DV, MT>(p, tmK, tmV, st); \
+        return run_decode<__nv_bfloat16, DQ, DV, MT>(p, tmK, tmV, st);               \
+    }
+    FA_DECODE_DIMS(FA_CASE)
+#undef FA_CASE
+    return cudaErrorInvalidValue;
+}
+
+int decode_stages(int d_qk, int d_v) {
+    int stage = 64 * (d_qk + d_v) * 2;
+    return std::max(2, std::min(8, (112 * 1024) / stage));
+}
+
+}  // namespace fa

@@ -1,0 +1,570 @@
+// fa_api.cu -- the C ABI of libfa.so: argument validation, the planner that
+// picks the kernels for a call, TMA descriptor set-up and the launches.
+//
+// Planner (one GPU, one stream, no allocation):
+//  * fa_kvcache_fwd with a short new chunk (s_q <= 8 and at most 32 query
+//    rows per kv head, the decode branch of s2.cpp PR #40's eval_cached):
+//    one split-KV decode launch that also rotates q / k_new and appends the
+//    new rows, then the LSE combine when a batch entry spans several splits.
+//  * otherwise (the prefill / concat branch): the rope+append kernel, then
+//    the attention kernel over the cache, on the same stream (write before
+//    read, s2.cpp PR #40 review).
+//  * fa_fwd: the attention kernel over dense k/v.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_internal.h"
+
+namespace fa {
+
+// The device status word (one per device that loads the library).
+__device__ int32_t g_status_word = 0;
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int32_t *status_word() {
+    static int32_t *ptrs[64] = {nullptr};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<int32_t *>(p);
+    }
+    return ptrs[dev];
+}
+
+// ---------------------------------------------------------------- validation
+struct Dims4 {
+    int64_t n[4];
+    int64_t s[4];
+};
+
+int check_tensor(const fa_tensor *t, const char *name, int ndim, int dtype, Dims4 *out) {
+    if (!t) return fail(FA_ERR_INVALID_ARG, "%s is NULL", name);
+    if (!t->data) return fail(FA_ERR_INVALID_ARG, "%s->data is NULL", name);
+    if (t->ndim != ndim) return fail(FA_ERR_INVALID_ARG, "%s must have %d dims (got %d)", name, ndim, t->ndim);
+    if (t->dtype != FA_DTYPE_F16 && t->dtype != FA_DTYPE_BF16)
+        return fail(FA_ERR_UNSUPPORTED, "%s: dtype %d is not fp16/bf16", name, t->dtype);
+    if (dtype && t->dtype != dtype)
+        return fail(FA_ERR_INVALID_ARG, "%s: dtype differs from q", name);
+    for (int k = 0; k < ndim; ++k)
+        if (t->shape[k] < 0) return fail(FA_ERR_INVALID_ARG, "%s: negative size", name);
+    if (t->stride[ndim - 1] != 1 && t->shape[ndim - 1] > 1)
+        return fail(FA_ERR_LAYOUT, "%s: innermost stride must be 1", name);
+    if ((reinterpret_cast<uintptr_t>(t->data) & 15) != 0)
+        return fail(FA_ERR_LAYOUT, "%s: base address not 16-byte aligned", name);
+    for (int k = 0; k < ndim - 1; ++k)
+        if (t->shape[k] > 1 && ((t->stride[k] * 2) % 16 != 0 || t->stride[k] <= 0))
+            return fail(FA_ERR_LAYOUT, "%s: stride of dim %d not a positive multiple of 16 bytes", name, k);
+    if (out) {
+        for (int k = 0; k < 4; ++k) {
+            out->n[k] = k < ndim ? t->shape[k] : 1;
+            out->s[k] = k < ndim ? t->stride[k] : 0;
+        }
+    }
+    return FA_OK;
+}
+
+bool head_dim_ok(int64_t d) { return d >= 8 && d <= 256 && d % 8 == 0; }
+
+Strides3 s3(const Dims4 &d) { return Strides3{d.s[0], d.s[1], d.s[2]}; }
+
+// ---------------------------------------------------------------- TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 4-D map over a [batch, rows, heads, dim] tensor, dims ordered (dim, heads,
+// rows, batch); box = (min(d, 64), 1, box_rows, 1) with the swizzle that
+// matches the box row width.
+int make_rows_map(CUtensorMap *map, const fa_tensor *t, int box_rows, const char *name) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const int64_t d = t->shape[3];
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)t->shape[2], (cuuint64_t)t->shape[1],
+                          (cuuint64_t)t->shape[0]};
+    // strides of dims 1..3 in bytes; a size-1 dim gets the packed stride
+    int64_t sh = t->shape[2] > 1 ? t->stride[2] : d;
+    int64_t ss = t->shape[1] > 1 ? t->stride[1] : sh * t->shape[2];
+    int64_t sb = t->shape[0] > 1 ? t->stride[0] : ss * t->shape[1];
+    cuuint64_t strides[3] = {(cuuint64_t)(sh * 2), (cuuint64_t)(ss * 2), (cuuint64_t)(sb * 2)};
+    const int bc = d < 64 ? (int)d : 64;
+    cuuint32_t box[4] = {(cuuint32_t)bc, 1, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUtensorMapSwizzle sw = bc * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : bc * 2 == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
+                                          : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUtensorMapDataType dt = t->dtype == FA_DTYPE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                      : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = fn(map, dt, 4, t->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed (%d)", name, (int)r);
+    return FA_OK;
+}
+
+// ---------------------------------------------------------------- planning
+struct KvPlan {
+    bool decode = false;
+    int mt = 1;
+    int chunk = 0;
+    int n_splits = 1;
+    size_t ws_bytes = 0;
+    size_t off_lse_part = 0;
+    bool rotate_q_to_ws = false;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+KvPlan plan_kvcache(int64_t b, int64_t s_q, int64_t h_q, int64_t h_kv, int64_t d_qk, int64_t d_v,
+                    int64_t cap, int64_t s_new, bool rotary) {
+    KvPlan pl;
+    const int64_t g = h_q / h_kv;
+    const int64_t M = g * s_q;
+    const int mt = M <= 16 ? 1 : 2;
+    if (s_q <= 8 && M <= 32 && (s_new == 0 || s_new == s_q) && decode_supported((int)d_qk, (int)d_v, mt) &&
+        cap >= 1) {
+        pl.decode = true;
+        pl.mt = mt;
+        // Aim for about 148 SMs x 8 splits in flight over caches that are on
+        // average half full; splits are whole 64-row tiles.
+        const int64_t units = b * h_kv;
+        int64_t chunk = (cap / 2 * units + 148 * 8 - 1) / (148 * 8);
+        chunk = std::max<int64_t>(64, (chunk + 63) / 64 * 64);
+        const int64_t cap_r = (cap + 63) / 64 * 64;
+        chunk = std::min(chunk, cap_r);
+        pl.chunk = (int)chunk;
+        pl.n_splits = (int)((cap + chunk - 1) / chunk);
+        if (pl.n_splits > 1) {
+            const size_t rows = (size_t)pl.n_splits * b * h_q * s_q;
+            pl.off_lse_part = align_up(rows * d_v * sizeof(float), 256);
+            pl.ws_bytes = pl.off_lse_part + align_up(rows * sizeof(float), 256);
+        }
+        return pl;
+    }
+    pl.decode = false;
+    if (rotary) {
+        pl.rotate_q_to_ws = true;
+        pl.ws_bytes = align_up((size_t)b * s_q * h_q * d_qk * 2, 256);
+    }
+    return pl;
+}
+
+struct KvArgs {
+    Dims4 q, kc, vc, kn, vn;
+    int dtype;
+    int64_t b, s_q, h_q, h_kv, d_qk, d_v, cap, s_new, s_ro;
+    int r;
+    bool has_new;
+};
+
+int validate_kvcache(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
+                     const fa_tensor *k_new, const fa_tensor *v_new, const fa_tensor *cos,
+                     const fa_tensor *sin, int32_t rotary_dim, KvArgs *a) {
+    int rc;
+    if ((rc = check_tensor(q, "q", 4, 0, &a->q))) return rc;
+    a->dtype = q->dtype;
+    if ((rc = check_tensor(k_cache, "k_cache", 4, a->dtype, &a->kc))) return rc;
+    if ((rc = check_tensor(v_cache, "v_cache", 4, a->dtype, &a->vc))) return rc;
+    a->b = a->q.n[0];
+    a->s_q = a->q.n[1];
+    a->h_q = a->q.n[2];
+    a->d_qk = a->q.n[3];
+    a->cap = a->kc.n[1];
+    a->h_kv = a->kc.n[2];
+    a->d_v = a->vc.n[3];
+    if (a->kc.n[0] != a->b || a->vc.n[0] != a->b) return fail(FA_ERR_INVALID_ARG, "cache batch differs from q");
+    if (a->kc.n[3] != a->d_qk) return fail(FA_ERR_INVALID_ARG, "k_cache head dim differs from q");
+    if (a->vc.n[1] != a->cap || a->vc.n[2] != a->h_kv)
+        return fail(FA_ERR_INVALID_ARG, "v_cache shape differs from k_cache");
+    if (a->h_kv <= 0 || a->h_q % a->h_kv != 0)
+        return fail(FA_ERR_INVALID_ARG, "h_q (%lld) must be a multiple of h_kv (%lld)", (long long)a->h_q,
+                    (long long)a->h_kv);
+    if (!head_dim_ok(a->d_qk) || !head_dim_ok(a->d_v))
+        return fail(FA_ERR_UNSUPPORTED, "head dims must be multiples of 8 in 8..256 (got %lld/%lld)",
+                    (long long)a->d_qk, (long long)a->d_v);
+    if (a->cap > INT32_MAX || a->s_q > INT32_MAX) return fail(FA_ERR_INVALID_ARG, "sequence too long");
+    a->has_new = k_new != nullptr;
+    if ((k_new == nullptr) != (v_new == nullptr))
+        return fail(FA_ERR_INVALID_ARG, "k_new and v_new must both be given or both be NULL");
+    a->s_new = 0;
+    if (a->has_new) {
+        if ((rc = check_tensor(k_new, "k_new", 4, a->dtype, &a->kn))) return rc;
+        if ((rc = check_tensor(v_new, "v_new", 4, a->dtype, &a->vn))) return rc;
+        a->s_new = a->kn.n[1];
+        if (a->kn.n[0] != a->b || a->kn.n[2] != a->h_kv || a->kn.n[3] != a->d_qk)
+            return fail(FA_ERR_INVALID_ARG, "k_new shape must be [b, s_new, h_kv, d_qk]");
+        if (a->vn.n[0] != a->b || a->vn.n[1] != a->s_new || a->vn.n[2] != a->h_kv || a->vn.n[3] != a->d_v)
+            return fail(FA_ERR_INVALID_ARG, "v_new shape must be [b, s_new, h_kv, d_v]");
+        if (a->s_new != a->s_q)
+            return fail(FA_ERR_INVALID_ARG, "s_new (%lld) must equal s_q (%lld)", (long long)a->s_new,
+                        (long long)a->s_q);
+        if (a->s_new > a->cap) return fail(FA_ERR_INVALID_ARG, "s_new exceeds the cache capacity");
+    }
+    a->r = 0;
+    a->s_ro = 0;
+    if ((cos == nullptr) != (sin == nullptr))
+        return fail(FA_ERR_INVALID_ARG, "cos and sin must both be given or both be NULL");
+    if (cos) {
+        Dims4 dc, ds;
+        if ((rc = check_tensor(cos, "cos", 2, a->dtype, &dc))) return rc;
+        if ((rc = check_tensor(sin, "sin", 2, a->dtype, &ds))) return rc;
+        if (dc.n[0] != ds.n[0] || dc.n[1] != ds.n[1] || dc.s[0] != ds.s[0])
+            return fail(FA_ERR_INVALID_ARG, "cos and sin must have the same shape and strides");
+        if (rotary_dim < 0 || rotary_dim % 2 || rotary_dim > a->d_qk)
+            return fail(FA_ERR_INVALID_ARG, "rotary_dim must be even and <= d_qk (got %d)", rotary_dim);
+        if (rotary_dim > 0 && dc.n[1] < rotary_dim / 2)
+            return fail(FA_ERR_INVALID_ARG, "cos/sin need rotary_dim/2 = %d columns (got %lld)", rotary_dim / 2,
+                        (long long)dc.n[1]);
+        a->r = rotary_dim;
+        a->s_ro = dc.n[0];
+    }
+    return FA_OK;
+}
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+const char *fa_last_error(void) { return g_last_error; }
+
+const char *fa_status_string(int s) {
+    switch (s) {
+        case FA_OK: return "ok";
+        case FA_ERR_INVALID_ARG: return "invalid argument";
+        case FA_ERR_UNSUPPORTED: return "unsupported dtype or head dim";
+        case FA_ERR_LAYOUT: return "unsupported memory layout";
+        case FA_ERR_WORKSPACE: return "workspace missing or too small";
+        case FA_ERR_CUDA: return "CUDA error";
+        case FA_ERR_DEVICE_PRECONDITION: return "cache_seqlens out of range (recorded on the device)";
+        case FA_ERR_DEVICE_TIMEOUT: return "bounded wait timed out on the device";
+        default: return "unknown status";
+    }
+}
+
+int fa_kvcache_workspace_size(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
+                              const fa_tensor *k_new, int32_t rotary_dim, size_t *bytes) {
+    g_last_error[0] = 0;
+    if (!bytes) return fail(FA_ERR_INVALID_ARG, "bytes is NULL");
+    KvArgs a;
+    int rc;
+    if ((rc = check_tensor(q, "q", 4, 0, &a.q))) return rc;
+    if ((rc = check_tensor(k_cache, "k_cache", 4, q->dtype, &a.kc))) return rc;
+    if ((rc = check_tensor(v_cache, "v_cache", 4, q->dtype, &a.vc))) return rc;
+    if (a.kc.n[2] <= 0 || a.q.n[2] % a.kc.n[2]) return fail(FA_ERR_INVALID_ARG, "h_q must be a multiple of h_kv");
+    int64_t s_new = k_new ? k_new->shape[1] : 0;
+    KvPlan pl = plan_kvcache(a.q.n[0], a.q.n[1], a.q.n[2], a.kc.n[2], a.q.n[3], a.vc.n[3], a.kc.n[1], s_new,
+                             rotary_dim > 0);
+    *bytes = pl.ws_bytes;
+    return FA_OK;
+}
+
+int fa_kvcache_plan(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
+                    const fa_tensor *k_new, int32_t rotary_dim, fa_plan *plan) {
+    g_last_error[0] = 0;
+    if (!plan) return fail(FA_ERR_INVALID_ARG, "plan is NULL");
+    Dims4 qd, kd, vd;
+    int rc;
+    if ((rc = check_tensor(q, "q", 4, 0, &qd))) return rc;
+    if ((rc = check_tensor(k_cache, "k_cache", 4, q->dtype, &kd))) return rc;
+    if ((rc = check_tensor(v_cache, "v_cache", 4, q->dtype, &vd))) return rc;
+    if (kd.n[2] <= 0 || qd.n[2] % kd.n[2]) return fail(FA_ERR_INVALID_ARG, "h_q must be a multiple of h_kv");
+    const int64_t s_new = k_new ? k_new->shape[1] : 0;
+    const KvPlan pl = plan_kvcache(qd.n[0], qd.n[1], qd.n[2], kd.n[2], qd.n[3], vd.n[3], kd.n[1], s_new,
+                                   rotary_dim > 0);
+    plan->path = pl.decode ? FA_PATH_DECODE : FA_PATH_PREFILL;
+    plan->n_splits = pl.decode ? pl.n_splits : 1;
+    plan->chunk = pl.decode ? pl.chunk : 0;
+    plan->launches = pl.decode ? (pl.n_splits > 1 ? 2 : 1) : ((s_new > 0 || rotary_dim > 0) ? 2 : 1);
+    plan->workspace_bytes = pl.ws_bytes;
+    return FA_OK;
+}
+
+int fa_fwd_plan(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, fa_plan *plan) {
+    g_last_error[0] = 0;
+    if (!plan) return fail(FA_ERR_INVALID_ARG, "plan is NULL");
+    int rc;
+    if ((rc = check_tensor(q, "q", 4, 0, nullptr))) return rc;
+    if ((rc = check_tensor(k, "k", 4, q->dtype, nullptr))) return rc;
+    if ((rc = check_tensor(v, "v", 4, q->dtype, nullptr))) return rc;
+    plan->path = FA_PATH_DENSE;
+    plan->launches = 1;
+    plan->n_splits = 1;
+    plan->chunk = 0;
+    plan->workspace_bytes = 0;
+    return FA_OK;
+}
+
+int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
+                   const fa_tensor *k_new, const fa_tensor *v_new, const fa_tensor *cos,
+                   const fa_tensor *sin, const int32_t *cache_seqlens, int32_t cache_seqlens_scalar,
+                   int32_t rotary_dim, int32_t interleaved, int32_t causal, float scale,
+                   const fa_tensor *out, float *lse, void *workspace, size_t workspace_bytes,
+                   void *stream) {
+    g_last_error[0] = 0;
+    KvArgs a;
+    int rc = validate_kvcache(q, k_cache, v_cache, k_new, v_new, cos, sin, rotary_dim, &a);
+    if (rc) return rc;
+    Dims4 od;
+    if ((rc = check_tensor(out, "out", 4, a.dtype, &od))) return rc;
+    if (od.n[0] != a.b || od.n[1] != a.s_q || od.n[2] != a.h_q || od.n[3] != a.d_v)
+        return fail(FA_ERR_INVALID_ARG, "out shape must be [b, s_q, h_q, d_v]");
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) return fail(FA_ERR_LAYOUT, "lse not 4-byte aligned");
+    if (!cache_seqlens) {
+        const int64_t L = cache_seqlens_scalar;
+        if (L < 0 || L + a.s_new > a.cap)
+            return fail(FA_ERR_INVALID_ARG, "cache_seqlens %lld + s_new %lld outside capacity %lld", (long long)L,
+                        (long long)a.s_new, (long long)a.cap);
+        if (a.r > 0 && L + std::max(a.s_q, a.s_new) > a.s_ro)
+            return fail(FA_ERR_INVALID_ARG, "rotary table has %lld rows, positions reach %lld", (long long)a.s_ro,
+                        (long long)(L + std::max(a.s_q, a.s_new)));
+    }
+    const KvPlan pl = plan_kvcache(a.b, a.s_q, a.h_q, a.h_kv, a.d_qk, a.d_v, a.cap, a.s_new, a.r > 0);
+    if (pl.ws_bytes > 0 && (workspace == nullptr || workspace_bytes < pl.ws_bytes))
+        return fail(FA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", pl.ws_bytes, workspace_bytes);
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return fail(FA_ERR_LAYOUT, "workspace must be 256-byte aligned");
+    if (a.b == 0 || a.s_q == 0 || a.h_q == 0) return FA_OK;
+    const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)a.d_qk);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t *status = status_word();
+    if (!status) return fail(FA_ERR_CUDA, "no CUDA device");
+    const int cs_row = cos ? (int)cos->stride[0] : 0;
+
+    if (pl.decode) {
+        CUtensorMap tmK, tmV;
+        if ((rc = make_rows_map(&tmK, k_cache, 64, "k_cache"))) return rc;
+        if ((rc = make_rows_map(&tmV, v_cache, 64, "v_cache"))) return rc;
+        DecodeParams p{};
+        p.status = status;
+        p.q = q->data;
+        p.qs = s3(a.q);
+        p.k_new = a.has_new ? k_new->data : nullptr;
+        p.kn = a.has_new ? s3(a.kn) : Strides3{0, 0, 0};
+        p.v_new = a.has_new ? v_new->data : nullptr;
+        p.vn = a.has_new ? s3(a.vn) : Strides3{0, 0, 0};
+        p.k_cache = k_cache->data;
+        p.kc = s3(a.kc);
+        p.v_cache = v_cache->data;
+        p.vc = s3(a.vc);
+        p.cos = a.r ? cos->data : nullptr;
+        p.sin = a.r ? sin->data : nullptr;
+        p.cs_row = cs_row;
+        p.cs_rows = a.s_ro;
+        p.seqlens = cache_seqlens;
+        p.seqlen_scalar = cache_seqlens_scalar;
+        p.out = out->data;
+        p.os = s3(od);
+        p.lse = lse;
+        p.o_part = static_cast<float *>(workspace);
+        p.lse_part = workspace ? reinterpret_cast<float *>(static_cast<char *>(workspace) + pl.off_lse_part) : nullptr;
+        p.b = (int)a.b;
+        p.s_q = (int)a.s_q;
+        p.s_new = (int)a.s_new;
+        p.h_q = (int)a.h_q;
+        p.h_kv = (int)a.h_kv;
+        p.g = (int)(a.h_q / a.h_kv);
+        p.r = a.r;
+        p.interleaved = interleaved ? 1 : 0;
+        p.causal = causal ? 1 : 0;
+        p.cap = a.cap;
+        p.scale_log2 = sc * 1.4426950408889634f;
+        p.chunk = pl.chunk;
+        p.n_splits = pl.n_splits;
+        cudaError_t e = launch_decode(p, tmK, tmV, a.dtype, (int)a.d_qk, (int)a.d_v, pl.mt, st);
+        if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+        return FA_OK;
+    }
+
+    // prefill / chunked path: rotate + append, then attention over the cache
+    void *q_att = q->data;
+    Strides3 q_att_s = s3(a.q);
+    if (a.has_new || pl.rotate_q_to_ws) {
+        RopeAppendParams p{};
+        p.status = status;
+        p.k_new = a.has_new ? k_new->data : nullptr;
+        p.kn = a.has_new ? s3(a.kn) : Strides3{0, 0, 0};
+        p.v_new = a.has_new ? v_new->data : nullptr;
+        p.vn = a.has_new ? s3(a.vn) : Strides3{0, 0, 0};
+        p.k_cache = k_cache->data;
+        p.kc = s3(a.kc);
+        p.v_cache = v_cache->data;
+        p.vc = s3(a.vc);
+        p.q = q->data;
+        p.qs = s3(a.q);
+        p.q_rot = pl.rotate_q_to_ws ? workspace : nullptr;
+        p.cos = a.r ? cos->data : nullptr;
+        p.sin = a.r ? sin->data : nullptr;
+        p.cs_row = cs_row;
+        p.cs_rows = a.s_ro;
+        p.seqlens = cache_seqlens;
+        p.seqlen_scalar = cache_seqlens_scalar;
+        p.b = (int)a.b;
+        p.s_q = (int)a.s_q;
+        p.s_new = (int)a.s_new;
+        p.h_q = (int)a.h_q;
+        p.h_kv = (int)a.h_kv;
+        p.d_qk = (int)a.d_qk;
+        p.d_v = (int)a.d_v;
+        p.r = a.r;
+        p.interleaved = interleaved ? 1 : 0;
+        p.cap = a.cap;
+        cudaError_t e = launch_rope_append(p, a.dtype, st);
+        if (e != cudaSuccess) return cuda_fail(e, "rope/append launch");
+        if (pl.rotate_q_to_ws) {
+            q_att = workspace;
+            q_att_s = Strides3{a.s_q * a.h_q * a.d_qk, a.h_q * a.d_qk, a.d_qk};
+        }
+    }
+    SimtAttnParams p{};
+    p.status = status;
+    p.q = q_att;
+    p.qs = q_att_s;
+    p.k = k_cache->data;
+    p.ks = s3(a.kc);
+    p.v = v_cache->data;
+    p.vs = s3(a.vc);
+    p.out = out->data;
+    p.os = s3(od);
+    p.lse = lse;
+    p.seqlens = cache_seqlens;
+    p.seqlen_scalar = cache_seqlens_scalar;
+    p.s_new = (int)a.s_new;
+    p.s_k = 0;
+    p.cap = a.cap;
+    p.b = (int)a.b;
+    p.s_q = (int)a.s_q;
+    p.h_q = (int)a.h_q;
+    p.h_kv = (int)a.h_kv;
+    p.g = (int)(a.h_q / a.h_kv);
+    p.d_qk = (int)a.d_qk;
+    p.d_v = (int)a.d_v;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = sc * 1.4426950408889634f;
+    cudaError_t e = launch_simt_attn(p, a.dtype, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    return FA_OK;
+}
+
+int fa_fwd_workspace_size(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, size_t *bytes) {
+    g_last_error[0] = 0;
+    if (!bytes) return fail(FA_ERR_INVALID_ARG, "bytes is NULL");
+    (void)q;
+    (void)k;
+    (void)v;
+    *bytes = 0;
+    return FA_OK;
+}
+
+int fa_fwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, int32_t causal, float scale,
+           const fa_tensor *out, float *lse, void *workspace, size_t workspace_bytes, void *stream) {
+    g_last_error[0] = 0;
+    (void)workspace;
+    (void)workspace_bytes;
+    Dims4 qd, kd, vd, od;
+    int rc;
+    if ((rc = check_tensor(q, "q", 4, 0, &qd))) return rc;
+    if ((rc = check_tensor(k, "k", 4, q->dtype, &kd))) return rc;
+    if ((rc = check_tensor(v, "v", 4, q->dtype, &vd))) return rc;
+    if ((rc = check_tensor(out, "out", 4, q->dtype, &od))) return rc;
+    const int64_t b = qd.n[0], s_q = qd.n[1], h_q = qd.n[2], d_qk = qd.n[3];
+    const int64_t s_k = kd.n[1], h_kv = kd.n[2], d_v = vd.n[3];
+    if (kd.n[0] != b || vd.n[0] != b) return fail(FA_ERR_INVALID_ARG, "k/v batch differs from q");
+    if (kd.n[3] != d_qk) return fail(FA_ERR_INVALID_ARG, "k head dim differs from q");
+    if (vd.n[1] != s_k || vd.n[2] != h_kv) return fail(FA_ERR_INVALID_ARG, "v shape differs from k");
+    if (h_kv <= 0 || h_q % h_kv) return fail(FA_ERR_INVALID_ARG, "h_q must be a multiple of h_kv");
+    if (!head_dim_ok(d_qk) || !head_dim_ok(d_v))
+        return fail(FA_ERR_UNSUPPORTED, "head dims must be multiples of 8 in 8..256");
+    if (od.n[0] != b || od.n[1] != s_q || od.n[2] != h_q || od.n[3] != d_v)
+        return fail(FA_ERR_INVALID_ARG, "out shape must be [b, s_q, h_q, d_v]");
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) return fail(FA_ERR_LAYOUT, "lse not 4-byte aligned");
+    if (b == 0 || s_q == 0 || h_q == 0) return FA_OK;
+    int32_t *status = status_word();
+    if (!status) return fail(FA_ERR_CUDA, "no CUDA device");
+    const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)d_qk);
+    SimtAttnParams p{};
+    p.status = status;
+    p.q = q->data;
+    p.qs = s3(qd);
+    p.k = k->data;
+    p.ks = s3(kd);
+    p.v = v->data;
+    p.vs = s3(vd);
+    p.out = out->data;
+    p.os = s3(od);
+    p.lse = lse;
+    p.seqlens = nullptr;
+    p.s_k = s_k;
+    p.cap = 0;
+    p.b = (int)b;
+    p.s_q = (int)s_q;
+    p.h_q = (int)h_q;
+    p.h_kv = (int)h_kv;
+    p.g = (int)(h_q / h_kv);
+    p.d_qk = (int)d_qk;
+    p.d_v = (int)d_v;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = sc * 1.4426950408889634f;
+    cudaError_t e = launch_simt_attn(p, q->dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    return FA_OK;
+}
+
+int fa_device_status(void *stream, int32_t *status) {
+    g_last_error[0] = 0;
+    if (!status) return fail(FA_ERR_INVALID_ARG, "status is NULL");
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int32_t v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, g_status_word, sizeof(v));
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
+    e = cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device status");
+    *status = v;
+    return FA_OK;
+}
+
+}  // extern "C"

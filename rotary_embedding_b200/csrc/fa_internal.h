@@ -1,0 +1,99 @@
+// fa_internal.h -- parameter blocks and launchers shared between the host
+// planner (fa_api.cu) and the kernels.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fa.h"
+
+namespace fa {
+
+// Strides of a [batch, seq, heads, dim] tensor in elements (dim stride is 1).
+struct Strides3 {
+    int64_t b, s, h;
+};
+
+// Rotary + append (+ optional rotated copy of q) for the prefill path.
+struct RopeAppendParams {
+    int32_t *status;  // device status word (see fa_device_status)
+    const void *k_new;
+    Strides3 kn;
+    const void *v_new;
+    Strides3 vn;
+    void *k_cache;
+    Strides3 kc;
+    void *v_cache;
+    Strides3 vc;
+    const void *q;
+    Strides3 qs;
+    void *q_rot;  // contiguous [b, s_q, h_q, d_qk]; nullptr = do not rotate q
+    const void *cos, *sin;
+    int64_t cs_row;   // row stride of cos/sin in elements
+    int64_t cs_rows;  // rows of cos/sin
+    const int32_t *seqlens;
+    int32_t seqlen_scalar;
+    int b, s_q, s_new, h_q, h_kv, d_qk, d_v, r, interleaved;
+    int64_t cap;
+};
+
+// Split-KV decode with fused RoPE/append (s_q * h_q / h_kv <= 32 query rows
+// per kv head).
+struct DecodeParams {
+    int32_t *status;  // device status word (see fa_device_status)
+    const void *q;
+    Strides3 qs;
+    const void *k_new;
+    Strides3 kn;
+    const void *v_new;
+    Strides3 vn;
+    void *k_cache;
+    Strides3 kc;
+    void *v_cache;
+    Strides3 vc;
+    const void *cos, *sin;
+    int64_t cs_row, cs_rows;
+    const int32_t *seqlens;
+    int32_t seqlen_scalar;
+    void *out;
+    Strides3 os;
+    float *lse;      // [b, h_q, s_q] or nullptr
+    float *o_part;   // [n_splits, b, h_q, s_q, d_v]
+    float *lse_part; // [n_splits, b, h_q, s_q]
+    int b, s_q, s_new, h_q, h_kv, g, r, interleaved, causal;
+    int64_t cap;
+    float scale_log2;
+    int chunk;     // key rows per split, multiple of 64
+    int n_splits;  // splits per (batch, kv head) = grid.x
+};
+
+// Generic attention (any supported head dim): keys from k/v (dense) or
+// from the cache after the append kernel ran.
+struct SimtAttnParams {
+    int32_t *status;  // device status word (see fa_device_status)
+    const void *q;
+    Strides3 qs;
+    const void *k;
+    Strides3 ks;
+    const void *v;
+    Strides3 vs;
+    void *out;
+    Strides3 os;
+    float *lse;
+    const int32_t *seqlens;  // kvcache mode: N_b = seqlens[b] + s_new; nullptr = dense
+    int32_t seqlen_scalar;
+    int s_new;
+    int64_t s_k;   // dense mode key rows
+    int64_t cap;   // kvcache mode capacity (precondition check)
+    int b, s_q, h_q, h_kv, g, d_qk, d_v, causal;
+    float scale_log2;
+};
+
+cudaError_t launch_rope_append(const RopeAppendParams &p, int dtype, cudaStream_t st);
+cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                          int dtype, int d_qk, int d_v, int mt, cudaStream_t st);
+bool decode_supported(int d_qk, int d_v, int mt);
+cudaError_t launch_simt_attn(const SimtAttnParams &p, int dtype, cudaStream_t st);
+
+}  // namespace fa
