@@ -55,6 +55,7 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU time budget of the oracle sample (cpu_baseline / reference arm)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     return ap.parse_args(argv)
 
 
@@ -298,13 +299,15 @@ def run_ours(args):
     ms_max = float(t.item())
     value = world * amount / (ms_max / 1e3)
 
-    e2e_times, h2d, d2h = time_e2e(w, inp, inp_dev, lambda: make_step(w, inp_dev, fa), args.steps,
-                                   max(args.warmup, 3), stream, flush_buf, barrier)
-    e_ms = sum(e2e_times) / len(e2e_times)
-    t = torch.tensor([e_ms], device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_value = world * amount / (float(t.item()) / 1e3)
+    e2e_value, h2d, d2h = None, 0, 0
+    if not args.no_e2e:
+        e2e_times, h2d, d2h = time_e2e(w, inp, inp_dev, lambda: make_step(w, inp_dev, fa), args.steps,
+                                       max(args.warmup, 3), stream, flush_buf, barrier)
+        e_ms = sum(e2e_times) / len(e2e_times)
+        t = torch.tensor([e_ms], device=device)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_value = round(world * amount / (float(t.item()) / 1e3), 3)
 
     peaks, peaks_src = load_peaks()
     if bound == "hbm":
@@ -340,7 +343,7 @@ def run_ours(args):
                      "kernel": ("decode_kernel (+combine_kernel in the same timed call)"
                                 if kernel_tag == "decode" else "whole call"),
                      "amount_per_launch": amount},
-        "e2e": {"value": round(e2e_value, 3), "unit": unit, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": int(plan["launches"]) * args.steps,
     }

@@ -64,7 +64,8 @@ struct Dims4 {
     int64_t s[4];
 };
 
-int check_tensor(const fa_tensor *t, const char *name, int ndim, int dtype, Dims4 *out) {
+int check_tensor(const fa_tensor *t, const char *name, int ndim, int dtype, Dims4 *out,
+                 bool vector_rows = true) {
     if (!t) return fail(FA_ERR_INVALID_ARG, "%s is NULL", name);
     if (!t->data) return fail(FA_ERR_INVALID_ARG, "%s->data is NULL", name);
     if (t->ndim != ndim) return fail(FA_ERR_INVALID_ARG, "%s must have %d dims (got %d)", name, ndim, t->ndim);
@@ -76,11 +77,20 @@ int check_tensor(const fa_tensor *t, const char *name, int ndim, int dtype, Dims
         if (t->shape[k] < 0) return fail(FA_ERR_INVALID_ARG, "%s: negative size", name);
     if (t->stride[ndim - 1] != 1 && t->shape[ndim - 1] > 1)
         return fail(FA_ERR_LAYOUT, "%s: innermost stride must be 1", name);
-    if ((reinterpret_cast<uintptr_t>(t->data) & 15) != 0)
-        return fail(FA_ERR_LAYOUT, "%s: base address not 16-byte aligned", name);
-    for (int k = 0; k < ndim - 1; ++k)
-        if (t->shape[k] > 1 && ((t->stride[k] * 2) % 16 != 0 || t->stride[k] <= 0))
-            return fail(FA_ERR_LAYOUT, "%s: stride of dim %d not a positive multiple of 16 bytes", name, k);
+    if (vector_rows) {
+        if ((reinterpret_cast<uintptr_t>(t->data) & 15) != 0)
+            return fail(FA_ERR_LAYOUT, "%s: base address not 16-byte aligned", name);
+        for (int k = 0; k < ndim - 1; ++k)
+            if (t->shape[k] > 1 && ((t->stride[k] * 2) % 16 != 0 || t->stride[k] <= 0))
+                return fail(FA_ERR_LAYOUT, "%s: stride of dim %d not a positive multiple of 16 bytes", name, k);
+    } else {
+        // read element by element: 2-byte alignment and positive strides suffice
+        if ((reinterpret_cast<uintptr_t>(t->data) & 1) != 0)
+            return fail(FA_ERR_LAYOUT, "%s: base address not 2-byte aligned", name);
+        for (int k = 0; k < ndim - 1; ++k)
+            if (t->shape[k] > 1 && t->stride[k] <= 0)
+                return fail(FA_ERR_LAYOUT, "%s: stride of dim %d must be positive", name, k);
+    }
     if (out) {
         for (int k = 0; k < 4; ++k) {
             out->n[k] = k < ndim ? t->shape[k] : 1;
@@ -164,15 +174,10 @@ KvPlan plan_kvcache(int64_t b, int64_t s_q, int64_t h_q, int64_t h_kv, int64_t d
         cap >= 1) {
         pl.decode = true;
         pl.mt = mt;
-        // Aim for about 148 SMs x 8 splits in flight over caches that are on
-        // average half full; splits are whole 64-row tiles.
-        const int64_t units = b * h_kv;
-        int64_t chunk = (cap / 2 * units + 148 * 8 - 1) / (148 * 8);
-        chunk = std::max<int64_t>(64, (chunk + 63) / 64 * 64);
-        const int64_t cap_r = (cap + 63) / 64 * 64;
-        chunk = std::min(chunk, cap_r);
-        pl.chunk = (int)chunk;
-        pl.n_splits = (int)((cap + chunk - 1) / chunk);
+        // The persistent decode kernel balances 64-row items across the SMs;
+        // each item owns one partial-result slot.
+        pl.chunk = 64;
+        pl.n_splits = (int)((cap + 63) / 64);
         if (pl.n_splits > 1) {
             const size_t rows = (size_t)pl.n_splits * b * h_q * s_q;
             pl.off_lse_part = align_up(rows * d_v * sizeof(float), 256);
@@ -245,8 +250,8 @@ int validate_kvcache(const fa_tensor *q, const fa_tensor *k_cache, const fa_tens
         return fail(FA_ERR_INVALID_ARG, "cos and sin must both be given or both be NULL");
     if (cos) {
         Dims4 dc, ds;
-        if ((rc = check_tensor(cos, "cos", 2, a->dtype, &dc))) return rc;
-        if ((rc = check_tensor(sin, "sin", 2, a->dtype, &ds))) return rc;
+        if ((rc = check_tensor(cos, "cos", 2, a->dtype, &dc, false))) return rc;
+        if ((rc = check_tensor(sin, "sin", 2, a->dtype, &ds, false))) return rc;
         if (dc.n[0] != ds.n[0] || dc.n[1] != ds.n[1] || dc.s[0] != ds.s[0])
             return fail(FA_ERR_INVALID_ARG, "cos and sin must have the same shape and strides");
         if (rotary_dim < 0 || rotary_dim % 2 || rotary_dim > a->d_qk)
