@@ -135,9 +135,10 @@ def fa_kvcache_fwd(q, k_cache, v_cache, k_new=None, v_new=None, rotary_cos=None,
         out = torch.empty((b, s_q, h_q, d_v), dtype=q.dtype, device=q.device)
     if lse is None and return_lse:
         lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
-    ws_bytes = fa_kvcache_workspace_size(q, k_cache, v_cache, k_new, rotary_dim)
-    if workspace is None and ws_bytes > 0:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    if workspace is None:
+        ws_bytes = fa_kvcache_workspace_size(q, k_cache, v_cache, k_new, rotary_dim)
+        if ws_bytes > 0:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     if isinstance(cache_seqlens, torch.Tensor):
         seq_ptr, seq_scalar = ctypes.c_void_p(cache_seqlens.data_ptr()), 0
     else:
@@ -163,9 +164,10 @@ def fa_fwd(q, k, v, causal=False, softmax_scale=None, out=None, lse=None, worksp
         out = torch.empty((b, s_q, h_q, d_v), dtype=q.dtype, device=q.device)
     if lse is None and return_lse:
         lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
-    ws_bytes = fa_fwd_workspace_size(q, k, v)
-    if workspace is None and ws_bytes > 0:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    if workspace is None:
+        ws_bytes = fa_fwd_workspace_size(q, k, v)
+        if ws_bytes > 0:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     _check(lib.fa_fwd(
         _ref(describe(q)), _ref(describe(k)), _ref(describe(v)), int(bool(causal)),
         float(softmax_scale or 0.0), _ref(describe(out)),

@@ -42,7 +42,13 @@ namespace fa {
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 constexpr int kDecodeTile = 64;   // key rows per tile and per item
-constexpr int kDecodeSmemBudget = 200 * 1024;
+// CTAs per SM: two when the per-thread state is small enough (one row tile,
+// d_v <= 128), so that one CTA's piece merge overlaps the other's stream.
+template <int D_V, int MT>
+struct DecodeOcc {
+    static constexpr int CTAS = (MT == 1 && D_V <= 128) ? 2 : 1;
+    static constexpr int BUDGET = CTAS == 2 ? 100 * 1024 : 200 * 1024;
+};
 
 template <int D_QK, int D_V, int MT>
 struct DecodeCfg {
@@ -53,7 +59,7 @@ struct DecodeCfg {
     static constexpr int QROWS = MT * 16;
     static constexpr int QBYTES = ((QROWS * D_QK * 2 + 1023) / 1024) * 1024;
     static constexpr int MERGE_BYTES = ((4 * QROWS * (D_V + 2) * 4 + 1023) / 1024) * 1024;
-    static constexpr int STAGES_RAW = (kDecodeSmemBudget - QBYTES - MERGE_BYTES) / STAGE;
+    static constexpr int STAGES_RAW = (DecodeOcc<D_V, MT>::BUDGET - QBYTES - MERGE_BYTES) / STAGE;
     static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 8 ? 8 : STAGES_RAW);
     static constexpr int SMEM = 1024 + QBYTES + STAGES * STAGE + MERGE_BYTES + 2 * STAGES * 8 + 64;
     static_assert(D_QK % 16 == 0 && D_V % 16 == 0, "head dims are multiples of 16");
@@ -134,7 +140,7 @@ __device__ void cta_item_range(const DecodeParams &p, int c, int G, ItemIter &fi
 }
 
 template <typename T, int D_QK, int D_V, int MT>
-__global__ void __launch_bounds__(160, 1) decode_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                         const __grid_constant__ CUtensorMap tmV,
                                                         const DecodeParams p) {
     using C = DecodeCfg<D_QK, D_V, MT>;
@@ -479,14 +485,14 @@ __global__ void __launch_bounds__(160, 1) decode_kernel(const __grid_constant__ 
                     reinterpret_cast<uint4 *>(dst)[c] = pack8<T>(acc);
                     if (c == 0 && p.lse) p.lse[((int64_t)b * p.h_q + hq) * p.s_q + i] = lse_v;
                 } else {
-                    const int64_t part = (((int64_t)s_first * p.b + b) * p.h_q + hq) * p.s_q + i;
-                    float4 *dst = reinterpret_cast<float4 *>(p.o_part + part * D_V + c * 8);
+                    // slots of one output row are contiguous: [b][h_q][s_q][n_splits]
+                    const int64_t row_slot0 = (((int64_t)b * p.h_q + hq) * p.s_q + i) * p.n_splits;
+                    float4 *dst = reinterpret_cast<float4 *>(p.o_part + (row_slot0 + s_first) * D_V + c * 8);
                     dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
                     dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
                     if (c == 0) {
-                        p.lse_part[part] = lse_v;
-                        for (int s2 = s_first + 1; s2 <= it.s; ++s2)
-                            p.lse_part[(((int64_t)s2 * p.b + b) * p.h_q + hq) * p.s_q + i] = -INFINITY;
+                        p.lse_part[row_slot0 + s_first] = lse_v;
+                        for (int s2 = s_first + 1; s2 <= it.s; ++s2) p.lse_part[row_slot0 + s2] = -INFINITY;
                     }
                 }
             }
@@ -509,9 +515,18 @@ __global__ void __launch_bounds__(256) combine_kernel(const DecodeParams p, int 
     const SegInfo sg = seg_info(p, b);
     const int n = sg.n_items;
     if (n <= 1) return;
-    auto part = [&](int s) { return (((int64_t)s * p.b + b) * p.h_q + hq) * p.s_q + i; };
+    // the row's slots are contiguous: read their lse values coalesced, keep
+    // them in registers (lane l holds slots l, l + 32, ...)
+    const int64_t row_slot0 = (((int64_t)b * p.h_q + hq) * p.s_q + i) * p.n_splits;
+    constexpr int MAXS = 16;  // up to 512 slots per row
+    float ls[MAXS];
     float mx = -INFINITY;
-    for (int s = lane; s < n; s += 32) mx = fmaxf(mx, p.lse_part[part(s)]);
+#pragma unroll
+    for (int k = 0; k < MAXS; ++k) {
+        const int s = lane + 32 * k;
+        ls[k] = s < n ? p.lse_part[row_slot0 + s] : -INFINITY;
+        mx = fmaxf(mx, ls[k]);
+    }
 #pragma unroll
     for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     T *dst = static_cast<T *>(p.out) + b * p.os.b + i * p.os.s + hq * p.os.h;
@@ -521,25 +536,31 @@ __global__ void __launch_bounds__(256) combine_kernel(const DecodeParams p, int 
         return;
     }
     float sum = 0.f;
-    for (int s = lane; s < n; s += 32) sum += ex2((p.lse_part[part(s)] - mx) * kLog2e);
+#pragma unroll
+    for (int k = 0; k < MAXS; ++k) sum += ex2((ls[k] - mx) * kLog2e);
 #pragma unroll
     for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float lse = mx + logf(sum);
     float a[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) a[e] = 0.f;
-    for (int s = 0; s < n; ++s) {
-        const float ls = p.lse_part[part(s)];
-        if (ls == -INFINITY) continue;
-        const float wgt = ex2((ls - lse) * kLog2e);
-        const float *src = p.o_part + part(s) * d_v;
+    // only the first slot of every piece holds an output; visit those
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int c = lane * 2 + e * 64;
-            if (c < d_v) {
-                const float2 v = *reinterpret_cast<const float2 *>(src + c);
-                a[2 * e] = fmaf(wgt, v.x, a[2 * e]);
-                a[2 * e + 1] = fmaf(wgt, v.y, a[2 * e + 1]);
+    for (int k = 0; k < MAXS; ++k) {
+        unsigned live = __ballot_sync(0xffffffffu, ls[k] != -INFINITY);
+        while (live) {
+            const int src_lane = __ffs(live) - 1;
+            live &= live - 1;
+            const float wgt = ex2((__shfl_sync(0xffffffffu, ls[k], src_lane) - lse) * kLog2e);
+            const float *src = p.o_part + (row_slot0 + src_lane + 32 * k) * d_v;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int c = lane * 2 + e * 64;
+                if (c < d_v) {
+                    const float2 v = *reinterpret_cast<const float2 *>(src + c);
+                    a[2 * e] = fmaf(wgt, v.x, a[2 * e]);
+                    a[2 * e + 1] = fmaf(wgt, v.y, a[2 * e + 1]);
+                }
             }
         }
     }
@@ -569,7 +590,7 @@ static cudaError_t run_decode(const DecodeParams &p, const CUtensorMap &tmK, con
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D_QK, D_V, MT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    decode_kernel<T, D_QK, D_V, MT><<<sm_count(), 160, C::SMEM, st>>>(tmK, tmV, p);
+    decode_kernel<T, D_QK, D_V, MT><<<sm_count() * DecodeOcc<D_V, MT>::CTAS, 160, C::SMEM, st>>>(tmK, tmV, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.n_splits > 1) {

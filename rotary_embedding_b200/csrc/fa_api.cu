@@ -67,8 +67,10 @@ struct Dims4 {
 int check_tensor(const fa_tensor *t, const char *name, int ndim, int dtype, Dims4 *out,
                  bool vector_rows = true) {
     if (!t) return fail(FA_ERR_INVALID_ARG, "%s is NULL", name);
-    if (!t->data) return fail(FA_ERR_INVALID_ARG, "%s->data is NULL", name);
     if (t->ndim != ndim) return fail(FA_ERR_INVALID_ARG, "%s must have %d dims (got %d)", name, ndim, t->ndim);
+    bool empty = false;
+    for (int k = 0; k < ndim; ++k) empty = empty || t->shape[k] == 0;
+    if (!t->data && !empty) return fail(FA_ERR_INVALID_ARG, "%s->data is NULL", name);
     if (t->dtype != FA_DTYPE_F16 && t->dtype != FA_DTYPE_BF16)
         return fail(FA_ERR_UNSUPPORTED, "%s: dtype %d is not fp16/bf16", name, t->dtype);
     if (dtype && t->dtype != dtype)
@@ -124,9 +126,9 @@ EncodeTiledFn encode_fn() {
 }
 
 // 4-D map over a [batch, rows, heads, dim] tensor, dims ordered (dim, heads,
-// rows, batch); box = (min(d, 64), 1, box_rows, 1) with the swizzle that
+// rows, batch); box = (min(d, 64), box_h, box_rows, 1) with the swizzle that
 // matches the box row width.
-int make_rows_map(CUtensorMap *map, const fa_tensor *t, int box_rows, const char *name) {
+int make_rows_map(CUtensorMap *map, const fa_tensor *t, int box_rows, const char *name, int box_h = 1) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     const int64_t d = t->shape[3];
@@ -138,7 +140,7 @@ int make_rows_map(CUtensorMap *map, const fa_tensor *t, int box_rows, const char
     int64_t sb = t->shape[0] > 1 ? t->stride[0] : ss * t->shape[1];
     cuuint64_t strides[3] = {(cuuint64_t)(sh * 2), (cuuint64_t)(ss * 2), (cuuint64_t)(sb * 2)};
     const int bc = d < 64 ? (int)d : 64;
-    cuuint32_t box[4] = {(cuuint32_t)bc, 1, (cuuint32_t)box_rows, 1};
+    cuuint32_t box[4] = {(cuuint32_t)bc, (cuuint32_t)box_h, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUtensorMapSwizzle sw = bc * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                           : bc * 2 == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -164,14 +166,55 @@ struct KvPlan {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Launch the tcgen05 attention kernel over q (any [b, s_q, h_q, d_qk] view),
+// k/v (dense [b, s_k, h_kv, d] or the caches).  Grouped heads are packed into
+// the 128-row tile when g divides 128.
+int run_tc_attention(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, const fa_tensor *out,
+                     float *lse, bool kvcache, const int32_t *seqlens, int32_t seqlen_scalar, int64_t s_new,
+                     int64_t cap, int causal, float scale_log2, int32_t *status, cudaStream_t st) {
+    const int64_t b = q->shape[0], s_q = q->shape[1], h_q = q->shape[2], d_qk = q->shape[3];
+    const int64_t h_kv = k->shape[2], d_v = v->shape[3];
+    const int64_t g = h_q / h_kv;
+    const int pack = (128 % g == 0) ? (int)g : 1;
+    CUtensorMap tmQ, tmK, tmV;
+    int rc;
+    if ((rc = make_rows_map(&tmQ, q, 128 / pack, "q", pack))) return rc;
+    if ((rc = make_rows_map(&tmK, k, 128, "k"))) return rc;
+    if ((rc = make_rows_map(&tmV, v, 128, "v"))) return rc;
+    PrefillParams p{};
+    p.status = status;
+    p.out = out->data;
+    p.os = Strides3{out->stride[0], out->stride[1], out->stride[2]};
+    p.lse = lse;
+    p.seqlens = seqlens;
+    p.seqlen_scalar = seqlen_scalar;
+    p.s_new = (int)s_new;
+    p.s_k = kvcache ? 0 : k->shape[1];
+    p.cap = cap;
+    p.kvcache = kvcache ? 1 : 0;
+    p.b = (int)b;
+    p.s_q = (int)s_q;
+    p.h_q = (int)h_q;
+    p.h_kv = (int)h_kv;
+    p.g = (int)g;
+    p.pack = pack;
+    p.causal = causal ? 1 : 0;
+    p.n_q_tiles = (int)((s_q * pack + 127) / 128);
+    p.scale_log2 = scale_log2;
+    cudaError_t e = launch_prefill(p, tmQ, tmK, tmV, q->dtype, (int)d_qk, (int)d_v, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tcgen05 attention launch");
+    return FA_OK;
+}
+
 KvPlan plan_kvcache(int64_t b, int64_t s_q, int64_t h_q, int64_t h_kv, int64_t d_qk, int64_t d_v,
                     int64_t cap, int64_t s_new, bool rotary) {
     KvPlan pl;
     const int64_t g = h_q / h_kv;
     const int64_t M = g * s_q;
     const int mt = M <= 16 ? 1 : 2;
+    // the combine holds up to 512 split slots per output row in registers
     if (s_q <= 8 && M <= 32 && (s_new == 0 || s_new == s_q) && decode_supported((int)d_qk, (int)d_v, mt) &&
-        cap >= 1) {
+        cap >= 1 && cap <= 512 * 64) {
         pl.decode = true;
         pl.mt = mt;
         // The persistent decode kernel balances 64-row items across the SMs;
@@ -464,6 +507,16 @@ int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor
             q_att_s = Strides3{a.s_q * a.h_q * a.d_qk, a.h_q * a.d_qk, a.d_qk};
         }
     }
+    if (prefill_supported((int)a.d_qk, (int)a.d_v)) {
+        fa_tensor qd = *q;
+        qd.data = q_att;
+        qd.stride[0] = q_att_s.b;
+        qd.stride[1] = q_att_s.s;
+        qd.stride[2] = q_att_s.h;
+        qd.stride[3] = 1;
+        return run_tc_attention(&qd, k_cache, v_cache, out, lse, true, cache_seqlens, cache_seqlens_scalar,
+                                a.s_new, a.cap, causal, sc * 1.4426950408889634f, status, st);
+    }
     SimtAttnParams p{};
     p.status = status;
     p.q = q_att;
@@ -530,6 +583,9 @@ int fa_fwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, int32_t c
     int32_t *status = status_word();
     if (!status) return fail(FA_ERR_CUDA, "no CUDA device");
     const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)d_qk);
+    if (prefill_supported((int)d_qk, (int)d_v))
+        return run_tc_attention(q, k, v, out, lse, false, nullptr, 0, 0, 0, causal, sc * 1.4426950408889634f,
+                                status, static_cast<cudaStream_t>(stream));
     SimtAttnParams p{};
     p.status = status;
     p.q = q->data;

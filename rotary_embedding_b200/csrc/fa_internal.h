@@ -90,7 +90,25 @@ struct SimtAttnParams {
     float scale_log2;
 };
 
+// tcgen05 prefill / dense attention over Q, K, V described by TMA maps.
+struct PrefillParams {
+    int32_t *status;
+    void *out;
+    Strides3 os;
+    float *lse;
+    const int32_t *seqlens;  // kvcache mode: N_b = seqlens[b] + s_new
+    int32_t seqlen_scalar;
+    int s_new;
+    int64_t s_k;   // dense mode key rows
+    int64_t cap;   // kvcache mode capacity (precondition check)
+    int kvcache, b, s_q, h_q, h_kv, g, pack, causal, n_q_tiles;
+    float scale_log2;
+};
+
 cudaError_t launch_rope_append(const RopeAppendParams &p, int dtype, cudaStream_t st);
+bool prefill_supported(int d_qk, int d_v);
+cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &tmQ, const CUtensorMap &tmK,
+                           const CUtensorMap &tmV, int dtype, int d_qk, int d_v, cudaStream_t st);
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
                           int dtype, int d_qk, int d_v, int mt, cudaStream_t st);
 bool decode_supported(int d_qk, int d_v, int mt);

@@ -1,0 +1,382 @@
+// prefill_sm100.cu -- prefill / chunked-prefill / dense attention forward on
+// the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// One CTA computes a 128-row query tile against every key tile it may see:
+//   out = softmax(scale * Q K^T + mask) V  with the online (rescaled) softmax
+// of the "optimizing-attention-flash" page (IO-aware tiling, no S in HBM).
+//
+// Roles (warp specialisation, 8 warps):
+//   warp 0      TMA producer: the Q tile once, then K_j / V_j 128-row tiles
+//               into a ring of shared-memory stages (128-byte swizzled boxes).
+//   warp 1      TMEM allocator and MMA issuer (one thread): S_j = Q K_j^T into
+//               one of two TMEM S buffers, then O += P_{j-1} V_{j-1} with P
+//               read from TMEM; order S_0, S_1, PV_0, S_2, PV_1, ... so the
+//               tensor core works on S_{j+1} while the softmax runs on S_j.
+//   warps 4-7   softmax warpgroup: thread t owns query row t of the tile
+//               (TMEM lane t).  Loads its S row, applies the bottom-right
+//               causal / sequence-end mask, keeps the running max (rescaling
+//               O in TMEM only when the max grows by more than 2^8), writes
+//               P = 2^(s*scale*log2e - m) as 16-bit values into TMEM, and at
+//               the end normalises O and writes out and lse.
+// Tiles are sized separately for d_qk (Q/K boxes) and d_v (V/O), so a
+// 192/128 head (flash-attention PR #1604) pays for neither padding.
+// Grouped-query heads (the page's Workflow 2 Step 3) are packed: when
+// g = h_q / h_kv divides 128, the tile's rows are (query position, head)
+// pairs of one kv head, loaded by one TMA box, so K/V tiles are shared by
+// the g heads.
+#include <algorithm>
+#include <type_traits>
+
+#include "fa_common.cuh"
+#include "fa_internal.h"
+#include "tcgen05.cuh"
+
+namespace fa {
+
+constexpr int kBM = 128;  // query rows per CTA
+constexpr int kBN = 128;  // key rows per tile
+
+template <int D_QK, int D_V>
+struct PrefillCfg {
+    static constexpr int QBYTES = kBM * D_QK * 2;
+    static constexpr int KBYTES = kBN * D_QK * 2;
+    static constexpr int VBYTES = kBN * D_V * 2;
+    static constexpr int QBOX = kBM * 128;   // bytes of one 64-column box of Q
+    static constexpr int KBOX = kBN * 128;
+    static constexpr int VBOX = kBN * 128;
+    static constexpr int BUDGET = 224 * 1024;
+    static constexpr int KST_RAW = (BUDGET - QBYTES) / (KBYTES + VBYTES);
+    static constexpr int KST = KST_RAW > 4 ? 4 : KST_RAW;
+    static constexpr int SMEM = 1024 + QBYTES + KST * (KBYTES + VBYTES) + 256;
+    // TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D_V), P [384, 448)
+    static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O = 256, T_P = 384;
+    static_assert(KST >= 2, "at least two K/V stages");
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+    static_assert(D_QK % 64 == 0 && D_V % 64 == 0 && D_V <= 128, "head dims");
+};
+
+template <typename T, int D_QK, int D_V>
+__global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                         const __grid_constant__ CUtensorMap tmK,
+                                                         const __grid_constant__ CUtensorMap tmV,
+                                                         const PrefillParams p) {
+    using C = PrefillCfg<D_QK, D_V>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem;
+    uint8_t *sK = sQ + C::QBYTES;                 // KST stages of K
+    uint8_t *sV = sK + C::KST * C::KBYTES;        // KST stages of V
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sV + C::KST * C::VBYTES);
+    uint64_t *q_full = bars;                      // 1
+    uint64_t *k_full = bars + 1;                  // KST
+    uint64_t *v_full = k_full + C::KST;           // KST
+    uint64_t *kv_empty = v_full + C::KST;         // KST
+    uint64_t *s_full = kv_empty + C::KST;         // 2
+    uint64_t *s_free = s_full + 2;                // 2
+    uint64_t *p_full = s_free + 2;                // 1
+    uint64_t *pv_done = p_full + 1;               // 1
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pv_done + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qt = (int)gridDim.x - 1 - (int)blockIdx.x;   // heaviest causal tiles first
+    const int hgrp = blockIdx.y, b = blockIdx.z;
+    const int pack = p.pack;
+    const int hq0 = hgrp * pack;                           // first query head of the tile
+    const int hk = hq0 / p.g;
+    const int i0 = qt * (kBM / pack);                      // first query position
+    const int i_last = min(p.s_q, i0 + kBM / pack) - 1;
+
+    int N;
+    if (p.kvcache) {
+        const int L = seqlen_of(p.seqlens, p.seqlen_scalar, b);
+        if (L < 0 || (int64_t)L + p.s_new > p.cap) {
+            if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
+            return;
+        }
+        N = L + p.s_new;
+    } else {
+        N = (int)p.s_k;
+    }
+    const int kv_end = p.causal ? max(0, min(N, i_last + N - p.s_q + 1)) : N;
+    const int n_kv = (kv_end + kBN - 1) / kBN;
+    // first key index that needs an element mask (diagonal band or sequence end)
+    const int mask_from = p.causal ? max(0, min(N, i0 + N - p.s_q + 1)) : N;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < C::KST; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_free[s], 4);
+        }
+        mbar_init(p_full, 4);
+        mbar_init(pv_done, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0 && n_kv > 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            mbar_arrive_expect_tx(q_full, C::QBYTES);
+#pragma unroll
+            for (int c = 0; c < D_QK / 64; ++c) tma_load_4d(sQ + c * C::QBOX, &tmQ, q_full, c * 64, hq0, i0, b);
+            for (int j = 0; j < n_kv; ++j) {
+                const int st = j % C::KST;
+                if (j >= C::KST && !mbar_wait(&kv_empty[st], ((j / C::KST) - 1) & 1, p.status)) break;
+                mbar_arrive_expect_tx(&k_full[st], C::KBYTES);
+#pragma unroll
+                for (int c = 0; c < D_QK / 64; ++c)
+                    tma_load_4d(sK + st * C::KBYTES + c * C::KBOX, &tmK, &k_full[st], c * 64, hk, j * kBN, b);
+                mbar_arrive_expect_tx(&v_full[st], C::VBYTES);
+#pragma unroll
+                for (int c = 0; c < D_V / 64; ++c)
+                    tma_load_4d(sV + st * C::VBYTES + c * C::VBOX, &tmV, &v_full[st], c * 64, hk, j * kBN, b);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0 && n_kv > 0) {
+            const uint32_t idesc_qk = tc::idesc_f16(bf16, kBM, kBN, false);
+            const uint32_t idesc_pv = tc::idesc_f16(bf16, kBM, D_V, true);
+            const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
+            bool ok = mbar_wait(q_full, 0, p.status);
+            auto issue_pv = [&](int jj) -> bool {
+                const int st = jj % C::KST;
+                if (!mbar_wait(p_full, jj & 1, p.status)) return false;
+                if (!mbar_wait(&v_full[st], (jj / C::KST) & 1, p.status)) return false;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int k = 0; k < kBN / 16; ++k) {
+                    const uint64_t bdesc = tc::smem_desc(aV + st * C::VBYTES + k * 16 * 128, C::VBOX, 1024);
+                    tc::mma_ts(tmem + C::T_O, tmem + C::T_P + k * 8, bdesc, idesc_pv, (jj > 0 || k > 0) ? 1u : 0u);
+                }
+                tc::commit(&kv_empty[st]);
+                tc::commit(pv_done);
+                return true;
+            };
+            for (int j = 0; j < n_kv && ok; ++j) {
+                const int st = j % C::KST, sb = j & 1;
+                if (!mbar_wait(&k_full[st], (j / C::KST) & 1, p.status)) break;
+                if (j >= 2 && !mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1, p.status)) break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int k = 0; k < D_QK / 16; ++k) {
+                    const uint64_t adesc = tc::smem_desc(aQ + (k >> 2) * C::QBOX + (k & 3) * 32, 16, 1024);
+                    const uint64_t bdesc =
+                        tc::smem_desc(aK + st * C::KBYTES + (k >> 2) * C::KBOX + (k & 3) * 32, 16, 1024);
+                    tc::mma_ss(tmem + (sb ? C::T_S1 : C::T_S0), adesc, bdesc, idesc_qk, k > 0 ? 1u : 0u);
+                }
+                tc::commit(&s_full[sb]);
+                if (j >= 1 && !issue_pv(j - 1)) {
+                    ok = false;
+                    break;
+                }
+            }
+            if (ok) issue_pv(n_kv - 1);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------ softmax warpgroup
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;                  // tile row = TMEM lane
+        const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+        const int prow = qt * kBM + r;                 // packed row
+        const int i = prow / pack;                     // query position
+        const int hq = hq0 + (prow % pack);
+        const bool row_valid = i < p.s_q;
+        const int last_vis = row_valid ? (p.causal ? min(N - 1, i + N - p.s_q) : N - 1) : -1;
+        const float c = p.scale_log2;
+        float m_ref = -INFINITY;   // raw-score max used as the exponent reference
+        float l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_kv && ok; ++j) {
+            const int sb = j & 1;
+            if (!mbar_wait(&s_full[sb], (j >> 1) & 1, p.status)) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            uint32_t sr[4][32];
+            const uint32_t s_addr = tmem + lane_addr + (sb ? C::T_S1 : C::T_S0);
+            tc::ld32(s_addr, sr[0]);
+            tc::ld32(s_addr + 32, sr[1]);
+            tc::ld32(s_addr + 64, sr[2]);
+            tc::ld32(s_addr + 96, sr[3]);
+            tc::wait_ld();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[sb]);
+
+            const int j0 = j * kBN;
+            float mt = -INFINITY;
+            if (j0 + kBN > mask_from) {
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int key = j0 + h * 32 + e;
+                        float v = __uint_as_float(sr[h][e]);
+                        v = key <= last_vis ? v : -INFINITY;
+                        sr[h][e] = __float_as_uint(v);
+                        mt = fmaxf(mt, v);
+                    }
+            } else {
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) mt = fmaxf(mt, __uint_as_float(sr[h][e]));
+            }
+            // lazy rescale: move the reference only when the max grows by > 2^8
+            float alpha = 1.f;
+            bool rescale = false;
+            if (mt > m_ref && (m_ref == -INFINITY || (mt - m_ref) * c > 8.f)) {
+                alpha = m_ref == -INFINITY ? 0.f : ex2((m_ref - mt) * c);
+                rescale = m_ref != -INFINITY;
+                m_ref = mt;
+            }
+            const float mc = m_ref == -INFINITY ? 0.f : m_ref * c;
+            uint32_t pk[2][32];
+            float rs = 0.f;
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const float p0 = ex2(fmaf(__uint_as_float(sr[h][e]), c, -mc));
+                    const float p1 = ex2(fmaf(__uint_as_float(sr[h][e + 1]), c, -mc));
+                    rs += p0 + p1;
+                    pk[h >> 1][(h & 1) * 16 + (e >> 1)] = Elem<T>::pack2(p0, p1);
+                }
+            l = l * alpha + rs;
+
+            if (j > 0) {
+                // O is stable and the P buffer free once PV_{j-1} has completed
+                if (!mbar_wait(pv_done, (j - 1) & 1, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                    for (int h = 0; h < D_V / 32; ++h) {
+                        uint32_t orr[32];
+                        const uint32_t o_addr = tmem + lane_addr + C::T_O + h * 32;
+                        tc::ld32(o_addr, orr);
+                        tc::wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                        tc::st32(o_addr, orr);
+                    }
+                }
+            }
+            tc::st32(tmem + lane_addr + C::T_P, pk[0]);
+            tc::st32(tmem + lane_addr + C::T_P + 32, pk[1]);
+            tc::wait_st();
+            if (p.kvcache && j == n_kv - 1 && j0 + kBN > N) {
+                // cache rows past N_b may hold anything: zero them in the V tile
+                const int st = j % C::KST;
+                if (!mbar_wait(&v_full[st], (j / C::KST) & 1, p.status)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *vt = sV + st * C::VBYTES;
+                const int first = N - j0;
+                const int n16 = (kBN - first) * 8 * (D_V / 64);
+                for (int idx = threadIdx.x - 128; idx < n16; idx += 128) {
+                    const int box = idx / ((kBN - first) * 8);
+                    const int rem = idx % ((kBN - first) * 8);
+                    *reinterpret_cast<uint4 *>(vt + box * C::VBOX + (first + rem / 8) * 128 + (rem % 8) * 16) =
+                        make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async();
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        // ------------------------------------------------ epilogue
+        if (ok && n_kv > 0 && !mbar_wait(pv_done, (n_kv - 1) & 1, p.status)) ok = false;
+        tc::fence_after_sync();
+        // every lane takes part in the (warp-collective) TMEM loads; only rows
+        // inside the sequence are stored
+        T *orow = static_cast<T *>(p.out) + b * p.os.b + (int64_t)i * p.os.s + hq * p.os.h;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+        for (int h = 0; h < D_V / 32; ++h) {
+            uint32_t orr[32];
+            if (n_kv > 0) {
+                tc::ld32(tmem + lane_addr + C::T_O + h * 32, orr);
+                tc::wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) orr[e] = 0u;
+            }
+            if (row_valid) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                    float f[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(orr[e + u]) * inv;
+                    reinterpret_cast<uint4 *>(orow + h * 32 + e)[0] = pack8<T>(f);
+                }
+            }
+        }
+        if (row_valid && p.lse)
+            p.lse[((int64_t)b * p.h_q + hq) * p.s_q + i] = l > 0.f ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+template <typename T, int D_QK, int D_V>
+static cudaError_t run_prefill(const PrefillParams &p, const CUtensorMap &tmQ, const CUtensorMap &tmK,
+                               const CUtensorMap &tmV, cudaStream_t st) {
+    using C = PrefillCfg<D_QK, D_V>;
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<T, D_QK, D_V>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.n_q_tiles, p.h_q / p.pack, p.b);
+    prefill_kernel<T, D_QK, D_V><<<grid, 256, C::SMEM, st>>>(tmQ, tmK, tmV, p);
+    return cudaGetLastError();
+}
+
+#define FA_PREFILL_DIMS(X) X(64, 64) X(128, 128) X(192, 128) X(128, 64) X(64, 128) X(192, 64)
+
+bool prefill_supported(int d_qk, int d_v) {
+#define FA_CASE(DQ, DV) if (d_qk == DQ && d_v == DV) return true;
+    FA_PREFILL_DIMS(FA_CASE)
+#undef FA_CASE
+    return false;
+}
+
+cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &tmQ, const CUtensorMap &tmK,
+                           const CUtensorMap &tmV, int dtype, int d_qk, int d_v, cudaStream_t st) {
+#define FA_CASE(DQ, DV)                                                                   \
+    if (d_qk == DQ && d_v == DV) {                                                        \
+        if (dtype == FA_DTYPE_F16) return run_prefill<__half, DQ, DV>(p, tmQ, tmK, tmV, st); \
+        return run_prefill<__nv_bfloat16, DQ, DV>(p, tmQ, tmK, tmV, st);                  \
+    }
+    FA_PREFILL_DIMS(FA_CASE)
+#undef FA_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace fa

@@ -182,6 +182,46 @@ def test_dense_small(dims, causal, cuda_device):
         check_dense(w, run_gpu_dense(w, inp, cuda_device), ref)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dims", [(128, 128, "bf16", 6, 2), (192, 128, "bf16", 4, 4), (64, 64, "fp16", 8, 1),
+                                  (128, 64, "fp16", 3, 3), (64, 128, "bf16", 2, 2)])
+def test_dense_multi_tile(dims, causal, cuda_device):
+    """Several 128-row query and key tiles with ragged tails; g = 3 takes the
+    unpacked path, g = 8 and g = 1 the packed one; the K/V ring wraps."""
+    d_qk, d_v, dt, hq, hkv = dims
+    w = W.Workload(name="dense-multi", mode="dense", dtype=dt, batch=2, h_q=hq, h_kv=hkv, d_qk=d_qk,
+                   d_v=d_v, s_q=1000, s_k=1000, causal=causal)
+    inp = W.make_inputs(w, seed=11)
+    ref = oracle.fwd(inp["q"].double().numpy(), inp["k"].double().numpy(), inp["v"].double().numpy(),
+                     causal=causal, scale=w.softmax_scale())
+    check_dense(w, run_gpu_dense(w, inp, cuda_device), ref)
+
+
+@pytest.mark.parametrize("s_new", [1, 300])
+def test_kvcache_garbage_past_sequence(s_new, cuda_device):
+    """Cache rows at and past N_b hold NaN: they must not reach the result (the
+    rows are masked in the scores and zeroed before the PV product)."""
+    w = W.Workload(name="nan-tail", mode="kvcache", dtype="bf16", batch=2, h_q=8, h_kv=2, d_qk=128,
+                   d_v=128, s_q=s_new, cap=900, seqlens=(100, 500), causal=True, rotary_dim=64)
+    inp = W.make_inputs(w, seed=4)
+    for b, L in enumerate(inp["cache_seqlens"].tolist()):
+        inp["k_cache"][b, L:] = float("nan")
+        inp["v_cache"][b, L:] = float("nan")
+    gpu = run_gpu_kvcache(w, inp, cuda_device)
+    ref_inp = dict(inp)
+    ref_inp["k_cache"] = torch.nan_to_num(inp["k_cache"])
+    ref_inp["v_cache"] = torch.nan_to_num(inp["v_cache"])
+    ref = run_oracle_kvcache(w, ref_inp)
+    out, lse, kc, vc = gpu
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+    assert np.abs(out.double().numpy() - ref[0]).max() <= OUT_TOL["bf16"]
+    assert np.abs(lse.double().numpy() - ref[1]).max() <= LSE_TOL
+    # the appended rows replaced the NaN rows at L_b .. L_b + s_new - 1
+    for b, L in enumerate(inp["cache_seqlens"].tolist()):
+        assert torch.isfinite(vc[b, L:L + s_new]).all()
+        assert torch.equal(vc[b, L:L + s_new], inp["v_new"][b])
+
+
 # ------------------------------------------------------------------ full-size configurations
 def _slice_kv_inputs(inp, batches, heads=None):
     out = {}
