@@ -47,9 +47,14 @@ constexpr int kDecodeTile = 64;   // key rows per tile and per item
 template <int D_V, int MT>
 struct DecodeOcc {
     static constexpr int CTAS = (MT == 1 && D_V <= 128) ? 2 : 1;
-    static constexpr int BUDGET = CTAS == 2 ? 100 * 1024 : 200 * 1024;
+    static constexpr int BUDGET = CTAS == 2 ? 112 * 1024 : 224 * 1024;
 };
 
+constexpr int kDecodeMaxStages = 8;
+
+// Shared memory: rotated q tile | ring of K/V stages | merge scratch for the
+// M live query rows | barriers.  The stage count is chosen at launch from the
+// budget left after the (runtime-sized) merge scratch.
 template <int D_QK, int D_V, int MT>
 struct DecodeCfg {
     static constexpr int TILE = kDecodeTile;
@@ -58,12 +63,14 @@ struct DecodeCfg {
     static constexpr int STAGE = KBYTES + VBYTES;
     static constexpr int QROWS = MT * 16;
     static constexpr int QBYTES = ((QROWS * D_QK * 2 + 1023) / 1024) * 1024;
-    static constexpr int MERGE_BYTES = ((4 * QROWS * (D_V + 2) * 4 + 1023) / 1024) * 1024;
-    static constexpr int STAGES_RAW = (DecodeOcc<D_V, MT>::BUDGET - QBYTES - MERGE_BYTES) / STAGE;
-    static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 8 ? 8 : STAGES_RAW);
-    static constexpr int SMEM = 1024 + QBYTES + STAGES * STAGE + MERGE_BYTES + 2 * STAGES * 8 + 64;
+    static constexpr int TAIL = 2 * kDecodeMaxStages * 8 + 64;
     static_assert(D_QK % 16 == 0 && D_V % 16 == 0, "head dims are multiples of 16");
-    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+    static int merge_bytes(int M) { return 4 * M * (D_V + 2) * 4; }
+    static int stages(int M) {
+        const int raw = (DecodeOcc<D_V, MT>::BUDGET - 1024 - QBYTES - merge_bytes(M) - TAIL) / STAGE;
+        return raw < 2 ? 2 : (raw > kDecodeMaxStages ? kDecodeMaxStages : raw);
+    }
+    static int smem(int M) { return 1024 + QBYTES + stages(M) * STAGE + merge_bytes(M) + TAIL; }
 };
 
 // Per-batch facts every thread can recompute: rows N_b and items n_b (0 when
@@ -149,24 +156,25 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
     constexpr int CK = D_QK / 8, CV = D_V / 8;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int M = p.g * p.s_q;
+    const int NST = p.n_stages;
     uint8_t *sQ = smem;
     uint8_t *sStage = smem + C::QBYTES;
-    float *red_o = reinterpret_cast<float *>(sStage + C::STAGES * C::STAGE);
-    float *red_m = red_o + 4 * C::QROWS * D_V;
-    float *red_l = red_m + 4 * C::QROWS;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sStage + C::STAGES * C::STAGE + C::MERGE_BYTES);
-    uint64_t *empty = full + C::STAGES;
-    int *sched = reinterpret_cast<int *>(empty + C::STAGES);   // b, hk, s, n_items
+    float *red_o = reinterpret_cast<float *>(sStage + NST * C::STAGE);   // [4][M][D_V]
+    float *red_m = red_o + 4 * M * D_V;                                   // [4][M]
+    float *red_l = red_m + 4 * M;                                         // [4][M]
+    uint64_t *full = reinterpret_cast<uint64_t *>(red_l + 4 * M);
+    uint64_t *empty = full + kDecodeMaxStages;
+    int *sched = reinterpret_cast<int *>(empty + kDecodeMaxStages);   // b, hk, s, n_items
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool inter = p.interleaved != 0;
-    const int M = p.g * p.s_q;
 
     // allow the combine kernel (launched as a programmatic dependent) to get scheduled
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 4);
         }
@@ -219,8 +227,8 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
             bool ok = true;
             for (int k = 0; k < n_items && ok; ++k) {
                 const int row0 = it.s * C::TILE;
-                const int s = t % C::STAGES;
-                if (t >= C::STAGES && !mbar_wait(&empty[s], ((t / C::STAGES) - 1) & 1, p.status)) {
+                const int s = t % NST;
+                if (t >= NST && !mbar_wait(&empty[s], ((t / NST) - 1) & 1, p.status)) {
                     ok = false;
                     break;
                 }
@@ -292,8 +300,8 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
 
         // ---- one 64-row tile = one item ----
         const int t = k;
-        const int s = t % C::STAGES;
-        if (!timed_out && !mbar_wait(&full[s], (t / C::STAGES) & 1, p.status)) timed_out = true;
+        const int s = t % NST;
+        if (!timed_out && !mbar_wait(&full[s], (t / NST) & 1, p.status)) timed_out = true;
         if (!timed_out) {
             uint8_t *sK = sStage + s * C::STAGE;
             uint8_t *sV = sK + C::KBYTES;
@@ -444,14 +452,17 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
 #pragma unroll
                 for (int hr = 0; hr < 2; ++hr) {
                     const int row = mt * 16 + (lane >> 2) + hr * 8;
-                    if ((lane & 3) == 0) {
-                        red_m[warp * C::QROWS + row] = m_r[mt][hr];
-                        red_l[warp * C::QROWS + row] = l_r[mt][hr];
-                    }
-                    float *dst = red_o + (warp * C::QROWS + row) * D_V + ((lane & 3) << 1);
+                    if (row < M) {
+                        if ((lane & 3) == 0) {
+                            red_m[warp * M + row] = m_r[mt][hr];
+                            red_l[warp * M + row] = l_r[mt][hr];
+                        }
+                        float *dst = red_o + (warp * M + row) * D_V + ((lane & 3) << 1);
 #pragma unroll
-                    for (int n = 0; n < D_V / 8; ++n)
-                        *reinterpret_cast<float2 *>(dst + n * 8) = make_float2(o[mt][n][hr * 2], o[mt][n][hr * 2 + 1]);
+                        for (int n = 0; n < D_V / 8; ++n)
+                            *reinterpret_cast<float2 *>(dst + n * 8) =
+                                make_float2(o[mt][n][hr * 2], o[mt][n][hr * 2 + 1]);
+                    }
                 }
             consumer_sync();
             const bool single = it.seg.n_items == 1;
@@ -460,7 +471,7 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
                 float mw[4], mx = -INFINITY;
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
-                    mw[w] = red_m[w * C::QROWS + row];
+                    mw[w] = red_m[w * M + row];
                     mx = fmaxf(mx, mw[w]);
                 }
                 const float mu = mx == -INFINITY ? 0.f : mx;
@@ -470,8 +481,8 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
                     const float sc = ex2(mw[w] - mu);
-                    ltot += red_l[w * C::QROWS + row] * sc;
-                    const float *src = red_o + (w * C::QROWS + row) * D_V + c * 8;
+                    ltot += red_l[w * M + row] * sc;
+                    const float *src = red_o + (w * M + row) * D_V + c * 8;
 #pragma unroll
                     for (int e = 0; e < 8; ++e) acc[e] += src[e] * sc;
                 }
@@ -544,15 +555,35 @@ __global__ void __launch_bounds__(256) combine_kernel(const DecodeParams p, int 
     float a[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) a[e] = 0.f;
-    // only the first slot of every piece holds an output; visit those
+    // Only the first slot of every piece holds an output.  Compact the live
+    // slots and their weights into this warp's shared-memory list, then read
+    // their outputs with independent (overlapping) loads.
+    constexpr int LIST = 64;
+    __shared__ int live_slot[8][LIST];
+    __shared__ float live_w[8][LIST];
+    const int wib = threadIdx.x >> 5;
+    int n_total = 0;
 #pragma unroll
-    for (int k = 0; k < MAXS; ++k) {
-        unsigned live = __ballot_sync(0xffffffffu, ls[k] != -INFINITY);
-        while (live) {
-            const int src_lane = __ffs(live) - 1;
-            live &= live - 1;
-            const float wgt = ex2((__shfl_sync(0xffffffffu, ls[k], src_lane) - lse) * kLog2e);
-            const float *src = p.o_part + (row_slot0 + src_lane + 32 * k) * d_v;
+    for (int k = 0; k < MAXS; ++k) n_total += __popc(__ballot_sync(0xffffffffu, ls[k] != -INFINITY));
+    for (int base = 0; base < n_total; base += LIST) {
+        int n_live = 0;
+#pragma unroll
+        for (int k = 0; k < MAXS; ++k) {
+            const bool is_live = ls[k] != -INFINITY;
+            const unsigned live = __ballot_sync(0xffffffffu, is_live);
+            const int pos = n_live + __popc(live & ((1u << lane) - 1u)) - base;
+            if (is_live && pos >= 0 && pos < LIST) {
+                live_slot[wib][pos] = lane + 32 * k;
+                live_w[wib][pos] = ex2((ls[k] - lse) * kLog2e);
+            }
+            n_live += __popc(live);
+        }
+        __syncwarp();
+        const int cnt = min(LIST, n_total - base);
+#pragma unroll 4
+        for (int t = 0; t < cnt; ++t) {
+            const float wgt = live_w[wib][t];
+            const float *src = p.o_part + (row_slot0 + live_slot[wib][t]) * d_v;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int c = lane * 2 + e * 64;
@@ -563,6 +594,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const DecodeParams p, int 
                 }
             }
         }
+        __syncwarp();
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -584,13 +616,17 @@ int sm_count() {
 }
 
 template <typename T, int D_QK, int D_V, int MT>
-static cudaError_t run_decode(const DecodeParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
+static cudaError_t run_decode(const DecodeParams &p_in, const CUtensorMap &tmK, const CUtensorMap &tmV,
                               cudaStream_t st) {
     using C = DecodeCfg<D_QK, D_V, MT>;
+    DecodeParams p = p_in;
+    const int M = p.g * p.s_q;
+    p.n_stages = C::stages(M);
+    const int smem = C::smem(M);
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D_QK, D_V, MT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    decode_kernel<T, D_QK, D_V, MT><<<sm_count() * DecodeOcc<D_V, MT>::CTAS, 160, C::SMEM, st>>>(tmK, tmV, p);
+    decode_kernel<T, D_QK, D_V, MT><<<sm_count() * DecodeOcc<D_V, MT>::CTAS, 160, smem, st>>>(tmK, tmV, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.n_splits > 1) {

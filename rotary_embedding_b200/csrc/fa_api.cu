@@ -201,6 +201,17 @@ int run_tc_attention(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
     p.causal = causal ? 1 : 0;
     p.n_q_tiles = (int)((s_q * pack + 127) / 128);
     p.scale_log2 = scale_log2;
+    // Two query tiles per CTA keep the tensor core busy during the softmax,
+    // but halve the CTA count: use them only when the grid still fills the
+    // SMs about twice over.
+    const int64_t ctas2 = (int64_t)((p.n_q_tiles + 1) / 2) * (h_q / pack) * b;
+    p.tiles_per_cta = ctas2 >= 2 * (int64_t)sm_count() ? 2 : 1;
+    // FA_PREFILL_TILES_PER_CTA=1|2 overrides the choice (tests use it to run
+    // both kernels on small shapes)
+    if (const char *env = getenv("FA_PREFILL_TILES_PER_CTA")) {
+        if (env[0] == '1') p.tiles_per_cta = 1;
+        if (env[0] == '2') p.tiles_per_cta = 2;
+    }
     cudaError_t e = launch_prefill(p, tmQ, tmK, tmV, q->dtype, (int)d_qk, (int)d_v, st);
     if (e != cudaSuccess) return cuda_fail(e, "tcgen05 attention launch");
     return FA_OK;

@@ -65,6 +65,7 @@ struct DecodeParams {
     int64_t cap;
     float scale_log2;
     int chunk;     // key rows per split, multiple of 64
+    int n_stages;  // K/V ring depth (set by the launcher from the shared-memory budget)
     int n_splits;  // splits per (batch, kv head) = grid.x
 };
 
@@ -102,8 +103,11 @@ struct PrefillParams {
     int64_t s_k;   // dense mode key rows
     int64_t cap;   // kvcache mode capacity (precondition check)
     int kvcache, b, s_q, h_q, h_kv, g, pack, causal, n_q_tiles;
+    int tiles_per_cta;  // 1: one 128-row tile per CTA; 2: two tiles, two softmax warpgroups
     float scale_log2;
 };
+
+int sm_count();
 
 cudaError_t launch_rope_append(const RopeAppendParams &p, int dtype, cudaStream_t st);
 bool prefill_supported(int d_qk, int d_v);

@@ -346,9 +346,346 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
     }
 }
 
+// ============================================================================
+// Two query tiles per CTA (256 query rows), two softmax warpgroups.
+//
+// The tensor core alternates between the tiles: while warpgroup A turns S_A
+// into P_A, it runs PV_B(j-1) and QK_B(j), and the other way round:
+//   QK_A(0) QK_B(0) | PV_A(0) QK_A(1) | PV_B(0) QK_B(1) | PV_A(1) QK_A(2) | ...
+// Each tile has one TMEM S buffer; P is written over the first 64 columns of
+// it as 16-bit pairs and read from there as the A operand of PV.  The next
+// QK of the same tile is issued after that PV by the same thread, and the
+// tensor pipe executes one thread's MMAs in issue order, so the PV reads P
+// before the QK overwrites it.  When softmax X sees S_X(j) complete, every
+// earlier MMA of the CTA has completed too, so O_X is stable and can be
+// rescaled without a further wait.
+// Warps: 0 TMA, 1 MMA, 4-7 softmax of tile A, 8-11 softmax of tile B.
+// ============================================================================
+template <int D_QK, int D_V>
+struct Prefill2Cfg {
+    static constexpr int QBYTES = kBM * D_QK * 2;   // per tile
+    static constexpr int KBYTES = kBN * D_QK * 2;
+    static constexpr int VBYTES = kBN * D_V * 2;
+    static constexpr int BOX = 128 * 128;            // bytes of one 64-column box of 128 rows
+    static constexpr int BUDGET = 224 * 1024;
+    static constexpr int AVAIL = BUDGET - 2 * QBYTES;
+    static constexpr bool EVEN = AVAIL >= 2 * (KBYTES + VBYTES);
+    static constexpr int KS_RAW = AVAIL / (KBYTES + VBYTES);
+    static constexpr int KST = EVEN ? (KS_RAW > 3 ? 3 : KS_RAW) : 2;
+    static constexpr int VST = EVEN ? KST : (AVAIL - 2 * KBYTES) / VBYTES;
+    static constexpr int SMEM = 1024 + 2 * QBYTES + KST * KBYTES + VST * VBYTES + 256;
+    // TMEM columns: S of tile x at [128 x, 128 x + 128), O of tile x at [256 + 128 x, ...)
+    static __device__ __forceinline__ uint32_t t_s(int x) { return (uint32_t)(x * 128); }
+    static __device__ __forceinline__ uint32_t t_o(int x) { return (uint32_t)(256 + x * 128); }
+    static_assert(VST >= 1 && KST >= 2, "K/V ring");
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+    static_assert(D_QK % 64 == 0 && D_V % 64 == 0 && D_V <= 128, "head dims");
+};
+
+template <typename T, int D_QK, int D_V>
+__global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                          const __grid_constant__ CUtensorMap tmK,
+                                                          const __grid_constant__ CUtensorMap tmV,
+                                                          const PrefillParams p) {
+    using C = Prefill2Cfg<D_QK, D_V>;
+    constexpr int KST = C::KST, VST = C::VST;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem;                              // 2 tiles
+    uint8_t *sK = sQ + 2 * C::QBYTES;
+    uint8_t *sV = sK + KST * C::KBYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sV + VST * C::VBYTES);
+    uint64_t *q_full = bars;                // 1
+    uint64_t *k_full = bars + 1;            // KST
+    uint64_t *k_empty = k_full + KST;       // KST
+    uint64_t *v_full = k_empty + KST;       // VST
+    uint64_t *v_empty = v_full + VST;       // VST
+    uint64_t *s_full = v_empty + VST;       // 2
+    uint64_t *p_full = s_full + 2;          // 2
+    uint64_t *o_full = p_full + 2;          // 2
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_full + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int blk = (int)gridDim.x - 1 - (int)blockIdx.x;   // heaviest causal blocks first
+    const int hgrp = blockIdx.y, b = blockIdx.z;
+    const int pack = p.pack;
+    const int hq0 = hgrp * pack;
+    const int hk = hq0 / p.g;
+    const int rows_per_tile = kBM / pack;                   // query positions per tile
+
+    int N;
+    if (p.kvcache) {
+        const int L = seqlen_of(p.seqlens, p.seqlen_scalar, b);
+        if (L < 0 || (int64_t)L + p.s_new > p.cap) {
+            if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
+            return;
+        }
+        N = L + p.s_new;
+    } else {
+        N = (int)p.s_k;
+    }
+    int i0[2], n_kv[2], mask_from[2];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        i0[x] = (2 * blk + x) * rows_per_tile;
+        const int i_last = min(p.s_q, i0[x] + rows_per_tile) - 1;
+        const int kv_end = i0[x] >= p.s_q ? 0 : (p.causal ? max(0, min(N, i_last + N - p.s_q + 1)) : N);
+        n_kv[x] = (kv_end + kBN - 1) / kBN;
+        mask_from[x] = p.causal ? max(0, min(N, i0[x] + N - p.s_q + 1)) : N;
+    }
+    const int n_all = max(n_kv[0], n_kv[1]);
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < KST; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < VST; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&s_full[x], 1);
+            mbar_init(&p_full[x], 4);
+            mbar_init(&o_full[x], 1);
+        }
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0 && n_all > 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            mbar_arrive_expect_tx(q_full, 2 * C::QBYTES);
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+                for (int c = 0; c < D_QK / 64; ++c)
+                    tma_load_4d(sQ + x * C::QBYTES + c * C::BOX, &tmQ, q_full, c * 64, hq0, i0[x], b);
+            for (int j = 0; j < n_all; ++j) {
+                const int ks = j % KST, vs = j % VST;
+                if (j >= KST && !mbar_wait(&k_empty[ks], ((j / KST) - 1) & 1, p.status)) break;
+                mbar_arrive_expect_tx(&k_full[ks], C::KBYTES);
+#pragma unroll
+                for (int c = 0; c < D_QK / 64; ++c)
+                    tma_load_4d(sK + ks * C::KBYTES + c * C::BOX, &tmK, &k_full[ks], c * 64, hk, j * kBN, b);
+                if (j >= VST && !mbar_wait(&v_empty[vs], ((j / VST) - 1) & 1, p.status)) break;
+                mbar_arrive_expect_tx(&v_full[vs], C::VBYTES);
+#pragma unroll
+                for (int c = 0; c < D_V / 64; ++c)
+                    tma_load_4d(sV + vs * C::VBYTES + c * C::BOX, &tmV, &v_full[vs], c * 64, hk, j * kBN, b);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0 && n_all > 0) {
+            const uint32_t idesc_qk = tc::idesc_f16(bf16, kBM, kBN, false);
+            const uint32_t idesc_pv = tc::idesc_f16(bf16, kBM, D_V, true);
+            const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
+            bool ok = mbar_wait(q_full, 0, p.status);
+            auto issue_qk = [&](int x, int j) {
+                const int ks = j % KST;
+#pragma unroll
+                for (int k = 0; k < D_QK / 16; ++k) {
+                    const uint64_t adesc =
+                        tc::smem_desc(aQ + x * C::QBYTES + (k >> 2) * C::BOX + (k & 3) * 32, 16, 1024);
+                    const uint64_t bdesc = tc::smem_desc(aK + ks * C::KBYTES + (k >> 2) * C::BOX + (k & 3) * 32, 16, 1024);
+                    tc::mma_ss(tmem + C::t_s(x), adesc, bdesc, idesc_qk, k > 0 ? 1u : 0u);
+                }
+                tc::commit(&s_full[x]);
+            };
+            auto issue_pv = [&](int x, int j) {
+                const int vs = j % VST;
+#pragma unroll
+                for (int k = 0; k < kBN / 16; ++k) {
+                    const uint64_t bdesc = tc::smem_desc(aV + vs * C::VBYTES + k * 16 * 128, C::BOX, 1024);
+                    tc::mma_ts(tmem + C::t_o(x), tmem + C::t_s(x) + k * 8, bdesc, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+                }
+            };
+            // prologue: QK of both tiles on key tile 0
+            if (ok && (ok = mbar_wait(&k_full[0], 0, p.status))) {
+                tc::fence_after_sync();
+                if (n_kv[0] > 0) issue_qk(0, 0);
+                if (n_kv[1] > 0) issue_qk(1, 0);
+                tc::commit(&k_empty[0]);
+            }
+            for (int j = 0; j < n_all && ok; ++j) {
+                const int vs = j % VST;
+                const bool next = j + 1 < n_all;
+                const int ks1 = (j + 1) % KST;
+                if (!(ok = mbar_wait(&v_full[vs], (j / VST) & 1, p.status))) break;
+                if (next && !(ok = mbar_wait(&k_full[ks1], ((j + 1) / KST) & 1, p.status))) break;
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    if (j < n_kv[x]) {
+                        if (!(ok = mbar_wait(&p_full[x], j & 1, p.status))) break;
+                        tc::fence_after_sync();
+                        issue_pv(x, j);
+                        if (j + 1 == n_kv[x]) tc::commit(&o_full[x]);
+                        if (j + 1 < n_kv[x]) issue_qk(x, j + 1);
+                    }
+                }
+                if (!ok) break;
+                tc::commit(&v_empty[vs]);
+                if (next) tc::commit(&k_empty[ks1]);
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------ softmax warpgroups
+        const int x = (warp - 4) >> 2;                 // tile of this warpgroup
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;                  // tile row = TMEM lane
+        const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+        const int prow = (2 * blk + x) * kBM + r;      // packed row
+        const int i = prow / pack;
+        const int hq = hq0 + (prow % pack);
+        const bool row_valid = i < p.s_q;
+        const int last_vis = row_valid ? (p.causal ? min(N - 1, i + N - p.s_q) : N - 1) : -1;
+        const float c = p.scale_log2;
+        const uint32_t s_addr = tmem + lane_addr + C::t_s(x);
+        const uint32_t o_addr = tmem + lane_addr + C::t_o(x);
+        const int nk = n_kv[x];
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nk && ok; ++j) {
+            if (!(ok = mbar_wait(&s_full[x], j & 1, p.status))) break;
+            tc::fence_after_sync();
+            const int j0 = j * kBN;
+            const bool masked = j0 + kBN > mask_from[x];
+            // pass 1: row max
+            float mt = -INFINITY;
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                uint32_t sr[32];
+                tc::ld32(s_addr + h * 32, sr);
+                tc::wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float v = __uint_as_float(sr[e]);
+                    mt = fmaxf(mt, (!masked || j0 + h * 32 + e <= last_vis) ? v : -INFINITY);
+                }
+            }
+            float alpha = 1.f;
+            bool rescale = false;
+            if (mt > m_ref && (m_ref == -INFINITY || (mt - m_ref) * c > 8.f)) {
+                alpha = m_ref == -INFINITY ? 0.f : ex2((m_ref - mt) * c);
+                rescale = m_ref != -INFINITY;
+                m_ref = mt;
+            }
+            const float mc = m_ref == -INFINITY ? 0.f : m_ref * c;
+            // pass 2: P = 2^(s c - m c) as 16-bit pairs over the first 64 columns
+            float rs = 0.f;
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                uint32_t sr[32], pk[16];
+                tc::ld32(s_addr + h * 32, sr);
+                tc::wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const bool vis0 = !masked || j0 + h * 32 + e <= last_vis;
+                    const bool vis1 = !masked || j0 + h * 32 + e + 1 <= last_vis;
+                    const float p0 = vis0 ? ex2(fmaf(__uint_as_float(sr[e]), c, -mc)) : 0.f;
+                    const float p1 = vis1 ? ex2(fmaf(__uint_as_float(sr[e + 1]), c, -mc)) : 0.f;
+                    rs += p0 + p1;
+                    pk[e >> 1] = Elem<T>::pack2(p0, p1);
+                }
+                // P of keys [32h, 32h+32) goes to columns [16h, 16h+16), whose
+                // S values were read in this or an earlier chunk
+                tc::st16(s_addr + h * 16, pk);
+            }
+            l = l * alpha + rs;
+            if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                for (int h = 0; h < D_V / 32; ++h) {
+                    uint32_t orr[32];
+                    tc::ld32(o_addr + h * 32, orr);
+                    tc::wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+                    tc::st32(o_addr + h * 32, orr);
+                }
+            }
+            tc::wait_st();
+            if (p.kvcache && j == nk - 1 && j0 + kBN > N) {
+                // cache rows past N_b may hold anything: zero them in the V tile
+                // (both tiles' warpgroups do it; the writes are identical)
+                const int vs = j % VST;
+                if (!(ok = mbar_wait(&v_full[vs], (j / VST) & 1, p.status))) break;
+                uint8_t *vt = sV + vs * C::VBYTES;
+                const int first = N - j0;
+                const int n16 = (kBN - first) * 8 * (D_V / 64);
+                for (int idx = threadIdx.x - 128 * (1 + x); idx < n16; idx += 128) {
+                    const int box = idx / ((kBN - first) * 8);
+                    const int rem = idx % ((kBN - first) * 8);
+                    *reinterpret_cast<uint4 *>(vt + box * C::BOX + (first + rem / 8) * 128 + (rem % 8) * 16) =
+                        make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async();
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[x]);
+        }
+        // ------------------------------------------------ epilogue
+        if (ok && nk > 0 && !mbar_wait(&o_full[x], 0, p.status)) ok = false;
+        tc::fence_after_sync();
+        T *orow = static_cast<T *>(p.out) + b * p.os.b + (int64_t)i * p.os.s + hq * p.os.h;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+        for (int h = 0; h < D_V / 32; ++h) {
+            uint32_t orr[32];
+            if (nk > 0) {
+                tc::ld32(o_addr + h * 32, orr);
+                tc::wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) orr[e] = 0u;
+            }
+            if (row_valid) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                    float f[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) f[u] = __uint_as_float(orr[e + u]) * inv;
+                    reinterpret_cast<uint4 *>(orow + h * 32 + e)[0] = pack8<T>(f);
+                }
+            }
+        }
+        if (row_valid && p.lse)
+            p.lse[((int64_t)b * p.h_q + hq) * p.s_q + i] = l > 0.f ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
 template <typename T, int D_QK, int D_V>
 static cudaError_t run_prefill(const PrefillParams &p, const CUtensorMap &tmQ, const CUtensorMap &tmK,
                                const CUtensorMap &tmV, cudaStream_t st) {
+    if (p.tiles_per_cta == 2) {
+        using C2 = Prefill2Cfg<D_QK, D_V>;
+        cudaError_t e = cudaFuncSetAttribute(prefill2_kernel<T, D_QK, D_V>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C2::SMEM);
+        if (e != cudaSuccess) return e;
+        dim3 grid((p.n_q_tiles + 1) / 2, p.h_q / p.pack, p.b);
+        prefill2_kernel<T, D_QK, D_V><<<grid, 384, C2::SMEM, st>>>(tmQ, tmK, tmV, p);
+        return cudaGetLastError();
+    }
     using C = PrefillCfg<D_QK, D_V>;
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel<T, D_QK, D_V>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);

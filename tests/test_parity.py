@@ -72,7 +72,7 @@ MLA_DECODE_SMALL = W.MLA_DECODE.scaled(name="mla-decode small", batch=2, h_q=4, 
 
 
 @pytest.mark.parametrize("w", [DECODE_SMALL, PREFILL_SMALL, MLA_DECODE_SMALL], ids=lambda w: w.name)
-def test_kvcache_small_configs(w, cuda_device):
+def test_kvcache_small_configs(w, prefill_tiles, cuda_device):
     inp = W.make_inputs(w)
     check_kvcache(w, inp, run_gpu_kvcache(w, inp, cuda_device), run_oracle_kvcache(w, inp))
 
@@ -169,9 +169,16 @@ def test_empty_batch(cuda_device):
 
 
 # ------------------------------------------------------------------ dense (fa_fwd)
+@pytest.fixture(params=["1", "2"], ids=["1tile", "2tiles"])
+def prefill_tiles(request, monkeypatch):
+    """Run the test with the one-tile and with the two-tile prefill kernel."""
+    monkeypatch.setenv("FA_PREFILL_TILES_PER_CTA", request.param)
+    return int(request.param)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("dims", [(64, 64, "fp16"), (192, 128, "bf16"), (128, 128, "bf16"), (16, 16, "fp16")])
-def test_dense_small(dims, causal, cuda_device):
+def test_dense_small(dims, causal, prefill_tiles, cuda_device):
     d_qk, d_v, dt = dims
     for s_q, s_k in ((200, 200), (77, 300), (300, 77)):
         w = W.Workload(name="dense-small", mode="dense", dtype=dt, batch=2, h_q=4, h_kv=2, d_qk=d_qk,
@@ -185,7 +192,7 @@ def test_dense_small(dims, causal, cuda_device):
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("dims", [(128, 128, "bf16", 6, 2), (192, 128, "bf16", 4, 4), (64, 64, "fp16", 8, 1),
                                   (128, 64, "fp16", 3, 3), (64, 128, "bf16", 2, 2)])
-def test_dense_multi_tile(dims, causal, cuda_device):
+def test_dense_multi_tile(dims, causal, prefill_tiles, cuda_device):
     """Several 128-row query and key tiles with ragged tails; g = 3 takes the
     unpacked path, g = 8 and g = 1 the packed one; the K/V ring wraps."""
     d_qk, d_v, dt, hq, hkv = dims
@@ -198,7 +205,7 @@ def test_dense_multi_tile(dims, causal, cuda_device):
 
 
 @pytest.mark.parametrize("s_new", [1, 300])
-def test_kvcache_garbage_past_sequence(s_new, cuda_device):
+def test_kvcache_garbage_past_sequence(s_new, prefill_tiles, cuda_device):
     """Cache rows at and past N_b hold NaN: they must not reach the result (the
     rows are masked in the scores and zeroed before the PV product)."""
     w = W.Workload(name="nan-tail", mode="kvcache", dtype="bf16", batch=2, h_q=8, h_kv=2, d_qk=128,
