@@ -63,14 +63,15 @@ struct DecodeCfg {
     static constexpr int STAGE = KBYTES + VBYTES;
     static constexpr int QROWS = MT * 16;
     static constexpr int QBYTES = ((QROWS * D_QK * 2 + 1023) / 1024) * 1024;
-    static constexpr int TAIL = 2 * kDecodeMaxStages * 8 + 64;
     static_assert(D_QK % 16 == 0 && D_V % 16 == 0, "head dims are multiples of 16");
     static int merge_bytes(int M) { return 4 * M * (D_V + 2) * 4; }
-    static int stages(int M) {
-        const int raw = (DecodeOcc<D_V, MT>::BUDGET - 1024 - QBYTES - merge_bytes(M) - TAIL) / STAGE;
+    // barriers, the 4-int schedule and the per-batch (L, N, items) table
+    static int tail_bytes(int B) { return 2 * kDecodeMaxStages * 8 + 16 + 12 * B + 16; }
+    static int stages(int M, int B) {
+        const int raw = (DecodeOcc<D_V, MT>::BUDGET - 1024 - QBYTES - merge_bytes(M) - tail_bytes(B)) / STAGE;
         return raw < 2 ? 2 : (raw > kDecodeMaxStages ? kDecodeMaxStages : raw);
     }
-    static int smem(int M) { return 1024 + QBYTES + stages(M) * STAGE + merge_bytes(M) + TAIL; }
+    static int smem(int M, int B) { return 1024 + QBYTES + stages(M, B) * STAGE + merge_bytes(M) + tail_bytes(B); }
 };
 
 // Per-batch facts every thread can recompute: rows N_b and items n_b (0 when
@@ -96,7 +97,8 @@ struct ItemIter {
     SegInfo seg;
 };
 
-__device__ __forceinline__ void iter_advance(const DecodeParams &p, ItemIter &it) {
+// `tab` is the per-batch SegInfo table the CTA staged in shared memory.
+__device__ __forceinline__ void iter_advance(const DecodeParams &p, const SegInfo *tab, ItemIter &it) {
     if (++it.s < it.seg.n_items) return;
     it.s = 0;
     if (++it.hk < p.h_kv) return;
@@ -104,20 +106,21 @@ __device__ __forceinline__ void iter_advance(const DecodeParams &p, ItemIter &it
     do {
         ++it.b;
         if (it.b >= p.b) return;
-        it.seg = seg_info(p, it.b);
+        it.seg = tab[it.b];
     } while (it.seg.n_items == 0);
 }
 
 // Global index of the first item whose first row is >= X in the concatenated
 // row space, and the CTA's item range [I(c R/G), I((c+1) R/G)).
-__device__ void cta_item_range(const DecodeParams &p, int c, int G, ItemIter &first, int &n_items) {
+__device__ void cta_item_range(const DecodeParams &p, const SegInfo *tab, int c, int G, ItemIter &first,
+                               int &n_items) {
     int64_t R = 0;
-    for (int b = 0; b < p.b; ++b) R += (int64_t)p.h_kv * seg_info(p, b).N;
+    for (int b = 0; b < p.b; ++b) R += (int64_t)p.h_kv * tab[b].N;
     const int64_t X0 = R * c / G, X1 = R * (c + 1) / G;
     int64_t I0 = -1, I1 = -1, items_before = 0, rows_before = 0;
     first.b = p.b;
     for (int b = 0; b < p.b && I1 < 0; ++b) {
-        const SegInfo sg = seg_info(p, b);
+        const SegInfo sg = tab[b];
         const int64_t seg_rows = (int64_t)p.h_kv * sg.N;
         for (int which = 0; which < 2; ++which) {
             const int64_t X = which ? X1 : X0;
@@ -134,7 +137,7 @@ __device__ void cta_item_range(const DecodeParams &p, int c, int G, ItemIter &fi
                 first.seg = sg;
                 if (first.s >= sg.n_items) {
                     first.s = sg.n_items - 1;
-                    iter_advance(p, first);
+                    iter_advance(p, tab, first);
                 }
             }
         }
@@ -166,6 +169,7 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
     uint64_t *full = reinterpret_cast<uint64_t *>(red_l + 4 * M);
     uint64_t *empty = full + kDecodeMaxStages;
     int *sched = reinterpret_cast<int *>(empty + kDecodeMaxStages);   // b, hk, s, n_items
+    SegInfo *tab = reinterpret_cast<SegInfo *>(sched + 4);             // [b]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool inter = p.interleaved != 0;
@@ -173,6 +177,9 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
     // allow the combine kernel (launched as a programmatic dependent) to get scheduled
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
+    // stage every batch entry's (L, N, items) once, with parallel loads
+    for (int b = threadIdx.x; b < p.b; b += blockDim.x) tab[b] = seg_info(p, b);
+    __syncthreads();
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
@@ -181,7 +188,7 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
         fence_barrier_init();
         ItemIter first;
         int n_items;
-        cta_item_range(p, blockIdx.x, gridDim.x, first, n_items);
+        cta_item_range(p, tab, blockIdx.x, gridDim.x, first, n_items);
         sched[0] = first.b;
         sched[1] = first.hk;
         sched[2] = first.s;
@@ -190,9 +197,9 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
     if (blockIdx.x == 0) {
         // batch entries with no key at all: out = 0, lse = -inf; bad entries: record
         for (int b = 0; b < p.b; ++b) {
-            const int L = seqlen_of(p.seqlens, p.seqlen_scalar, b);
-            const SegInfo sg = seg_info(p, b);
+            const SegInfo sg = tab[b];
             if (sg.n_items > 0) continue;
+            const int L = sg.L;
             const bool bad = L < 0 || (int64_t)L + p.s_new > p.cap ||
                              (p.r > 0 && (int64_t)L + (p.s_q > p.s_new ? p.s_q : p.s_new) > p.cs_rows);
             if (bad) {
@@ -215,7 +222,7 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
     it0.b = sched[0];
     it0.hk = sched[1];
     it0.s = sched[2];
-    it0.seg = seg_info(p, it0.b);
+    it0.seg = tab[it0.b];
 
     if (warp == 4) {
         // ---------------- producer: TMA stream of K/V tiles over all items ----------------
@@ -242,7 +249,7 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
                 for (int c = 0; c < D_V / CHV; ++c)
                     tma_load_4d(vd + c * C::TILE * RBV, &tmV, &full[s], c * CHV, it.hk, row0, it.b);
                 ++t;
-                iter_advance(p, it);
+                iter_advance(p, tab, it);
             }
         }
         return;
@@ -508,7 +515,7 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
                 }
             }
         }
-        iter_advance(p, it);
+        iter_advance(p, tab, it);
     }
 }
 
@@ -621,8 +628,9 @@ static cudaError_t run_decode(const DecodeParams &p_in, const CUtensorMap &tmK, 
     using C = DecodeCfg<D_QK, D_V, MT>;
     DecodeParams p = p_in;
     const int M = p.g * p.s_q;
-    p.n_stages = C::stages(M);
-    const int smem = C::smem(M);
+    p.n_stages = C::stages(M, p.b);
+    const int smem = C::smem(M, p.b);
+    if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D_QK, D_V, MT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;

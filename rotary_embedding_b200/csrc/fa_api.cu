@@ -224,8 +224,9 @@ KvPlan plan_kvcache(int64_t b, int64_t s_q, int64_t h_q, int64_t h_kv, int64_t d
     const int64_t M = g * s_q;
     const int mt = M <= 16 ? 1 : 2;
     // the combine holds up to 512 split slots per output row in registers
+    // the decode kernel stages a 12-byte record per batch entry in shared memory
     if (s_q <= 8 && M <= 32 && (s_new == 0 || s_new == s_q) && decode_supported((int)d_qk, (int)d_v, mt) &&
-        cap >= 1 && cap <= 512 * 64) {
+        cap >= 1 && cap <= 512 * 64 && b <= 1024) {
         pl.decode = true;
         pl.mt = mt;
         // The persistent decode kernel balances 64-row items across the SMs;
@@ -320,6 +321,9 @@ int validate_kvcache(const fa_tensor *q, const fa_tensor *k_cache, const fa_tens
 }
 
 }  // namespace
+
+int set_last_error(int code, const char *msg) { return fail(code, "%s", msg); }
+
 }  // namespace fa
 
 using namespace fa;

@@ -109,6 +109,9 @@ struct PrefillParams {
 
 int sm_count();
 
+// Sets the thread-local message fa_last_error() returns; returns `code`.
+int set_last_error(int code, const char *msg);
+
 cudaError_t launch_rope_append(const RopeAppendParams &p, int dtype, cudaStream_t st);
 bool prefill_supported(int d_qk, int d_v);
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &tmQ, const CUtensorMap &tmK,

@@ -359,7 +359,12 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
 // before the QK overwrites it.  When softmax X sees S_X(j) complete, every
 // earlier MMA of the CTA has completed too, so O_X is stable and can be
 // rescaled without a further wait.
-// Warps: 0 TMA, 1 MMA, 4-7 softmax of tile A, 8-11 softmax of tile B.
+// Warps: 0 TMA, 1 MMA, 2-3 idle (warpgroup 0), 4-7 softmax of tile A
+// (warpgroup 1), 8-11 softmax of tile B (warpgroup 2); warp w reaches TMEM
+// lanes 32 (w % 4) .. 32 (w % 4) + 31.  The register file is split with
+// setmaxnreg: warpgroup 0 drops to 64 registers per thread, the two softmax
+// warpgroups rise to 216 so that a whole 128-column S row stays in registers
+// (128 x 64 + 256 x 216 = 63488, within the 384 x 168 the block is launched with).
 // ============================================================================
 template <int D_QK, int D_V>
 struct Prefill2Cfg {
@@ -462,6 +467,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
 
+    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0 && n_all > 0) {
@@ -544,8 +550,9 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         }
     } else if (warp >= 4) {
         // ------------------------------------------------ softmax warpgroups
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 216;" ::: "memory");
         const int x = (warp - 4) >> 2;                 // tile of this warpgroup
-        const int q4 = warp & 3;
+        const int q4 = warp & 3;                       // TMEM lane quadrant this warp may access
         const int r = q4 * 32 + lane;                  // tile row = TMEM lane
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
         const int prow = (2 * blk + x) * kBM + r;      // packed row
@@ -554,6 +561,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         const bool row_valid = i < p.s_q;
         const int last_vis = row_valid ? (p.causal ? min(N - 1, i + N - p.s_q) : N - 1) : -1;
         const float c = p.scale_log2;
+        const uint64_t c2 = f2_pack(c, c);
         const uint32_t s_addr = tmem + lane_addr + C::t_s(x);
         const uint32_t o_addr = tmem + lane_addr + C::t_o(x);
         const int nk = n_kv[x];
@@ -563,20 +571,27 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             if (!(ok = mbar_wait(&s_full[x], j & 1, p.status))) break;
             tc::fence_after_sync();
             const int j0 = j * kBN;
-            const bool masked = j0 + kBN > mask_from[x];
-            // pass 1: row max
-            float mt = -INFINITY;
+            uint32_t sr[4][32];
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                uint32_t sr[32];
-                tc::ld32(s_addr + h * 32, sr);
-                tc::wait_ld();
+            for (int h = 0; h < 4; ++h) tc::ld32(s_addr + h * 32, sr[h]);
+            tc::wait_ld();
+            if (j0 + kBN > mask_from[x]) {
+                // diagonal band or sequence end: -inf outside the visible keys
+                // (only these tiles pay for the comparisons)
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float v = __uint_as_float(sr[e]);
-                    mt = fmaxf(mt, (!masked || j0 + h * 32 + e <= last_vis) ? v : -INFINITY);
-                }
+                for (int h = 0; h < 4; ++h)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (j0 + h * 32 + e > last_vis) sr[h][e] = __float_as_uint(-INFINITY);
             }
+            // row max over 128 scores: four independent three-input chains
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+#pragma unroll
+                for (int e = 0; e < 32; e += 2)
+                    mx[h] = fmax3(mx[h], __uint_as_float(sr[h][e]), __uint_as_float(sr[h][e + 1]));
+            const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             float alpha = 1.f;
             bool rescale = false;
             if (mt > m_ref && (m_ref == -INFINITY || (mt - m_ref) * c > 8.f)) {
@@ -585,26 +600,30 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                 m_ref = mt;
             }
             const float mc = m_ref == -INFINITY ? 0.f : m_ref * c;
-            // pass 2: P = 2^(s c - m c) as 16-bit pairs over the first 64 columns
-            float rs = 0.f;
+            const uint64_t nmc2 = f2_pack(-mc, -mc);
+            // P = 2^(s c - m c), written as 16-bit pairs over the first 64
+            // columns of the S buffer (keys [32h, 32h+32) -> columns [16h, 16h+16),
+            // all of which were read above)
+            uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-                uint32_t sr[32], pk[16];
-                tc::ld32(s_addr + h * 32, sr);
-                tc::wait_ld();
+                uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const bool vis0 = !masked || j0 + h * 32 + e <= last_vis;
-                    const bool vis1 = !masked || j0 + h * 32 + e + 1 <= last_vis;
-                    const float p0 = vis0 ? ex2(fmaf(__uint_as_float(sr[e]), c, -mc)) : 0.f;
-                    const float p1 = vis1 ? ex2(fmaf(__uint_as_float(sr[e + 1]), c, -mc)) : 0.f;
-                    rs += p0 + p1;
+                    const uint64_t t = f2_fma(f2_pack(__uint_as_float(sr[h][e]), __uint_as_float(sr[h][e + 1])), c2, nmc2);
+                    float t0, t1;
+                    f2_unpack(t, t0, t1);
+                    const float p0 = ex2(t0), p1 = ex2(t1);
+                    const uint64_t pp = f2_pack(p0, p1);
+                    rs2[(e >> 1) & 1] = f2_add(rs2[(e >> 1) & 1], pp);
                     pk[e >> 1] = Elem<T>::pack2(p0, p1);
                 }
-                // P of keys [32h, 32h+32) goes to columns [16h, 16h+16), whose
-                // S values were read in this or an earlier chunk
                 tc::st16(s_addr + h * 16, pk);
             }
+            float ra, rb, rc_, rd;
+            f2_unpack(rs2[0], ra, rb);
+            f2_unpack(rs2[1], rc_, rd);
+            const float rs = (ra + rb) + (rc_ + rd);
             l = l * alpha + rs;
             if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
@@ -626,7 +645,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                 uint8_t *vt = sV + vs * C::VBYTES;
                 const int first = N - j0;
                 const int n16 = (kBN - first) * 8 * (D_V / 64);
-                for (int idx = threadIdx.x - 128 * (1 + x); idx < n16; idx += 128) {
+                for (int idx = threadIdx.x - 128 - 128 * x; idx < n16; idx += 128) {
                     const int box = idx / ((kBN - first) * 8);
                     const int rem = idx % ((kBN - first) * 8);
                     *reinterpret_cast<uint4 *>(vt + box * C::BOX + (first + rem / 8) * 128 + (rem % 8) * 16) =
