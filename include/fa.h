@@ -134,6 +134,41 @@ int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor
                    const fa_tensor *out, float *lse,
                    void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * fa_kvcache_fwd_noalloc -- the same call as fa_kvcache_fwd, without a
+ * workspace argument.  (The pages have no counterpart: this exists for
+ * callers of this library.)
+ *
+ * For callers that cannot allocate device memory when they run attention:
+ * a plug-in whose host application owns every device allocation and gives
+ * it no allocator, or a latency-critical loop that must never enter the CUDA
+ * allocator (cudaMalloc can synchronise the device).  The caller still
+ * passes inputs and outputs; the scratch comes from a fixed array of
+ * FA_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.
+ *
+ *  - Arguments, layouts and results are those of fa_kvcache_fwd.
+ *  - Shapes whose fa_kvcache_workspace_size exceeds FA_NOALLOC_SCRATCH_BYTES
+ *    are rejected with FA_ERR_WORKSPACE (fa_last_error() says how much they
+ *    need); nothing is enqueued.
+ *  - The first call on a device looks up the scratch array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - No cudaMalloc, cudaFree or other allocating routine is called.
+ *  - Every call on a device shares the one scratch array: calls whose work
+ *    overlaps on the GPU (different streams, or another thread) race on it
+ *    and must be serialised by the caller.  The array keeps the last call's
+ *    contents; nothing in it needs to start at zero.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+int fa_kvcache_fwd_noalloc(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
+                           const fa_tensor *k_new, const fa_tensor *v_new,
+                           const fa_tensor *cos, const fa_tensor *sin,
+                           const int32_t *cache_seqlens, int32_t cache_seqlens_scalar,
+                           int32_t rotary_dim, int32_t interleaved, int32_t causal, float scale,
+                           const fa_tensor *out, float *lse, void *stream);
+
 /* Workspace bytes fa_kvcache_fwd needs for these shapes (k_new may be NULL). */
 int fa_kvcache_workspace_size(const fa_tensor *q, const fa_tensor *k_cache,
                               const fa_tensor *v_cache, const fa_tensor *k_new,

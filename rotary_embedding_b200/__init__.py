@@ -155,6 +155,44 @@ def fa_kvcache_fwd(q, k_cache, v_cache, k_new=None, v_new=None, rotary_cos=None,
     return out, lse
 
 
+lib.fa_kvcache_fwd_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _v, _i32, _i32, _i32, _i32, ctypes.c_float,
+                                        _P, _v, _v]
+lib.fa_kvcache_fwd_noalloc.restype = ctypes.c_int
+FA_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def fa_kvcache_fwd_noalloc(q, k_cache, v_cache, k_new=None, v_new=None, rotary_cos=None,
+                           rotary_sin=None, cache_seqlens=0, rotary_dim=None,
+                           rotary_interleaved=False, causal=False, softmax_scale=None, out=None,
+                           lse=None, return_lse=True, stream=None):
+    """fa_kvcache_fwd whose scratch comes from the library's built-in array
+    (FA_NOALLOC_SCRATCH_BYTES) instead of a workspace: for callers that must not
+    allocate device memory when attention runs.  The library call itself
+    allocates nothing; this Python wrapper only allocates `out`/`lse` when they
+    are not passed.  Calls that overlap on the GPU share the scratch and race."""
+    b, s_q, h_q, _ = q.shape
+    d_v = v_cache.shape[3]
+    if rotary_cos is not None and rotary_dim is None:
+        rotary_dim = 2 * rotary_cos.shape[1]
+    rotary_dim = int(rotary_dim or 0) if rotary_cos is not None else 0
+    if out is None:
+        out = torch.empty((b, s_q, h_q, d_v), dtype=q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
+    if isinstance(cache_seqlens, torch.Tensor):
+        seq_ptr, seq_scalar = ctypes.c_void_p(cache_seqlens.data_ptr()), 0
+    else:
+        seq_ptr, seq_scalar = None, int(cache_seqlens)
+    _check(lib.fa_kvcache_fwd_noalloc(
+        _ref(describe(q)), _ref(describe(k_cache)), _ref(describe(v_cache)), _ref(describe(k_new)),
+        _ref(describe(v_new)), _ref(describe(rotary_cos)), _ref(describe(rotary_sin)), seq_ptr,
+        seq_scalar, rotary_dim, int(bool(rotary_interleaved)), int(bool(causal)),
+        float(softmax_scale or 0.0), _ref(describe(out)),
+        ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+        _stream_handle(stream, q.device)))
+    return out, lse
+
+
 def fa_fwd(q, k, v, causal=False, softmax_scale=None, out=None, lse=None, workspace=None,
            return_lse=True, stream=None):
     """Cache-less attention: q [b, s_q, h_q, d_qk], k/v [b, s_k, h_kv, d]; returns (out, lse)."""
