@@ -265,6 +265,18 @@ def cpu_sample(w, inp, budget_s):
     return amount, t_total, desc
 
 
+def aggregate_over_ranks(ms_local: float, amount: float, world: int, device):
+    """Whole-job throughput: every rank processed `amount` units in its own
+    device time; the job takes the slowest rank's time (max over ranks)."""
+    ms_max = ms_local
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms_local], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    return ms_max, world * amount / (ms_max / 1e3)
+
+
 def run_ours(args):
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -307,21 +319,15 @@ def run_ours(args):
             torch.cuda.synchronize()
         times = time_steps(graph.replay, args.steps, max(args.warmup, 3), stream, flush_buf, barrier)
     ms = sum(times) / len(times)
-    t = torch.tensor([ms], device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
-    value = world * amount / (ms_max / 1e3)
+    ms_max, value = aggregate_over_ranks(ms, amount, world, device)
 
     e2e_value, h2d, d2h = None, 0, 0
     if not args.no_e2e:
         e2e_times, h2d, d2h = time_e2e(w, inp, inp_dev, lambda: make_step(w, inp_dev, fa), args.steps,
                                        max(args.warmup, 3), stream, flush_buf, barrier)
         e_ms = sum(e2e_times) / len(e2e_times)
-        t = torch.tensor([e_ms], device=device)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_value = round(world * amount / (float(t.item()) / 1e3), 3)
+        _, e2e_value = aggregate_over_ranks(e_ms, amount, world, device)
+        e2e_value = round(e2e_value, 3)
 
     peaks, peaks_src = load_peaks()
     if bound == "hbm":
