@@ -176,11 +176,6 @@ int run_tc_attention(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
     const int64_t h_kv = k->shape[2], d_v = v->shape[3];
     const int64_t g = h_q / h_kv;
     const int pack = (128 % g == 0) ? (int)g : 1;
-    CUtensorMap tmQ, tmK, tmV;
-    int rc;
-    if ((rc = make_rows_map(&tmQ, q, 128 / pack, "q", pack))) return rc;
-    if ((rc = make_rows_map(&tmK, k, 128, "k"))) return rc;
-    if ((rc = make_rows_map(&tmV, v, 128, "v"))) return rc;
     PrefillParams p{};
     p.status = status;
     p.out = out->data;
@@ -212,6 +207,12 @@ int run_tc_attention(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
         if (env[0] == '1') p.tiles_per_cta = 1;
         if (env[0] == '2') p.tiles_per_cta = 2;
     }
+    const int bn = prefill_block_n((int)d_qk, (int)d_v, p.tiles_per_cta);
+    CUtensorMap tmQ, tmK, tmV;
+    int rc;
+    if ((rc = make_rows_map(&tmQ, q, 128 / pack, "q", pack))) return rc;
+    if ((rc = make_rows_map(&tmK, k, bn, "k"))) return rc;
+    if ((rc = make_rows_map(&tmV, v, bn, "v"))) return rc;
     cudaError_t e = launch_prefill(p, tmQ, tmK, tmV, q->dtype, (int)d_qk, (int)d_v, st);
     if (e != cudaSuccess) return cuda_fail(e, "tcgen05 attention launch");
     return FA_OK;

@@ -114,6 +114,7 @@ int set_last_error(int code, const char *msg);
 
 cudaError_t launch_rope_append(const RopeAppendParams &p, int dtype, cudaStream_t st);
 bool prefill_supported(int d_qk, int d_v);
+int prefill_block_n(int d_qk, int d_v, int tiles_per_cta);  // key rows per K/V tile (TMA box rows)
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &tmQ, const CUtensorMap &tmK,
                            const CUtensorMap &tmV, int dtype, int d_qk, int d_v, cudaStream_t st);
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,

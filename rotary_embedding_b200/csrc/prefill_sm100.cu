@@ -368,10 +368,15 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
 // ============================================================================
 template <int D_QK, int D_V>
 struct Prefill2Cfg {
+    // Key rows per tile: 128, or 96 for d_qk > 128 so that K and V both stay
+    // double-buffered next to the two Q tiles (a single V buffer would expose
+    // every V load in full).
+    static constexpr int BN = D_QK > 128 ? 96 : 128;
     static constexpr int QBYTES = kBM * D_QK * 2;   // per tile
-    static constexpr int KBYTES = kBN * D_QK * 2;
-    static constexpr int VBYTES = kBN * D_V * 2;
-    static constexpr int BOX = 128 * 128;            // bytes of one 64-column box of 128 rows
+    static constexpr int KBYTES = BN * D_QK * 2;
+    static constexpr int VBYTES = BN * D_V * 2;
+    static constexpr int QBOX = kBM * 128;           // bytes of one 64-column box of a Q tile
+    static constexpr int KBOX = BN * 128;            // ... of a K or V tile
     static constexpr int BUDGET = 224 * 1024;
     static constexpr int AVAIL = BUDGET - 2 * QBYTES;
     static constexpr bool EVEN = AVAIL >= 2 * (KBYTES + VBYTES);
@@ -393,7 +398,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                                                           const __grid_constant__ CUtensorMap tmV,
                                                           const PrefillParams p) {
     using C = Prefill2Cfg<D_QK, D_V>;
-    constexpr int KST = C::KST, VST = C::VST;
+    constexpr int KST = C::KST, VST = C::VST, BN = C::BN;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem;                              // 2 tiles
@@ -435,7 +440,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         i0[x] = (2 * blk + x) * rows_per_tile;
         const int i_last = min(p.s_q, i0[x] + rows_per_tile) - 1;
         const int kv_end = i0[x] >= p.s_q ? 0 : (p.causal ? max(0, min(N, i_last + N - p.s_q + 1)) : N);
-        n_kv[x] = (kv_end + kBN - 1) / kBN;
+        n_kv[x] = (kv_end + BN - 1) / BN;
         mask_from[x] = p.causal ? max(0, min(N, i0[x] + N - p.s_q + 1)) : N;
     }
     const int n_all = max(n_kv[0], n_kv[1]);
@@ -479,25 +484,25 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             for (int x = 0; x < 2; ++x)
 #pragma unroll
                 for (int c = 0; c < D_QK / 64; ++c)
-                    tma_load_4d(sQ + x * C::QBYTES + c * C::BOX, &tmQ, q_full, c * 64, hq0, i0[x], b);
+                    tma_load_4d(sQ + x * C::QBYTES + c * C::QBOX, &tmQ, q_full, c * 64, hq0, i0[x], b);
             for (int j = 0; j < n_all; ++j) {
                 const int ks = j % KST, vs = j % VST;
                 if (j >= KST && !mbar_wait(&k_empty[ks], ((j / KST) - 1) & 1, p.status)) break;
                 mbar_arrive_expect_tx(&k_full[ks], C::KBYTES);
 #pragma unroll
                 for (int c = 0; c < D_QK / 64; ++c)
-                    tma_load_4d(sK + ks * C::KBYTES + c * C::BOX, &tmK, &k_full[ks], c * 64, hk, j * kBN, b);
+                    tma_load_4d(sK + ks * C::KBYTES + c * C::KBOX, &tmK, &k_full[ks], c * 64, hk, j * BN, b);
                 if (j >= VST && !mbar_wait(&v_empty[vs], ((j / VST) - 1) & 1, p.status)) break;
                 mbar_arrive_expect_tx(&v_full[vs], C::VBYTES);
 #pragma unroll
                 for (int c = 0; c < D_V / 64; ++c)
-                    tma_load_4d(sV + vs * C::VBYTES + c * C::BOX, &tmV, &v_full[vs], c * 64, hk, j * kBN, b);
+                    tma_load_4d(sV + vs * C::VBYTES + c * C::KBOX, &tmV, &v_full[vs], c * 64, hk, j * BN, b);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0 && n_all > 0) {
-            const uint32_t idesc_qk = tc::idesc_f16(bf16, kBM, kBN, false);
+            const uint32_t idesc_qk = tc::idesc_f16(bf16, kBM, BN, false);
             const uint32_t idesc_pv = tc::idesc_f16(bf16, kBM, D_V, true);
             const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
             bool ok = mbar_wait(q_full, 0, p.status);
@@ -506,8 +511,8 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
 #pragma unroll
                 for (int k = 0; k < D_QK / 16; ++k) {
                     const uint64_t adesc =
-                        tc::smem_desc(aQ + x * C::QBYTES + (k >> 2) * C::BOX + (k & 3) * 32, 16, 1024);
-                    const uint64_t bdesc = tc::smem_desc(aK + ks * C::KBYTES + (k >> 2) * C::BOX + (k & 3) * 32, 16, 1024);
+                        tc::smem_desc(aQ + x * C::QBYTES + (k >> 2) * C::QBOX + (k & 3) * 32, 16, 1024);
+                    const uint64_t bdesc = tc::smem_desc(aK + ks * C::KBYTES + (k >> 2) * C::KBOX + (k & 3) * 32, 16, 1024);
                     tc::mma_ss(tmem + C::t_s(x), adesc, bdesc, idesc_qk, k > 0 ? 1u : 0u);
                 }
                 tc::commit(&s_full[x]);
@@ -515,8 +520,8 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             auto issue_pv = [&](int x, int j) {
                 const int vs = j % VST;
 #pragma unroll
-                for (int k = 0; k < kBN / 16; ++k) {
-                    const uint64_t bdesc = tc::smem_desc(aV + vs * C::VBYTES + k * 16 * 128, C::BOX, 1024);
+                for (int k = 0; k < BN / 16; ++k) {
+                    const uint64_t bdesc = tc::smem_desc(aV + vs * C::VBYTES + k * 16 * 128, C::KBOX, 1024);
                     tc::mma_ts(tmem + C::t_o(x), tmem + C::t_s(x) + k * 8, bdesc, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
                 }
             };
@@ -570,28 +575,33 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         for (int j = 0; j < nk && ok; ++j) {
             if (!(ok = mbar_wait(&s_full[x], j & 1, p.status))) break;
             tc::fence_after_sync();
-            const int j0 = j * kBN;
-            uint32_t sr[4][32];
+            const int j0 = j * BN;
+            constexpr int NCH = BN / 32;               // 32-column chunks of the S row
+            uint32_t sr[NCH][32];
 #pragma unroll
-            for (int h = 0; h < 4; ++h) tc::ld32(s_addr + h * 32, sr[h]);
+            for (int h = 0; h < NCH; ++h) tc::ld32(s_addr + h * 32, sr[h]);
             tc::wait_ld();
-            if (j0 + kBN > mask_from[x]) {
+            if (j0 + BN > mask_from[x]) {
                 // diagonal band or sequence end: -inf outside the visible keys
                 // (only these tiles pay for the comparisons)
 #pragma unroll
-                for (int h = 0; h < 4; ++h)
+                for (int h = 0; h < NCH; ++h)
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
                         if (j0 + h * 32 + e > last_vis) sr[h][e] = __float_as_uint(-INFINITY);
             }
-            // row max over 128 scores: four independent three-input chains
-            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            // row max: one independent three-input chain per chunk
+            float mx[NCH];
 #pragma unroll
-            for (int h = 0; h < 4; ++h)
+            for (int h = 0; h < NCH; ++h) {
+                mx[h] = -INFINITY;
 #pragma unroll
                 for (int e = 0; e < 32; e += 2)
                     mx[h] = fmax3(mx[h], __uint_as_float(sr[h][e]), __uint_as_float(sr[h][e + 1]));
-            const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            }
+            float mt = mx[0];
+#pragma unroll
+            for (int h = 1; h < NCH; ++h) mt = fmaxf(mt, mx[h]);
             float alpha = 1.f;
             bool rescale = false;
             if (mt > m_ref && (m_ref == -INFINITY || (mt - m_ref) * c > 8.f)) {
@@ -601,12 +611,12 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             }
             const float mc = m_ref == -INFINITY ? 0.f : m_ref * c;
             const uint64_t nmc2 = f2_pack(-mc, -mc);
-            // P = 2^(s c - m c), written as 16-bit pairs over the first 64
+            // P = 2^(s c - m c), written as 16-bit pairs over the first BN/2
             // columns of the S buffer (keys [32h, 32h+32) -> columns [16h, 16h+16),
             // all of which were read above)
             uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
+            for (int h = 0; h < NCH; ++h) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
@@ -637,18 +647,18 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                 }
             }
             tc::wait_st();
-            if (p.kvcache && j == nk - 1 && j0 + kBN > N) {
+            if (p.kvcache && j == nk - 1 && j0 + BN > N) {
                 // cache rows past N_b may hold anything: zero them in the V tile
                 // (both tiles' warpgroups do it; the writes are identical)
                 const int vs = j % VST;
                 if (!(ok = mbar_wait(&v_full[vs], (j / VST) & 1, p.status))) break;
                 uint8_t *vt = sV + vs * C::VBYTES;
                 const int first = N - j0;
-                const int n16 = (kBN - first) * 8 * (D_V / 64);
+                const int n16 = (BN - first) * 8 * (D_V / 64);
                 for (int idx = threadIdx.x - 128 - 128 * x; idx < n16; idx += 128) {
-                    const int box = idx / ((kBN - first) * 8);
-                    const int rem = idx % ((kBN - first) * 8);
-                    *reinterpret_cast<uint4 *>(vt + box * C::BOX + (first + rem / 8) * 128 + (rem % 8) * 16) =
+                    const int box = idx / ((BN - first) * 8);
+                    const int rem = idx % ((BN - first) * 8);
+                    *reinterpret_cast<uint4 *>(vt + box * C::KBOX + (first + rem / 8) * 128 + (rem % 8) * 16) =
                         make_uint4(0, 0, 0, 0);
                 }
                 fence_proxy_async();
@@ -715,6 +725,11 @@ static cudaError_t run_prefill(const PrefillParams &p, const CUtensorMap &tmQ, c
 }
 
 #define FA_PREFILL_DIMS(X) X(64, 64) X(128, 128) X(192, 128) X(128, 64) X(64, 128) X(192, 64)
+
+int prefill_block_n(int d_qk, int d_v, int tiles_per_cta) {
+    (void)d_v;
+    return (tiles_per_cta == 2 && d_qk > 128) ? 96 : kBN;
+}
 
 bool prefill_supported(int d_qk, int d_v) {
 #define FA_CASE(DQ, DV) if (d_qk == DQ && d_v == DV) return true;
