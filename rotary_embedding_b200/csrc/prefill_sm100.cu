@@ -362,9 +362,10 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
 // Warps: 0 TMA, 1 MMA, 2-3 idle (warpgroup 0), 4-7 softmax of tile A
 // (warpgroup 1), 8-11 softmax of tile B (warpgroup 2); warp w reaches TMEM
 // lanes 32 (w % 4) .. 32 (w % 4) + 31.  The register file is split with
-// setmaxnreg: warpgroup 0 drops to 64 registers per thread, the two softmax
-// warpgroups rise to 216 so that a whole 128-column S row stays in registers
-// (128 x 64 + 256 x 216 = 63488, within the 384 x 168 the block is launched with).
+// setmaxnreg: warpgroup 0 drops to 96 registers per thread (the MMA issue loop
+// must not spill), the two softmax warpgroups rise to 200 so that a whole
+// 128-column S row stays in registers (128 x 96 + 256 x 200 = 63488, within
+// the 384 x 168 the block is launched with).
 // ============================================================================
 template <int D_QK, int D_V>
 struct Prefill2Cfg {
@@ -472,7 +473,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
 
-    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
+    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0 && n_all > 0) {
@@ -501,36 +502,55 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0 && n_all > 0) {
+        // The whole warp runs the loop (waits, warp-uniform descriptors); one
+        // elected lane issues the MMAs and the commits that track them.
+        if (n_all > 0) {
+            const bool leader = tc::elect_one();
             const uint32_t idesc_qk = tc::idesc_f16(bf16, kBM, BN, false);
             const uint32_t idesc_pv = tc::idesc_f16(bf16, kBM, D_V, true);
-            const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
+            // Descriptors of the first k-step of every operand buffer; a k-step
+            // only moves the start address (low 14 bits, 16-byte units), so the
+            // issue loop adds a compile-time constant per MMA.
+            const uint64_t dQ0 = tc::smem_desc(smem_addr(sQ), 16, 1024);
+            const uint64_t dK0 = tc::smem_desc(smem_addr(sK), 16, 1024);
+            const uint64_t dV0 = tc::smem_desc(smem_addr(sV), C::KBOX, 1024);
             bool ok = mbar_wait(q_full, 0, p.status);
             auto issue_qk = [&](int x, int j) {
-                const int ks = j % KST;
+                const uint64_t dq = dQ0 + (uint64_t)((x * C::QBYTES) >> 4);
+                const uint64_t dk = dK0 + (uint64_t)(((j % KST) * C::KBYTES) >> 4);
+                const uint32_t ts = tmem + C::t_s(x);
+                if (leader) {
 #pragma unroll
-                for (int k = 0; k < D_QK / 16; ++k) {
-                    const uint64_t adesc =
-                        tc::smem_desc(aQ + x * C::QBYTES + (k >> 2) * C::QBOX + (k & 3) * 32, 16, 1024);
-                    const uint64_t bdesc = tc::smem_desc(aK + ks * C::KBYTES + (k >> 2) * C::KBOX + (k & 3) * 32, 16, 1024);
-                    tc::mma_ss(tmem + C::t_s(x), adesc, bdesc, idesc_qk, k > 0 ? 1u : 0u);
+                    for (int k = 0; k < D_QK / 16; ++k) {
+                        const uint64_t qoff = (uint64_t)((((k >> 2) * C::QBOX) + (k & 3) * 32) >> 4);
+                        const uint64_t koff = (uint64_t)((((k >> 2) * C::KBOX) + (k & 3) * 32) >> 4);
+                        tc::mma_ss(ts, dq + qoff, dk + koff, idesc_qk, k > 0 ? 1u : 0u);
+                    }
+                    tc::commit(&s_full[x]);
                 }
-                tc::commit(&s_full[x]);
+                __syncwarp();
             };
             auto issue_pv = [&](int x, int j) {
-                const int vs = j % VST;
+                const uint64_t dv = dV0 + (uint64_t)(((j % VST) * C::VBYTES) >> 4);
+                const uint32_t to = tmem + C::t_o(x), tp = tmem + C::t_s(x);
+                const uint32_t acc0 = j > 0 ? 1u : 0u;
+                if (leader) {
 #pragma unroll
-                for (int k = 0; k < BN / 16; ++k) {
-                    const uint64_t bdesc = tc::smem_desc(aV + vs * C::VBYTES + k * 16 * 128, C::KBOX, 1024);
-                    tc::mma_ts(tmem + C::t_o(x), tmem + C::t_s(x) + k * 8, bdesc, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < BN / 16; ++k)
+                        tc::mma_ts(to, tp + k * 8, dv + (uint64_t)(k * 16 * 128 / 16), idesc_pv, k > 0 ? 1u : acc0);
                 }
+                __syncwarp();
+            };
+            auto commit = [&](uint64_t *bar) {
+                if (leader) tc::commit(bar);
+                __syncwarp();
             };
             // prologue: QK of both tiles on key tile 0
             if (ok && (ok = mbar_wait(&k_full[0], 0, p.status))) {
                 tc::fence_after_sync();
                 if (n_kv[0] > 0) issue_qk(0, 0);
                 if (n_kv[1] > 0) issue_qk(1, 0);
-                tc::commit(&k_empty[0]);
+                commit(&k_empty[0]);
             }
             for (int j = 0; j < n_all && ok; ++j) {
                 const int vs = j % VST;
@@ -544,18 +564,18 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                         if (!(ok = mbar_wait(&p_full[x], j & 1, p.status))) break;
                         tc::fence_after_sync();
                         issue_pv(x, j);
-                        if (j + 1 == n_kv[x]) tc::commit(&o_full[x]);
+                        if (j + 1 == n_kv[x]) commit(&o_full[x]);
                         if (j + 1 < n_kv[x]) issue_qk(x, j + 1);
                     }
                 }
                 if (!ok) break;
-                tc::commit(&v_empty[vs]);
-                if (next) tc::commit(&k_empty[ks1]);
+                commit(&v_empty[vs]);
+                if (next) commit(&k_empty[ks1]);
             }
         }
     } else if (warp >= 4) {
         // ------------------------------------------------ softmax warpgroups
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 216;" ::: "memory");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
         const int x = (warp - 4) >> 2;                 // tile of this warpgroup
         const int q4 = warp & 3;                       // TMEM lane quadrant this warp may access
         const int r = q4 * 32 + lane;                  // tile row = TMEM lane
