@@ -248,6 +248,32 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
+// 2^x for a pair of values on the FMA / integer pipes, leaving the special
+// function unit free (Cody-Waite reduction x = n + f, n = round(x),
+// f in [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial whose coefficients
+// exp2_poly.py derives by the Remez exchange; 2^n added to the exponent
+// field).  Maximum relative error 7.5e-5.  x is clamped to >= -126 first, so
+// very negative inputs give a result in [0, 2^-125] instead of exactly 0;
+// callers that need exact zeros (masked scores) use ex2().
+__device__ __forceinline__ uint64_t ex2_poly2(float x0, float x1) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: x + kMagic rounds x to an integer
+    x0 = fmaxf(x0, -126.0f);
+    x1 = fmaxf(x1, -126.0f);
+    const uint64_t x = f2_pack(x0, x1);
+    const uint64_t t = f2_add(x, f2_pack(kMagic, kMagic));
+    const uint64_t n = f2_add(t, f2_pack(-kMagic, -kMagic));
+    const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), x);           // x - n
+    uint64_t p = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f,
+                        f2_pack(0.2426111251115799f, 0.2426111251115799f));
+    p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+    p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+    // the low bits of t hold n (two's complement); shift it into the exponent
+    const uint32_t t_lo = static_cast<uint32_t>(t), t_hi = static_cast<uint32_t>(t >> 32);
+    const uint32_t p_lo = static_cast<uint32_t>(p), p_hi = static_cast<uint32_t>(p >> 32);
+    const uint32_t r_lo = p_lo + (t_lo << 23), r_hi = p_hi + (t_hi << 23);
+    return (static_cast<uint64_t>(r_hi) << 32) | r_lo;
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

@@ -33,6 +33,12 @@
 
 namespace fa {
 
+// Pairs out of every 8 whose 2^x the two-tile softmax evaluates on the FMA
+// pipe (ex2_poly2) instead of the special function unit, in unmasked tiles.
+#ifndef FA_EXP2_EMU_PAIRS
+#define FA_EXP2_EMU_PAIRS 3
+#endif
+
 constexpr int kBM = 128;  // query rows per CTA
 constexpr int kBN = 128;  // key rows per tile
 
@@ -634,27 +640,39 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             // P = 2^(s c - m c), written as 16-bit pairs over the first BN/2
             // columns of the S buffer (keys [32h, 32h+32) -> columns [16h, 16h+16),
             // all of which were read above)
-            uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+            // In tiles without masked keys, 6 of every 16 pairs take 2^x on the
+            // FMA pipe (ex2_poly2) and the rest on the special function unit,
+            // which alone would bound the softmax; masked tiles need exact
+            // zeros and use the special function unit throughout.
+            // The fp32 P values overwrite S in registers; the row sum is taken
+            // after P has been handed to the MMA warp (off the critical path).
+            auto exp_row = [&](auto split) {
 #pragma unroll
-            for (int h = 0; h < NCH; ++h) {
-                uint32_t pk[16];
+                for (int h = 0; h < NCH; ++h) {
+                    uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const uint64_t t = f2_fma(f2_pack(__uint_as_float(sr[h][e]), __uint_as_float(sr[h][e + 1])), c2, nmc2);
-                    float t0, t1;
-                    f2_unpack(t, t0, t1);
-                    const float p0 = ex2(t0), p1 = ex2(t1);
-                    const uint64_t pp = f2_pack(p0, p1);
-                    rs2[(e >> 1) & 1] = f2_add(rs2[(e >> 1) & 1], pp);
-                    pk[e >> 1] = Elem<T>::pack2(p0, p1);
+                    for (int e = 0; e < 32; e += 2) {
+                        const uint64_t t =
+                            f2_fma(f2_pack(__uint_as_float(sr[h][e]), __uint_as_float(sr[h][e + 1])), c2, nmc2);
+                        float t0, t1, p0, p1;
+                        f2_unpack(t, t0, t1);
+                        if (decltype(split)::value && ((e >> 1) & 7) < FA_EXP2_EMU_PAIRS) {
+                            f2_unpack(ex2_poly2(t0, t1), p0, p1);
+                        } else {
+                            p0 = ex2(t0);
+                            p1 = ex2(t1);
+                        }
+                        sr[h][e] = __float_as_uint(p0);
+                        sr[h][e + 1] = __float_as_uint(p1);
+                        pk[e >> 1] = Elem<T>::pack2(p0, p1);
+                    }
+                    tc::st16(s_addr + h * 16, pk);
                 }
-                tc::st16(s_addr + h * 16, pk);
-            }
-            float ra, rb, rc_, rd;
-            f2_unpack(rs2[0], ra, rb);
-            f2_unpack(rs2[1], rc_, rd);
-            const float rs = (ra + rb) + (rc_ + rd);
-            l = l * alpha + rs;
+            };
+            if (j0 + BN > mask_from[x])
+                exp_row(std::integral_constant<bool, false>());
+            else
+                exp_row(std::integral_constant<bool, true>());
             if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
                 for (int h = 0; h < D_V / 32; ++h) {
@@ -686,6 +704,20 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[x]);
+            // row sum of the fp32 P values (four independent packed chains)
+            uint64_t rs2[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int h = 0; h < NCH; ++h)
+#pragma unroll
+                for (int e = 0; e < 32; e += 2)
+                    rs2[(e >> 1) & 3] =
+                        f2_add(rs2[(e >> 1) & 3], f2_pack(__uint_as_float(sr[h][e]), __uint_as_float(sr[h][e + 1])));
+            float r0, r1, r2, r3, r4, r5, r6, r7;
+            f2_unpack(rs2[0], r0, r1);
+            f2_unpack(rs2[1], r2, r3);
+            f2_unpack(rs2[2], r4, r5);
+            f2_unpack(rs2[3], r6, r7);
+            l = l * alpha + (((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7)));
         }
         // ------------------------------------------------ epilogue
         if (ok && nk > 0 && !mbar_wait(&o_full[x], 0, p.status)) ok = false;
