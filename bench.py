@@ -135,11 +135,12 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- traffic record
-def traffic_record(kernel_tag: str):
-    """DRAM traffic per launch from the committed ncu summary of this kernel, if
-    it was taken on the current kernel source (its sha256 prefix must match)."""
+def traffic_record(config_key: str, kernel_tag: str):
+    """DRAM traffic per launch of the attention kernel on this workload, from
+    the committed ncu summary profiles/traffic_<workload>.md, if it was taken
+    on the current kernel source (its sha256 prefix must match)."""
     src = {"decode": "decode.cu", "prefill": "prefill_sm100.cu"}.get(kernel_tag)
-    summ = os.path.join(ROOT, "profiles", f"traffic_{kernel_tag}.md")
+    summ = os.path.join(ROOT, "profiles", f"traffic_{config_key}.md")
     if not src or not os.path.exists(summ):
         return None
     path = os.path.join(ROOT, "rotary_embedding_b200", "csrc", src)
@@ -147,11 +148,11 @@ def traffic_record(kernel_tag: str):
         return None
     sha = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
     text = open(summ).read()
-    m = re.search(r"source_sha256_16:\s*([0-9a-f]{16}).*?traffic_bytes_per_launch_full_size:\s*([0-9.eE+]+)",
-                  text, re.S)
-    if not m or m.group(1) != sha:
+    m = re.search(r"source_file:\s*(\S+).*?source_sha256_16:\s*([0-9a-f]{16}).*?"
+                  r"traffic_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text, re.S)
+    if not m or m.group(1) != src or m.group(2) != sha:
         return None
-    return float(m.group(2))
+    return float(m.group(3))
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -277,6 +278,37 @@ def aggregate_over_ranks(ms_local: float, amount: float, world: int, device):
     return ms_max, world * amount / (ms_max / 1e3)
 
 
+def time_kernel(fa, step, steps, flush_buf):
+    """Per-step duration (ms) of the attention kernel alone: CUDA events that
+    the library records on the launching stream right before and after that
+    kernel (fa_set_kernel_events), replayed from a CUDA graph so that no host
+    latency sits between the start event and the launch; L2 flushed before
+    every step.  None if the events cannot be timed."""
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    fa.fa_set_kernel_events(start, stop)
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+            step()
+    finally:
+        fa.fa_set_kernel_events()
+    torch.cuda.synchronize()
+    try:
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(steps):
+            flush_buf.zero_()
+            graph.replay()
+            torch.cuda.synchronize()
+            times.append(start.elapsed_time(stop))
+    except RuntimeError:
+        return None
+    return times
+
+
 def run_ours(args):
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -318,7 +350,9 @@ def run_ours(args):
                 graph.replay()
             torch.cuda.synchronize()
         times = time_steps(graph.replay, args.steps, max(args.warmup, 3), stream, flush_buf, barrier)
+        k_times = time_kernel(fa, step, args.steps, flush_buf)
     ms = sum(times) / len(times)
+    kernel_ms = sum(k_times) / len(k_times) if k_times else None
     ms_max, value = aggregate_over_ranks(ms, amount, world, device)
 
     e2e_value, h2d, d2h = None, 0, 0
@@ -334,9 +368,13 @@ def run_ours(args):
         peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     else:
         peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    achieved = amount / (ms / 1e3)   # this rank, per launch of the call
+    # algorithmic amount of one call / the attention kernel's own duration
+    # (the whole call's duration if the kernel events could not be timed)
+    achieved = amount / ((kernel_ms if kernel_ms else ms) / 1e3)
     kernel_tag = "decode" if plan["path"] == fa.FA_PATH_DECODE else "prefill"
-    traffic = traffic_record(kernel_tag)
+    kernel_name = {fa.FA_PATH_DECODE: "decode_kernel", fa.FA_PATH_PREFILL: "prefill2_kernel / prefill_kernel",
+                   fa.FA_PATH_DENSE: "prefill2_kernel / prefill_kernel"}.get(plan["path"], "attention kernel")
+    traffic = traffic_record(args.config, kernel_tag)
     result = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -360,8 +398,11 @@ def run_ours(args):
         "roofline": {"bound": bound, "achieved": round(achieved, 3), "peak": peak,
                      "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": f"{peaks_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
-                     "kernel": ("decode_kernel (+combine_kernel in the same timed call)"
-                                if kernel_tag == "decode" else "whole call"),
+                     "kernel": kernel_name,
+                     "kernel_ms": round(kernel_ms, 5) if kernel_ms else None,
+                     "timing": ("CUDA events around the kernel's launch on its stream, graph replay, "
+                                "L2 flushed per step" if kernel_ms else "whole call (kernel events unavailable)"),
+                     "call_ms": round(ms, 5),
                      "amount_per_launch": amount},
         "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

@@ -213,6 +213,22 @@ int fa_fwd_plan(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, fa_p
  * synchronising `stream`; *status receives FA_OK or an FA_ERR_DEVICE_* code. */
 int fa_device_status(void *stream, int32_t *status);
 
+/* Profiling hook; the pages have no counterpart (it exists so that a
+ * benchmark can time the attention kernel alone, apart from the RoPE/append
+ * kernel before it and the split-combine kernel after it).
+ *  - start, stop: cudaEvent_t handles created by the caller with timing
+ *    enabled, or both NULL to switch the hook off.  The library does not own
+ *    them; the caller keeps them alive while the hook is on.
+ *  - While set, every fa_kvcache_fwd / fa_kvcache_fwd_noalloc / fa_fwd call
+ *    records `start` on its stream just before the launch of its attention
+ *    kernel (decode, prefill or generic) and `stop` just after it (inside a
+ *    stream capture as external event-record nodes).  The events sit between
+ *    the decode and combine kernels, so while the hook is on the combine
+ *    launch no longer overlaps the decode kernel's tail.
+ *  - Process-wide state, not synchronised: set it while no other thread is
+ *    calling the library.  Returns FA_ERR_INVALID_ARG if exactly one is NULL. */
+int fa_set_kernel_events(void *start, void *stop);
+
 /* Static message for a status code. */
 const char *fa_status_string(int status);
 

@@ -71,6 +71,8 @@ lib.fa_last_error.argtypes = []
 lib.fa_last_error.restype = ctypes.c_char_p
 lib.fa_version.argtypes = []
 lib.fa_version.restype = ctypes.c_int
+lib.fa_set_kernel_events.argtypes = [_v, _v]
+lib.fa_set_kernel_events.restype = ctypes.c_int
 
 
 def describe(t: torch.Tensor | None):
@@ -250,3 +252,18 @@ def fa_device_status(stream=None) -> int:
 
 def fa_version() -> int:
     return lib.fa_version()
+
+
+def fa_set_kernel_events(start=None, stop=None) -> None:
+    """Profiling hook: record `start` / `stop` (torch.cuda.Event, timing
+    enabled) around the attention kernel of every following call, or switch
+    it off with no arguments.  Both events are recorded once here on the
+    current stream so that their CUDA handles exist."""
+    if start is None and stop is None:
+        _check(lib.fa_set_kernel_events(None, None))
+        return
+    if start is None or stop is None:
+        raise ValueError("pass both events or neither")
+    start.record()
+    stop.record()
+    _check(lib.fa_set_kernel_events(ctypes.c_void_p(start.cuda_event), ctypes.c_void_p(stop.cuda_event)))

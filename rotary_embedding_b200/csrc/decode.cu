@@ -634,8 +634,10 @@ static cudaError_t run_decode(const DecodeParams &p_in, const CUtensorMap &tmK, 
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D_QK, D_V, MT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    kernel_event(0, st);
     decode_kernel<T, D_QK, D_V, MT><<<sm_count() * DecodeOcc<D_V, MT>::CTAS, 160, smem, st>>>(tmK, tmV, p);
     e = cudaGetLastError();
+    kernel_event(1, st);
     if (e != cudaSuccess) return e;
     if (p.n_splits > 1) {
         const int64_t warps = (int64_t)p.b * p.h_q * p.s_q;

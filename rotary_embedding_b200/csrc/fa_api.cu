@@ -325,6 +325,19 @@ int validate_kvcache(const fa_tensor *q, const fa_tensor *k_cache, const fa_tens
 
 int set_last_error(int code, const char *msg) { return fail(code, "%s", msg); }
 
+static cudaEvent_t g_kernel_events[2] = {nullptr, nullptr};
+
+void kernel_event(int which, cudaStream_t st) {
+    cudaEvent_t ev = g_kernel_events[which];
+    if (!ev) return;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(st, &cs);
+    if (cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, st);
+}
+
 }  // namespace fa
 
 using namespace fa;
@@ -332,6 +345,14 @@ using namespace fa;
 extern "C" {
 
 int fa_version(void) { return 100; }
+
+int fa_set_kernel_events(void *start, void *stop) {
+    if ((start == nullptr) != (stop == nullptr))
+        return fail(FA_ERR_INVALID_ARG, "fa_set_kernel_events: pass both events or neither");
+    g_kernel_events[0] = static_cast<cudaEvent_t>(start);
+    g_kernel_events[1] = static_cast<cudaEvent_t>(stop);
+    return FA_OK;
+}
 
 const char *fa_last_error(void) { return g_last_error; }
 

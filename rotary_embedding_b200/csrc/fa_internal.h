@@ -112,6 +112,10 @@ int sm_count();
 // Sets the thread-local message fa_last_error() returns; returns `code`.
 int set_last_error(int code, const char *msg);
 
+// Records the caller's profiling event (fa_set_kernel_events) on `st`, if set:
+// which = 0 before the attention kernel's launch, 1 after it.
+void kernel_event(int which, cudaStream_t st);
+
 cudaError_t launch_rope_append(const RopeAppendParams &p, int dtype, cudaStream_t st);
 bool prefill_supported(int d_qk, int d_v);
 int prefill_block_n(int d_qk, int d_v, int tiles_per_cta);  // key rows per K/V tile (TMA box rows)

@@ -764,16 +764,22 @@ static cudaError_t run_prefill(const PrefillParams &p, const CUtensorMap &tmQ, c
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C2::SMEM);
         if (e != cudaSuccess) return e;
         dim3 grid((p.n_q_tiles + 1) / 2, p.h_q / p.pack, p.b);
+        kernel_event(0, st);
         prefill2_kernel<T, D_QK, D_V><<<grid, 384, C2::SMEM, st>>>(tmQ, tmK, tmV, p);
-        return cudaGetLastError();
+        e = cudaGetLastError();
+        kernel_event(1, st);
+        return e;
     }
     using C = PrefillCfg<D_QK, D_V>;
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel<T, D_QK, D_V>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(p.n_q_tiles, p.h_q / p.pack, p.b);
+    kernel_event(0, st);
     prefill_kernel<T, D_QK, D_V><<<grid, 256, C::SMEM, st>>>(tmQ, tmK, tmV, p);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    kernel_event(1, st);
+    return e;
 }
 
 #define FA_PREFILL_DIMS(X) X(64, 64) X(128, 128) X(192, 128) X(128, 64) X(64, 128) X(192, 64)

@@ -104,11 +104,14 @@ cudaError_t launch_simt_attn(const SimtAttnParams &p, int dtype, cudaStream_t st
     if (warps == 0) return cudaSuccess;
     const int64_t blocks = (warps * 32 + 255) / 256;
     const size_t smem = 8 * p.d_qk * sizeof(float);
+    kernel_event(0, st);
     if (dtype == FA_DTYPE_F16)
         simt_attn_kernel<__half><<<(unsigned)blocks, 256, smem, st>>>(p);
     else
         simt_attn_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, smem, st>>>(p);
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    kernel_event(1, st);
+    return e;
 }
 
 }  // namespace fa

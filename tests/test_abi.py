@@ -168,3 +168,10 @@ def test_fa_fwd_validation():
     rc = fa.lib.fa_fwd(ctypes.byref(d(q)), ctypes.byref(d(k)), ctypes.byref(d(v)), 1, 0.0,
                        ctypes.byref(d(out)), None, None, 0, None)
     assert rc == fa.FA_ERR_INVALID_ARG
+
+
+def test_kernel_events_hook_arguments():
+    # both or neither: a lone event is rejected, clearing is always allowed
+    assert fa.lib.fa_set_kernel_events(ctypes.c_void_p(16), None) == fa.FA_ERR_INVALID_ARG
+    assert fa.lib.fa_set_kernel_events(None, ctypes.c_void_p(16)) == fa.FA_ERR_INVALID_ARG
+    assert fa.lib.fa_set_kernel_events(None, None) == fa.FA_OK
