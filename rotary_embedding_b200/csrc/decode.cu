@@ -1,29 +1,40 @@
-// decode.cu -- persistent split-KV decode attention with fused RoPE + cache
-// append, and the LSE combine of the split partials.
+// decode.cu -- persistent split-KV decode attention over the KV cache, and
+// the LSE combine of the split partials.
 //
 // Path (the single-token / short-chunk branch of the attention-with-KV-cache
 // call: s2.cpp PR #40's eval_cached decode branch, flash_attn_with_kvcache of
-// flash-attention issue #1402 with a short new chunk):
+// flash-attention issue #1402 with a short new chunk).  The RoPE/append
+// kernel runs first on the same stream: it rotates q into the workspace,
+// writes the rotated new key rows and the new value rows into the cache, and
+// zeroes the work-pool counter.  This kernel is launched as its programmatic
+// dependent, so its CTAs start while that kernel is still running; the
+// producer waits for it (griddepcontrol) only before loading q or a tile that
+// holds new rows, and before touching the pool counter.
 //  * Work is the key rows of every (batch, kv head) segment, N_b = L_b + s_new
-//    rows each, cut into 64-row items.  One CTA per SM; CTA c takes the items
-//    whose first row falls in [c R / G, (c+1) R / G) of the concatenated rows
-//    R (computed on the device from cache_seqlens), so every SM streams the
-//    same number of bytes whatever the mix of sequence lengths.  A CTA's items
-//    form runs ("pieces") of consecutive rows of one segment; each piece is one
-//    online-softmax pass.
+//    rows each, cut into n_b 64-row items.  The last floor(n_b / 4) items of
+//    every segment form the pool; the rest is split statically: CTA c takes
+//    the static items whose first row falls in [c R_s / G, (c+1) R_s / G) of
+//    the concatenated static rows R_s (computed on the device from
+//    cache_seqlens).  When its static share is done a CTA claims 2-item chunks
+//    of the pool (segment tails, in segment order) with an atomic counter, so
+//    SMs that stream faster take more of the tail.  A CTA's items form runs
+//    ("pieces") of consecutive rows of one segment; a piece ends where the
+//    segment, the segment's static part, the static share or a chunk ends,
+//    and each piece is one online-softmax pass.
 //  * All g * s_q query rows that read a kv head (grouped-query heads of the
 //    "optimizing-attention-flash" page, Workflow 2 Step 3) share one 16- or
 //    32-row MMA tile, so each key/value row is read from HBM once.
-//  * Warp 4 streams 64-row K and V tiles with TMA (swizzled boxes) through a
-//    ring of shared-memory stages across item and piece boundaries; warps 0-3
-//    each take 16 keys of every tile, keep their own running max / sum /
-//    output, and merge at the end of a piece while the ring keeps filling.
-//  * The tile holding rows >= L_b is patched in shared memory by the warp that
-//    owns those keys: new key rows are rotated (the same rotation as the
-//    append kernel) and rounded, new value rows copied, both written to the
-//    cache (the only writer of those rows); rows >= N_b are zeroed so garbage
-//    past the sequence cannot reach the PV product.
-//  * q rows are rotated at position L_b + i while being staged.
+//  * Warp 4 is the only warp that touches global memory while the stream
+//    runs: it loads every piece's rotated q rows (a two-buffer ring) and the
+//    64-row K and V tiles (a ring of stages) with TMA, and posts each stage's
+//    item in shared memory.  Warps 0-3 each take 16 keys of every tile, keep
+//    their own running max / sum / output, and merge at the end of a piece.
+//    (With HBM saturated by the stream, an ordinary load or store issued by a
+//    consumer warp waits behind the queued tile requests for microseconds, so
+//    consumers issue none until a piece ends.)
+//  * Rows >= N_b of a segment's last tile are zeroed in shared memory by the
+//    warp that owns them, so whatever the cache holds past the sequence
+//    cannot reach the PV product (their scores are masked to -inf).
 //  * A segment that fits one item writes out / lse directly.  Otherwise every
 //    piece writes its normalised output and lse to the slot of its first item
 //    and lse = -inf to the slots of its other items; the combine kernel merges
@@ -41,7 +52,10 @@ namespace fa {
 
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-constexpr int kDecodeTile = 64;   // key rows per tile and per item
+constexpr int kDecodeTile = 64;        // key rows per tile and per item
+constexpr int kPoolChunk = 2;          // items per claim from the pool
+constexpr int kPoolDen = 4;            // the pool holds floor(n_b / 4) items of each segment
+
 // CTAs per SM: two when the per-thread state is small enough (one row tile,
 // d_v <= 128), so that one CTA's piece merge overlaps the other's stream.
 template <int D_V, int MT>
@@ -52,9 +66,18 @@ struct DecodeOcc {
 
 constexpr int kDecodeMaxStages = 8;
 
-// Shared memory: rotated q tile | ring of K/V stages | merge scratch for the
-// M live query rows | barriers.  The stage count is chosen at launch from the
-// budget left after the (runtime-sized) merge scratch.
+// The item of one stage, posted by the producer before the stage's TMA.
+struct StageItem {
+    int b, hk, s, flags;
+};
+constexpr int kPieceStart = 1, kPieceEnd = 2, kEndOfStream = 4;
+
+// Shared memory: two q buffers | ring of K/V stages | merge scratch for the
+// M live query rows | barriers, stage items, schedule, per-batch table.  A q
+// buffer holds QT = M rounded up to 8 rows per 64-column box (the TMA writes
+// the M live rows; the MMA tile reads up to 16 * MT rows, and rows >= M only
+// feed output rows that are never written).  The stage count is chosen at
+// launch from the budget left.
 template <int D_QK, int D_V, int MT>
 struct DecodeCfg {
     static constexpr int TILE = kDecodeTile;
@@ -62,20 +85,27 @@ struct DecodeCfg {
     static constexpr int VBYTES = TILE * D_V * 2;
     static constexpr int STAGE = KBYTES + VBYTES;
     static constexpr int QROWS = MT * 16;
-    static constexpr int QBYTES = ((QROWS * D_QK * 2 + 1023) / 1024) * 1024;
     static_assert(D_QK % 16 == 0 && D_V % 16 == 0, "head dims are multiples of 16");
+    __host__ __device__ static int qt(int M) { return (M + 7) / 8 * 8; }
+    __host__ __device__ static int qbuf_bytes(int M) { return (qt(M) * D_QK * 2 + 1023) / 1024 * 1024; }
     static int merge_bytes(int M) { return 4 * M * (D_V + 2) * 4; }
-    // barriers, the 4-int schedule and the per-batch (L, N, items) table
-    static int tail_bytes(int B) { return 2 * kDecodeMaxStages * 8 + 16 + 12 * B + 16; }
+    // ring and q barriers, stage items, the 4-int64 schedule, the per-batch table
+    static int tail_bytes(int B) {
+        return (2 * kDecodeMaxStages + 4) * 8 + kDecodeMaxStages * 16 + 32 + 12 * B + 16;
+    }
     static int stages(int M, int B) {
-        const int raw = (DecodeOcc<D_V, MT>::BUDGET - 1024 - QBYTES - merge_bytes(M) - tail_bytes(B)) / STAGE;
+        const int raw =
+            (DecodeOcc<D_V, MT>::BUDGET - 1024 - 2 * qbuf_bytes(M) - merge_bytes(M) - tail_bytes(B)) / STAGE;
         return raw < 2 ? 2 : (raw > kDecodeMaxStages ? kDecodeMaxStages : raw);
     }
-    static int smem(int M, int B) { return 1024 + QBYTES + stages(M, B) * STAGE + merge_bytes(M) + tail_bytes(B); }
+    static int smem(int M, int B) {
+        return 1024 + 2 * qbuf_bytes(M) + stages(M, B) * STAGE + merge_bytes(M) + tail_bytes(B);
+    }
 };
 
 // Per-batch facts every thread can recompute: rows N_b and items n_b (0 when
-// the batch entry violates the device-side preconditions).
+// the batch entry violates the device-side preconditions, which the
+// RoPE/append kernel records and skips in the same way).
 struct SegInfo {
     int L, N, n_items;
 };
@@ -91,91 +121,123 @@ __device__ __forceinline__ SegInfo seg_info(const DecodeParams &p, int b) {
     return s;
 }
 
-// Iterator over the items (b, hk, s) in segment order.
+// Items [0, ns) of a segment are split statically, [ns, n) are in the pool.
+__device__ __forceinline__ int pool_items(int n) { return n / kPoolDen; }
+__device__ __forceinline__ int static_items(int n) { return n - pool_items(n); }
+// Rows of a segment's static part (all of it when the pool holds none).
+__device__ __forceinline__ int static_rows(const SegInfo &sg) {
+    return pool_items(sg.n_items) > 0 ? static_items(sg.n_items) * kDecodeTile : sg.N;
+}
+
+// An item (b, hk, s) and its segment; POOL selects which items of a segment
+// the iteration visits ([0, ns) or [ns, n)).
 struct ItemIter {
     int b, hk, s;
     SegInfo seg;
 };
 
-// `tab` is the per-batch SegInfo table the CTA staged in shared memory.
+template <bool POOL>
+__device__ __forceinline__ int part_first(const SegInfo &sg) { return POOL ? static_items(sg.n_items) : 0; }
+template <bool POOL>
+__device__ __forceinline__ int part_end(const SegInfo &sg) { return POOL ? sg.n_items : static_items(sg.n_items); }
+template <bool POOL>
+__device__ __forceinline__ int part_count(const SegInfo &sg) { return part_end<POOL>(sg) - part_first<POOL>(sg); }
+
+// Next item of the same part, in (batch, kv head, item) order.
+template <bool POOL>
 __device__ __forceinline__ void iter_advance(const DecodeParams &p, const SegInfo *tab, ItemIter &it) {
-    if (++it.s < it.seg.n_items) return;
-    it.s = 0;
-    if (++it.hk < p.h_kv) return;
+    if (++it.s < part_end<POOL>(it.seg)) return;
+    if (++it.hk < p.h_kv) {
+        it.s = part_first<POOL>(it.seg);
+        return;
+    }
     it.hk = 0;
     do {
         ++it.b;
         if (it.b >= p.b) return;
         it.seg = tab[it.b];
-    } while (it.seg.n_items == 0);
+    } while (part_count<POOL>(it.seg) == 0);
+    it.s = part_first<POOL>(it.seg);
 }
 
-// Global index of the first item whose first row is >= X in the concatenated
-// row space, and the CTA's item range [I(c R/G), I((c+1) R/G)).
-__device__ void cta_item_range(const DecodeParams &p, const SegInfo *tab, int c, int G, ItemIter &first,
-                               int &n_items) {
-    int64_t R = 0;
-    for (int b = 0; b < p.b; ++b) R += (int64_t)p.h_kv * tab[b].N;
-    const int64_t X0 = R * c / G, X1 = R * (c + 1) / G;
-    int64_t I0 = -1, I1 = -1, items_before = 0, rows_before = 0;
-    first.b = p.b;
-    for (int b = 0; b < p.b && I1 < 0; ++b) {
+// Index (among all static items) of the first static item whose first row is
+// >= X in the concatenated static rows (the static item count if none).
+__device__ int64_t static_item_at_row(const DecodeParams &p, const SegInfo *tab, int64_t X) {
+    int64_t items_before = 0, rows_before = 0;
+    for (int b = 0; b < p.b; ++b) {
         const SegInfo sg = tab[b];
-        const int64_t seg_rows = (int64_t)p.h_kv * sg.N;
-        for (int which = 0; which < 2; ++which) {
-            const int64_t X = which ? X1 : X0;
-            int64_t &I = which ? I1 : I0;
-            if (I >= 0 || X >= rows_before + seg_rows) continue;
+        const int rs = static_rows(sg), ns = static_items(sg.n_items);
+        const int64_t seg_rows = (int64_t)p.h_kv * rs;
+        if (X < rows_before + seg_rows) {
             const int64_t off = X - rows_before;
-            const int64_t hk = off / sg.N, within = off - hk * sg.N;
-            I = items_before + hk * sg.n_items + (within + kDecodeTile - 1) / kDecodeTile;
-            if (which == 0) {
-                // decode I0 into (b, hk, s), rolling over to the next item if needed
-                first.b = b;
-                first.hk = (int)hk;
-                first.s = (int)((within + kDecodeTile - 1) / kDecodeTile);
-                first.seg = sg;
-                if (first.s >= sg.n_items) {
-                    first.s = sg.n_items - 1;
-                    iter_advance(p, tab, first);
-                }
-            }
+            const int64_t hk = off / rs, within = off - hk * rs;
+            return items_before + hk * ns + (within + kDecodeTile - 1) / kDecodeTile;
         }
-        items_before += (int64_t)p.h_kv * sg.n_items;
+        items_before += (int64_t)p.h_kv * ns;
         rows_before += seg_rows;
     }
-    if (I0 < 0) I0 = items_before;
-    if (I1 < 0) I1 = items_before;
-    n_items = (int)(I1 - I0);
+    return items_before;
 }
 
+// Position of the I-th item of a part, advancing a batch cursor (cb, items of
+// the part before batch cb) that only moves forward.
+template <bool POOL>
+__device__ __forceinline__ ItemIter part_item(const DecodeParams &p, const SegInfo *tab, int64_t I, int &cb,
+                                              int64_t &cb_items) {
+    while (cb < p.b && cb_items + (int64_t)p.h_kv * part_count<POOL>(tab[cb]) <= I) {
+        cb_items += (int64_t)p.h_kv * part_count<POOL>(tab[cb]);
+        ++cb;
+    }
+    ItemIter it;
+    it.b = cb;
+    it.seg = tab[cb];
+    const int cnt = part_count<POOL>(it.seg);
+    const int64_t off = I - cb_items;
+    it.hk = (int)(off / cnt);
+    it.s = part_first<POOL>(it.seg) + (int)(off - (int64_t)it.hk * cnt);
+    return it;
+}
+
+// Wait until the grid this kernel depends on (the RoPE/append kernel) has
+// completed and its writes are visible; returns at once without one.
+__device__ __forceinline__ void wait_prerequisite_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 template <typename T, int D_QK, int D_V, int MT>
-__global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(const __grid_constant__ CUtensorMap tmK,
-                                                        const __grid_constant__ CUtensorMap tmV,
-                                                        const DecodeParams p) {
+__global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS)
+    decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const DecodeParams p) {
     using C = DecodeCfg<D_QK, D_V, MT>;
     constexpr int CHK = box_cols(D_QK), RBK = box_row_bytes(D_QK);
     constexpr int CHV = box_cols(D_V), RBV = box_row_bytes(D_V);
-    constexpr int CK = D_QK / 8, CV = D_V / 8;
+    constexpr int CV = D_V / 8;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int M = p.g * p.s_q;
+    const int QT = C::qt(M);
+    const int QBUF = C::qbuf_bytes(M);
     const int NST = p.n_stages;
-    uint8_t *sQ = smem;
-    uint8_t *sStage = smem + C::QBYTES;
+    uint8_t *sQ = smem;                       // [2][QBUF]
+    uint8_t *sStage = smem + 2 * QBUF;
     float *red_o = reinterpret_cast<float *>(sStage + NST * C::STAGE);   // [4][M][D_V]
     float *red_m = red_o + 4 * M * D_V;                                   // [4][M]
     float *red_l = red_m + 4 * M;                                         // [4][M]
     uint64_t *full = reinterpret_cast<uint64_t *>(red_l + 4 * M);
     uint64_t *empty = full + kDecodeMaxStages;
-    int *sched = reinterpret_cast<int *>(empty + kDecodeMaxStages);   // b, hk, s, n_items
-    SegInfo *tab = reinterpret_cast<SegInfo *>(sched + 4);             // [b]
+    uint64_t *q_full = empty + kDecodeMaxStages;   // [2]
+    uint64_t *q_empty = q_full + 2;                // [2]
+    StageItem *items = reinterpret_cast<StageItem *>(q_empty + 2);            // [kDecodeMaxStages]
+    int64_t *sched = reinterpret_cast<int64_t *>(items + kDecodeMaxStages);   // I0, n_static, pool, total
+    SegInfo *tab = reinterpret_cast<SegInfo *>(sched + 4);                    // [b]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const bool inter = p.interleaved != 0;
 
     // allow the combine kernel (launched as a programmatic dependent) to get scheduled
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (threadIdx.x == 128) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
 
     // stage every batch entry's (L, N, items) once, with parallel loads
     for (int b = threadIdx.x; b < p.b; b += blockDim.x) tab[b] = seg_info(p, b);
@@ -185,16 +247,29 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 4);
         }
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(&q_full[q], 1);
+            mbar_init(&q_empty[q], 4);
+        }
         fence_barrier_init();
-        ItemIter first;
-        int n_items;
-        cta_item_range(p, tab, blockIdx.x, gridDim.x, first, n_items);
-        sched[0] = first.b;
-        sched[1] = first.hk;
-        sched[2] = first.s;
-        sched[3] = n_items;
+        int64_t Rs = 0, n_pool = 0, n_all = 0;
+        for (int b = 0; b < p.b; ++b) {
+            Rs += (int64_t)p.h_kv * static_rows(tab[b]);
+            n_pool += (int64_t)p.h_kv * pool_items(tab[b].n_items);
+            n_all += (int64_t)p.h_kv * tab[b].n_items;
+        }
+        const int c = blockIdx.x, G = gridDim.x;
+        const int64_t I0 = static_item_at_row(p, tab, Rs * c / G);
+        sched[0] = I0;
+        sched[1] = static_item_at_row(p, tab, Rs * (c + 1) / G) - I0;
+        sched[2] = n_pool;
+        sched[3] = n_all;
     }
-    if (blockIdx.x == 0) {
+    __syncthreads();
+    const int64_t I_static = sched[0];
+    const int n_static = (int)sched[1];
+    const int64_t n_pool = sched[2], T_items = sched[3];
+    if (blockIdx.x == 0 && threadIdx.x < 128) {
         // batch entries with no key at all: out = 0, lse = -inf; bad entries: record
         for (int b = 0; b < p.b; ++b) {
             const SegInfo sg = tab[b];
@@ -206,7 +281,7 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
                 if (threadIdx.x == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
                 continue;
             }
-            for (int idx = threadIdx.x; idx < p.h_q * p.s_q * CV; idx += blockDim.x) {
+            for (int idx = threadIdx.x; idx < p.h_q * p.s_q * CV; idx += 128) {
                 const int c = idx % CV, row = idx / CV;
                 const int hq = row / p.s_q, i = row % p.s_q;
                 T *dst = static_cast<T *>(p.out) + b * p.os.b + i * p.os.s + hq * p.os.h;
@@ -215,79 +290,151 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
             }
         }
     }
-    __syncthreads();
-    const int n_items = sched[3];
-    if (n_items == 0) return;
-    ItemIter it0;
-    it0.b = sched[0];
-    it0.hk = sched[1];
-    it0.s = sched[2];
-    it0.seg = tab[it0.b];
+    if (T_items == 0) return;
 
     if (warp == 4) {
-        // ---------------- producer: TMA stream of K/V tiles over all items ----------------
+        // ---------------- producer: TMA stream of q rows and K/V tiles ----------------
         if (lane == 0) {
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            ItemIter it = it0;
-            int t = 0;
-            bool ok = true;
-            for (int k = 0; k < n_items && ok; ++k) {
-                const int row0 = it.s * C::TILE;
-                const int s = t % NST;
-                if (t >= NST && !mbar_wait(&empty[s], ((t / NST) - 1) & 1, p.status)) {
-                    ok = false;
-                    break;
+            // the cache is read once: evict its lines first, keeping the
+            // partial results (and everything else) in L2
+            const uint64_t stream_policy = l2_evict_first_policy();
+            bool waited = false;   // prerequisite grid (RoPE/append) known complete
+            auto ensure_waited = [&]() {
+                if (!waited) {
+                    wait_prerequisite_grid();
+                    waited = true;
                 }
+            };
+            int qi = 0;            // q tiles issued
+            // q rows of the piece that starts at `pc`, into buffer qi % 2
+            auto issue_q = [&](const ItemIter &pc) {
+                const int qb = qi & 1;
+                if (qi >= 2 && !mbar_wait(&q_empty[qb], ((qi >> 1) - 1) & 1, p.status)) return false;
+                ensure_waited();
+                mbar_arrive_expect_tx(&q_full[qb], (uint32_t)(M * D_QK * 2));
+                uint8_t *qd = sQ + qb * QBUF;
+#pragma unroll
+                for (int c = 0; c < D_QK / CHK; ++c)
+                    tma_load_4d(qd + c * QT * RBK, &tmQ, &q_full[qb], c * CHK, pc.hk * p.g, 0, pc.b);
+                ++qi;
+                return true;
+            };
+            int k = 0;              // stages issued
+            ItemIter first_piece;   // the first piece's q goes out after the first tiles
+            first_piece.b = -1;
+            bool q0_issued = false;
+            auto issue_first_q = [&]() {
+                if (q0_issued || first_piece.b < 0) return true;
+                q0_issued = true;
+                return issue_q(first_piece);
+            };
+            // one stage: the item's K/V tile, after the q of a new piece
+            auto issue_item = [&](const ItemIter &itm, int flags) {
+                if (flags & kPieceStart) {
+                    if (first_piece.b < 0) {
+                        first_piece = itm;
+                    } else {
+                        if (!issue_first_q()) return false;
+                        if (!issue_q(itm)) return false;
+                    }
+                }
+                const int row0 = itm.s * C::TILE;
+                // rows >= L of this tile were written by the RoPE/append kernel
+                if (p.s_new > 0 && row0 + C::TILE > itm.seg.L) ensure_waited();
+                const int s = k % NST;
+                if (k >= NST && !mbar_wait(&empty[s], ((k / NST) - 1) & 1, p.status)) return false;
+                items[s] = StageItem{itm.b, itm.hk, itm.s, flags};
                 mbar_arrive_expect_tx(&full[s], C::STAGE);
                 uint8_t *kd = sStage + s * C::STAGE;
                 uint8_t *vd = kd + C::KBYTES;
 #pragma unroll
                 for (int c = 0; c < D_QK / CHK; ++c)
-                    tma_load_4d(kd + c * C::TILE * RBK, &tmK, &full[s], c * CHK, it.hk, row0, it.b);
+                    tma_load_4d_hint(kd + c * C::TILE * RBK, &tmK, &full[s], c * CHK, itm.hk, row0, itm.b, stream_policy);
 #pragma unroll
                 for (int c = 0; c < D_V / CHV; ++c)
-                    tma_load_4d(vd + c * C::TILE * RBV, &tmV, &full[s], c * CHV, it.hk, row0, it.b);
-                ++t;
-                iter_advance(p, tab, it);
+                    tma_load_4d_hint(vd + c * C::TILE * RBV, &tmV, &full[s], c * CHV, itm.hk, row0, itm.b, stream_policy);
+                ++k;
+                // the old cache rows of the first stages are in flight before q
+                if (k == NST && !issue_first_q()) return false;
+                return true;
+            };
+            bool ok = true;
+            int cb = 0;            // batch cursor of part_item
+            int64_t cb_items = 0;
+            int grab = -1;         // claimed pool chunk, or -1
+            // static share
+            if (n_static > 0) {
+                ItemIter it = part_item<false>(p, tab, I_static, cb, cb_items);
+                for (int i = 0; i < n_static && ok; ++i) {
+                    // claim the first pool chunk at the last item of the share
+                    if (i == n_static - 1) {
+                        ensure_waited();
+                        grab = atomicAdd(p.pool, 1);
+                    }
+                    const int flags = ((i == 0 || it.s == 0) ? kPieceStart : 0) |
+                                      ((i == n_static - 1 || it.s + 1 == static_items(it.seg.n_items)) ? kPieceEnd : 0);
+                    ok = issue_item(it, flags);
+                    iter_advance<false>(p, tab, it);
+                }
+            }
+            // pool chunks
+            cb = 0;
+            cb_items = 0;
+            while (ok) {
+                if (grab < 0) {
+                    ensure_waited();
+                    grab = atomicAdd(p.pool, 1);
+                }
+                const int64_t J0 = (int64_t)grab * kPoolChunk;
+                if (J0 >= n_pool) break;
+                const int64_t J1 = J0 + kPoolChunk < n_pool ? J0 + kPoolChunk : n_pool;
+                ItemIter it = part_item<true>(p, tab, J0, cb, cb_items);
+                int next = -1;
+                for (int64_t J = J0; J < J1 && ok; ++J) {
+                    // claim the next chunk at this chunk's last item; its index
+                    // is read after the item is issued
+                    if (J == J1 - 1) next = atomicAdd(p.pool, 1);
+                    const int flags = ((J == J0 || it.s == static_items(it.seg.n_items)) ? kPieceStart : 0) |
+                                      ((J == J1 - 1 || it.s + 1 == it.seg.n_items) ? kPieceEnd : 0);
+                    ok = issue_item(it, flags);
+                    iter_advance<true>(p, tab, it);
+                }
+                grab = next;
+            }
+            if (ok) ok = issue_first_q();
+            if (ok) {
+                // end of stream: an item-less stage
+                const int s = k % NST;
+                if (k < NST || mbar_wait(&empty[s], ((k / NST) - 1) & 1, p.status)) {
+                    items[s] = StageItem{0, 0, 0, kEndOfStream};
+                    mbar_arrive(&full[s]);
+                }
             }
         }
         return;
     }
 
     // ---------------- consumers ----------------
-    const T *cos_t = static_cast<const T *>(p.cos);
-    const T *sin_t = static_cast<const T *>(p.sin);
-    const uint32_t sQa = smem_addr(sQ);
     float o[MT][D_V / 8][4];
     float m_r[MT][2], l_r[MT][2];
     int last_vis[MT][2];
     int s_first = 0;
-    bool timed_out = false;
-    ItemIter it = it0;
-    for (int k = 0; k < n_items; ++k) {
-        const int b = it.b, hk = it.hk;
-        const int L = it.seg.L, N = it.seg.N;
-        const int hq0 = hk * p.g;
-        const bool piece_start = (k == 0) || it.s == 0;
-        if (piece_start) {
-            s_first = it.s;
-            // stage the rotated q rows of this (batch, kv head)
-            for (int idx = threadIdx.x; idx < C::QROWS * CK; idx += 128) {
-                const int r = idx / CK, c = idx % CK;
-                float f[8];
-                if (r < M) {
-                    const int i = r / p.g, hq = hq0 + r % p.g;
-                    const T *src = static_cast<const T *>(p.q) + b * p.qs.b + i * p.qs.s + hq * p.qs.h;
-                    const int64_t pos = (int64_t)L + i;
-                    load_rotated_chunk<T>(src, c, p.r, inter, p.r ? cos_t + pos * p.cs_row : nullptr,
-                                          p.r ? sin_t + pos * p.cs_row : nullptr, f);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = 0.f;
-                }
-                *reinterpret_cast<uint4 *>(sQ + swz_offset<D_QK>(r, c * 8, C::QROWS)) = pack8<T>(f);
-            }
+    int qi = 0;            // pieces started
+    uint32_t sQa = 0;
+    for (int k = 0;; ++k) {
+        const int s = k % NST;
+        if (!mbar_wait(&full[s], (k / NST) & 1, p.status)) break;
+        const StageItem itm = items[s];
+        if (itm.flags & kEndOfStream) break;
+        const int b = itm.b;
+        const SegInfo seg = tab[b];
+        const int N = seg.N;
+        const int hq0 = itm.hk * p.g;
+        if (itm.flags & kPieceStart) {
+            s_first = itm.s;
+            const int qb = qi & 1;
+            sQa = smem_addr(sQ + qb * QBUF);
+            if (!mbar_wait(&q_full[qb], (qi >> 1) & 1, p.status)) break;
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
@@ -302,53 +449,22 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
                     last_vis[mt][hr] = r < M ? (p.causal ? min(N - 1, r / p.g + N - p.s_q) : N - 1) : -1;
                 }
             }
-            consumer_sync();
         }
 
         // ---- one 64-row tile = one item ----
-        const int t = k;
-        const int s = t % NST;
-        if (!timed_out && !mbar_wait(&full[s], (t / NST) & 1, p.status)) timed_out = true;
-        if (!timed_out) {
+        {
             uint8_t *sK = sStage + s * C::STAGE;
             uint8_t *sV = sK + C::KBYTES;
-            const int tile_row0 = it.s * C::TILE;
-            const int key0 = tile_row0 + warp * 16;
-            if (key0 + 16 > L) {
-                for (int item = lane; item < 16 * (CK + CV); item += 32) {
-                    const int rr = item / (CK + CV), c = item % (CK + CV);
-                    const int j = key0 + rr;
-                    if (j < L) continue;
-                    const int tr = warp * 16 + rr;
-                    if (j < N) {
-                        const int i = j - L;
-                        if (c < CK) {
-                            const T *src = static_cast<const T *>(p.k_new) + b * p.kn.b + i * p.kn.s + hk * p.kn.h;
-                            float f[8];
-                            load_rotated_chunk<T>(src, c, p.r, inter,
-                                                  p.r ? cos_t + (int64_t)j * p.cs_row : nullptr,
-                                                  p.r ? sin_t + (int64_t)j * p.cs_row : nullptr, f);
-                            const uint4 v = pack8<T>(f);
-                            *reinterpret_cast<uint4 *>(sK + swz_offset<D_QK>(tr, c * 8, C::TILE)) = v;
-                            T *dst = static_cast<T *>(p.k_cache) + b * p.kc.b + (int64_t)j * p.kc.s + hk * p.kc.h;
-                            reinterpret_cast<uint4 *>(dst)[c] = v;
-                        } else {
-                            const int cv = c - CK;
-                            const T *src = static_cast<const T *>(p.v_new) + b * p.vn.b + i * p.vn.s + hk * p.vn.h;
-                            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(src) + cv);
-                            *reinterpret_cast<uint4 *>(sV + swz_offset<D_V>(tr, cv * 8, C::TILE)) = v;
-                            T *dst = static_cast<T *>(p.v_cache) + b * p.vc.b + (int64_t)j * p.vc.s + hk * p.vc.h;
-                            reinterpret_cast<uint4 *>(dst)[cv] = v;
-                        }
-                    } else {
-                        const uint4 z = make_uint4(0, 0, 0, 0);
-                        if (c < CK)
-                            *reinterpret_cast<uint4 *>(sK + swz_offset<D_QK>(tr, c * 8, C::TILE)) = z;
-                        else
-                            *reinterpret_cast<uint4 *>(sV + swz_offset<D_V>(tr, (c - CK) * 8, C::TILE)) = z;
-                    }
+            const int key0 = itm.s * C::TILE + warp * 16;
+            const bool tail = key0 + 16 > N;
+            if (tail) {
+                // rows past the sequence: zero this warp's value rows
+                for (int item = lane; item < 16 * CV; item += 32) {
+                    const int rr = item / CV, c = item % CV;
+                    if (key0 + rr >= N)
+                        *reinterpret_cast<uint4 *>(sV + swz_offset<D_V>(warp * 16 + rr, c * 8, C::TILE)) =
+                            make_uint4(0, 0, 0, 0);
                 }
-                fence_proxy_async();
                 __syncwarp();
             }
 
@@ -370,8 +486,7 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
                     uint32_t a[4];
-                    ldmatrix_x4(sQa + swz_offset<D_QK>(mt * 16 + (lane & 15), kk * 16 + ((lane >> 4) << 3),
-                                                       C::QROWS),
+                    ldmatrix_x4(sQa + swz_offset<D_QK>(mt * 16 + (lane & 15), kk * 16 + ((lane >> 4) << 3), QT),
                                 a[0], a[1], a[2], a[3]);
                     Mma<T>::run(sacc[mt][0], a, kb[0], kb[1]);
                     Mma<T>::run(sacc[mt][1], a, kb[2], kb[3]);
@@ -439,13 +554,18 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
                     Mma<T>::run(o[mt][2 * nn + 1], pa[mt], vb[2], vb[3]);
                 }
             }
+            // the zeroed rows were written through the generic proxy; the next
+            // TMA into this stage writes through the async proxy
+            if (tail) fence_proxy_async();
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
 
-        // ---- end of piece: merge the four warps and write ----
-        const bool piece_end = (k == n_items - 1) || (it.s + 1 >= it.seg.n_items);
-        if (piece_end) {
+        // ---- end of piece: release q, merge the four warps and write ----
+        if (itm.flags & kPieceEnd) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_empty[qi & 1]);
+            ++qi;
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -472,7 +592,7 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
                     }
                 }
             consumer_sync();
-            const bool single = it.seg.n_items == 1;
+            const bool single = seg.n_items == 1;
             for (int idx = threadIdx.x; idx < M * CV; idx += 128) {
                 const int row = idx / CV, c = idx % CV;
                 float mw[4], mx = -INFINITY;
@@ -510,105 +630,146 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS) decode_kernel(c
                     dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
                     if (c == 0) {
                         p.lse_part[row_slot0 + s_first] = lse_v;
-                        for (int s2 = s_first + 1; s2 <= it.s; ++s2) p.lse_part[row_slot0 + s2] = -INFINITY;
+                        for (int s2 = s_first + 1; s2 <= itm.s; ++s2) p.lse_part[row_slot0 + s2] = -INFINITY;
                     }
                 }
             }
         }
-        iter_advance(p, tab, it);
     }
 }
 
-// One warp per (batch, query head, query row): merge the split slots.
+// One 128-thread block per (batch, query head, query row): merge the split
+// slots.  The row's slots are contiguous; every thread loads up to four lse
+// values (slots t, t + 128, ...) at once with the batch entry's item count,
+// the block reduces max and sum, compacts the live slots (the first slot of
+// each piece) in slot order, and the four warps read the live partial outputs
+// with independent 16-byte loads (lane l owns columns 4 l .. 4 l + 3 and
+// 4 l + 128 .. 4 l + 131), summed across warps in shared memory.
+constexpr int kCombineThreads = 128;
+constexpr int kCombineSlots = 4 * kCombineThreads;   // slots per row the combine handles
+
 template <typename T>
-__global__ void __launch_bounds__(256) combine_kernel(const DecodeParams p, int d_v) {
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const DecodeParams p, int d_v) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    const int64_t total = (int64_t)p.b * p.h_q * p.s_q;
-    if (w >= total) return;
-    const int i = (int)(w % p.s_q);
-    const int hq = (int)((w / p.s_q) % p.h_q);
-    const int b = (int)(w / ((int64_t)p.s_q * p.h_q));
+    const int64_t row = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int i = (int)(row % p.s_q);
+    const int hq = (int)((row / p.s_q) % p.h_q);
+    const int b = (int)(row / ((int64_t)p.s_q * p.h_q));
+    const int64_t row_slot0 = (((int64_t)b * p.h_q + hq) * p.s_q + i) * p.n_splits;
+    float ls[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int s = tid + kCombineThreads * k;
+        ls[k] = s < p.n_splits ? p.lse_part[row_slot0 + s] : -INFINITY;
+    }
     const SegInfo sg = seg_info(p, b);
     const int n = sg.n_items;
-    if (n <= 1) return;
-    // the row's slots are contiguous: read their lse values coalesced, keep
-    // them in registers (lane l holds slots l, l + 32, ...)
-    const int64_t row_slot0 = (((int64_t)b * p.h_q + hq) * p.s_q + i) * p.n_splits;
-    constexpr int MAXS = 16;  // up to 512 slots per row
-    float ls[MAXS];
+    if (n <= 1) return;   // written by the decode kernel (or the empty-entry path)
+
+    __shared__ float red[4];
+    __shared__ int counts[4][4];           // live slots per (k, warp)
+    __shared__ int live_slot[kCombineSlots];
+    __shared__ float live_w[kCombineSlots];
+    __shared__ __align__(16) float acc_s[4][256];
+
     float mx = -INFINITY;
 #pragma unroll
-    for (int k = 0; k < MAXS; ++k) {
-        const int s = lane + 32 * k;
-        ls[k] = s < n ? p.lse_part[row_slot0 + s] : -INFINITY;
+    for (int k = 0; k < 4; ++k) {
+        if (tid + kCombineThreads * k >= n) ls[k] = -INFINITY;
         mx = fmaxf(mx, ls[k]);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
     T *dst = static_cast<T *>(p.out) + b * p.os.b + i * p.os.s + hq * p.os.h;
     if (mx == -INFINITY) {
-        for (int c = lane * 2; c < d_v; c += 64) *reinterpret_cast<uint32_t *>(dst + c) = 0u;
-        if (lane == 0 && p.lse) p.lse[((int64_t)b * p.h_q + hq) * p.s_q + i] = -INFINITY;
+        for (int c = tid * 2; c < d_v; c += 2 * kCombineThreads) *reinterpret_cast<uint32_t *>(dst + c) = 0u;
+        if (tid == 0 && p.lse) p.lse[((int64_t)b * p.h_q + hq) * p.s_q + i] = -INFINITY;
         return;
     }
     float sum = 0.f;
 #pragma unroll
-    for (int k = 0; k < MAXS; ++k) sum += ex2((ls[k] - mx) * kLog2e);
+    for (int k = 0; k < 4; ++k) sum += ex2((ls[k] - mx) * kLog2e);
 #pragma unroll
     for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    const float lse = mx + logf(sum);
+    __syncthreads();   // everyone has read red[] (max)
+    if (lane == 0) red[warp] = sum;
+    unsigned live[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        live[k] = __ballot_sync(0xffffffffu, ls[k] != -INFINITY);
+        if (lane == 0) counts[k][warp] = __popc(live[k]);
+    }
+    __syncthreads();
+    const float lse = mx + logf(red[0] + red[1] + red[2] + red[3]);
+    // ordered compaction: slot order is (k, warp, lane)
+    int n_live = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) n_live += counts[k][w];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        int before = 0;
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2)
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                if (k2 < k || (k2 == k && w < warp)) before += counts[k2][w];
+        if (ls[k] != -INFINITY) {
+            const int pos = before + __popc(live[k] & ((1u << lane) - 1u));
+            live_slot[pos] = tid + kCombineThreads * k;
+            live_w[pos] = ex2((ls[k] - lse) * kLog2e);
+        }
+    }
+    __syncthreads();
     float a[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) a[e] = 0.f;
-    // Only the first slot of every piece holds an output.  Compact the live
-    // slots and their weights into this warp's shared-memory list, then read
-    // their outputs with independent (overlapping) loads.
-    constexpr int LIST = 64;
-    __shared__ int live_slot[8][LIST];
-    __shared__ float live_w[8][LIST];
-    const int wib = threadIdx.x >> 5;
-    int n_total = 0;
+    // warp w reads live slots w, w + 4, ...: a batch of up to 16 loads per
+    // column group is in flight before any is used
+    constexpr int BATCH = 16;
+    for (int t0 = warp; t0 < n_live; t0 += 4 * BATCH) {
 #pragma unroll
-    for (int k = 0; k < MAXS; ++k) n_total += __popc(__ballot_sync(0xffffffffu, ls[k] != -INFINITY));
-    for (int base = 0; base < n_total; base += LIST) {
-        int n_live = 0;
+        for (int h = 0; h < 2; ++h) {
+            const int c = lane * 4 + h * 128;
+            if (c >= d_v) continue;
+            float4 v[BATCH];
+            float wgt[BATCH];
 #pragma unroll
-        for (int k = 0; k < MAXS; ++k) {
-            const bool is_live = ls[k] != -INFINITY;
-            const unsigned live = __ballot_sync(0xffffffffu, is_live);
-            const int pos = n_live + __popc(live & ((1u << lane) - 1u)) - base;
-            if (is_live && pos >= 0 && pos < LIST) {
-                live_slot[wib][pos] = lane + 32 * k;
-                live_w[wib][pos] = ex2((ls[k] - lse) * kLog2e);
-            }
-            n_live += __popc(live);
-        }
-        __syncwarp();
-        const int cnt = min(LIST, n_total - base);
-#pragma unroll 4
-        for (int t = 0; t < cnt; ++t) {
-            const float wgt = live_w[wib][t];
-            const float *src = p.o_part + (row_slot0 + live_slot[wib][t]) * d_v;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int c = lane * 2 + e * 64;
-                if (c < d_v) {
-                    const float2 v = *reinterpret_cast<const float2 *>(src + c);
-                    a[2 * e] = fmaf(wgt, v.x, a[2 * e]);
-                    a[2 * e + 1] = fmaf(wgt, v.y, a[2 * e + 1]);
+            for (int u = 0; u < BATCH; ++u) {
+                const int t = t0 + 4 * u;
+                wgt[u] = 0.f;
+                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (t < n_live) {
+                    wgt[u] = live_w[t];
+                    v[u] = *reinterpret_cast<const float4 *>(p.o_part + (row_slot0 + live_slot[t]) * d_v + c);
                 }
             }
+#pragma unroll
+            for (int u = 0; u < BATCH; ++u) {
+                a[4 * h + 0] = fmaf(wgt[u], v[u].x, a[4 * h + 0]);
+                a[4 * h + 1] = fmaf(wgt[u], v[u].y, a[4 * h + 1]);
+                a[4 * h + 2] = fmaf(wgt[u], v[u].z, a[4 * h + 2]);
+                a[4 * h + 3] = fmaf(wgt[u], v[u].w, a[4 * h + 3]);
+            }
         }
-        __syncwarp();
     }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const int c = lane * 2 + e * 64;
-        if (c < d_v) *reinterpret_cast<uint32_t *>(dst + c) = Elem<T>::pack2(a[2 * e], a[2 * e + 1]);
+    for (int h = 0; h < 2; ++h) {
+        const int c = lane * 4 + h * 128;
+        if (c < d_v) *reinterpret_cast<float4 *>(&acc_s[warp][c]) = make_float4(a[4 * h], a[4 * h + 1], a[4 * h + 2], a[4 * h + 3]);
     }
-    if (lane == 0 && p.lse) p.lse[((int64_t)b * p.h_q + hq) * p.s_q + i] = lse;
+    __syncthreads();
+    for (int c = tid * 2; c < d_v; c += 2 * kCombineThreads) {
+        const float v0 = acc_s[0][c] + acc_s[1][c] + acc_s[2][c] + acc_s[3][c];
+        const float v1 = acc_s[0][c + 1] + acc_s[1][c + 1] + acc_s[2][c + 1] + acc_s[3][c + 1];
+        *reinterpret_cast<uint32_t *>(dst + c) = Elem<T>::pack2(v0, v1);
+    }
+    if (tid == 0 && p.lse) p.lse[((int64_t)b * p.h_q + hq) * p.s_q + i] = lse;
 }
 
 int sm_count() {
@@ -622,9 +783,13 @@ int sm_count() {
     return n;
 }
 
+// The decode kernel is a programmatic dependent of the RoPE/append kernel
+// launched just before it (its CTAs start early and wait for that grid before
+// reading what it wrote); the combine kernel is a programmatic dependent of
+// the decode kernel.
 template <typename T, int D_QK, int D_V, int MT>
-static cudaError_t run_decode(const DecodeParams &p_in, const CUtensorMap &tmK, const CUtensorMap &tmV,
-                              cudaStream_t st) {
+static cudaError_t run_decode(const DecodeParams &p_in, const CUtensorMap &tmQ, const CUtensorMap &tmK,
+                              const CUtensorMap &tmV, cudaStream_t st) {
     using C = DecodeCfg<D_QK, D_V, MT>;
     DecodeParams p = p_in;
     const int M = p.g * p.s_q;
@@ -634,24 +799,30 @@ static cudaError_t run_decode(const DecodeParams &p_in, const CUtensorMap &tmK, 
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D_QK, D_V, MT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(sm_count() * DecodeOcc<D_V, MT>::CTAS));
+    cfg.blockDim = dim3(160);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     kernel_event(0, st);
-    decode_kernel<T, D_QK, D_V, MT><<<sm_count() * DecodeOcc<D_V, MT>::CTAS, 160, smem, st>>>(tmK, tmV, p);
-    e = cudaGetLastError();
+    e = cudaLaunchKernelEx(&cfg, decode_kernel<T, D_QK, D_V, MT>, tmQ, tmK, tmV, p);
     kernel_event(1, st);
     if (e != cudaSuccess) return e;
     if (p.n_splits > 1) {
-        const int64_t warps = (int64_t)p.b * p.h_q * p.s_q;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)((warps * 32 + 255) / 256));
-        cfg.blockDim = dim3(256);
-        cfg.dynamicSmemBytes = 0;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, combine_kernel<T>, p, D_V);
+        const int64_t rows = (int64_t)p.b * p.h_q * p.s_q;
+        cudaLaunchConfig_t ccfg = {};
+        ccfg.gridDim = dim3((unsigned)rows);
+        ccfg.blockDim = dim3(kCombineThreads);
+        ccfg.dynamicSmemBytes = 0;
+        ccfg.stream = st;
+        ccfg.attrs = attr;
+        ccfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&ccfg, combine_kernel<T>, p, D_V);
     }
     return e;
 }
@@ -667,12 +838,12 @@ bool decode_supported(int d_qk, int d_v, int mt) {
     return false;
 }
 
-cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
-                          int dtype, int d_qk, int d_v, int mt, cudaStream_t st) {
-#define FA_CASE(DQ, DV, MT)                                                                \
-    if (d_qk == DQ && d_v == DV && mt == MT) {                                             \
-        if (dtype == FA_DTYPE_F16) return run_decode<__half, DQ, DV, MT>(p, tmK, tmV, st); \
-        return run_decode<__nv_bfloat16, DQ, DV, MT>(p, tmK, tmV, st);                     \
+cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmQ, const CUtensorMap &tmK,
+                          const CUtensorMap &tmV, int dtype, int d_qk, int d_v, int mt, cudaStream_t st) {
+#define FA_CASE(DQ, DV, MT)                                                                     \
+    if (d_qk == DQ && d_v == DV && mt == MT) {                                                  \
+        if (dtype == FA_DTYPE_F16) return run_decode<__half, DQ, DV, MT>(p, tmQ, tmK, tmV, st); \
+        return run_decode<__nv_bfloat16, DQ, DV, MT>(p, tmQ, tmK, tmV, st);                     \
     }
     FA_DECODE_DIMS(FA_CASE)
 #undef FA_CASE

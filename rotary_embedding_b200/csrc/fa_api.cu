@@ -4,8 +4,9 @@
 // Planner (one GPU, one stream, no allocation):
 //  * fa_kvcache_fwd with a short new chunk (s_q <= 8 and at most 32 query
 //    rows per kv head, the decode branch of s2.cpp PR #40's eval_cached):
-//    one split-KV decode launch that also rotates q / k_new and appends the
-//    new rows, then the LSE combine when a batch entry spans several splits.
+//    the rope+append kernel (new rows into the cache, rotated q into the
+//    workspace), the persistent split-KV decode kernel as its programmatic
+//    dependent, then the LSE combine when a batch entry spans several items.
 //  * otherwise (the prefill / concat branch): the rope+append kernel, then
 //    the attention kernel over the cache, on the same stream (write before
 //    read, s2.cpp PR #40 review).
@@ -160,6 +161,8 @@ struct KvPlan {
     int chunk = 0;
     int n_splits = 1;
     size_t ws_bytes = 0;
+    size_t off_pool = 0;      // decode: workspace = q_rot | pool counter | o_part | lse_part
+    size_t off_o_part = 0;
     size_t off_lse_part = 0;
     bool rotate_q_to_ws = false;
 };
@@ -234,9 +237,14 @@ KvPlan plan_kvcache(int64_t b, int64_t s_q, int64_t h_q, int64_t h_kv, int64_t d
         // each item owns one partial-result slot.
         pl.chunk = 64;
         pl.n_splits = (int)((cap + 63) / 64);
+        // the decode kernel reads q through a TMA map over a contiguous rotated copy
+        pl.rotate_q_to_ws = true;
+        pl.off_pool = align_up((size_t)b * s_q * h_q * d_qk * 2, 256);
+        pl.off_o_part = pl.off_pool + 256;
+        pl.ws_bytes = pl.off_o_part;
         if (pl.n_splits > 1) {
             const size_t rows = (size_t)pl.n_splits * b * h_q * s_q;
-            pl.off_lse_part = align_up(rows * d_v * sizeof(float), 256);
+            pl.off_lse_part = pl.off_o_part + align_up(rows * d_v * sizeof(float), 256);
             pl.ws_bytes = pl.off_lse_part + align_up(rows * sizeof(float), 256);
         }
         return pl;
@@ -403,7 +411,7 @@ int fa_kvcache_plan(const fa_tensor *q, const fa_tensor *k_cache, const fa_tenso
     plan->path = pl.decode ? FA_PATH_DECODE : FA_PATH_PREFILL;
     plan->n_splits = pl.decode ? pl.n_splits : 1;
     plan->chunk = pl.decode ? pl.chunk : 0;
-    plan->launches = pl.decode ? (pl.n_splits > 1 ? 2 : 1) : ((s_new > 0 || rotary_dim > 0) ? 2 : 1);
+    plan->launches = pl.decode ? (pl.n_splits > 1 ? 3 : 2) : ((s_new > 0 || rotary_dim > 0) ? 2 : 1);
     plan->workspace_bytes = pl.ws_bytes;
     return FA_OK;
 }
@@ -459,55 +467,9 @@ int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor
     if (!status) return fail(FA_ERR_CUDA, "no CUDA device");
     const int cs_row = cos ? (int)cos->stride[0] : 0;
 
-    if (pl.decode) {
-        CUtensorMap tmK, tmV;
-        if ((rc = make_rows_map(&tmK, k_cache, 64, "k_cache"))) return rc;
-        if ((rc = make_rows_map(&tmV, v_cache, 64, "v_cache"))) return rc;
-        DecodeParams p{};
-        p.status = status;
-        p.q = q->data;
-        p.qs = s3(a.q);
-        p.k_new = a.has_new ? k_new->data : nullptr;
-        p.kn = a.has_new ? s3(a.kn) : Strides3{0, 0, 0};
-        p.v_new = a.has_new ? v_new->data : nullptr;
-        p.vn = a.has_new ? s3(a.vn) : Strides3{0, 0, 0};
-        p.k_cache = k_cache->data;
-        p.kc = s3(a.kc);
-        p.v_cache = v_cache->data;
-        p.vc = s3(a.vc);
-        p.cos = a.r ? cos->data : nullptr;
-        p.sin = a.r ? sin->data : nullptr;
-        p.cs_row = cs_row;
-        p.cs_rows = a.s_ro;
-        p.seqlens = cache_seqlens;
-        p.seqlen_scalar = cache_seqlens_scalar;
-        p.out = out->data;
-        p.os = s3(od);
-        p.lse = lse;
-        p.o_part = static_cast<float *>(workspace);
-        p.lse_part = workspace ? reinterpret_cast<float *>(static_cast<char *>(workspace) + pl.off_lse_part) : nullptr;
-        p.b = (int)a.b;
-        p.s_q = (int)a.s_q;
-        p.s_new = (int)a.s_new;
-        p.h_q = (int)a.h_q;
-        p.h_kv = (int)a.h_kv;
-        p.g = (int)(a.h_q / a.h_kv);
-        p.r = a.r;
-        p.interleaved = interleaved ? 1 : 0;
-        p.causal = causal ? 1 : 0;
-        p.cap = a.cap;
-        p.scale_log2 = sc * 1.4426950408889634f;
-        p.chunk = pl.chunk;
-        p.n_splits = pl.n_splits;
-        cudaError_t e = launch_decode(p, tmK, tmV, a.dtype, (int)a.d_qk, (int)a.d_v, pl.mt, st);
-        if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-        return FA_OK;
-    }
-
-    // prefill / chunked path: rotate + append, then attention over the cache
-    void *q_att = q->data;
-    Strides3 q_att_s = s3(a.q);
-    if (a.has_new || pl.rotate_q_to_ws) {
+    // The rope+append kernel: rotated k_new and raw v_new into the cache at
+    // L_b, and (when asked) q rotated at L_b + i into `q_rot`.
+    auto rope_append = [&](void *q_rot, int32_t *zero_word) -> int {
         RopeAppendParams p{};
         p.status = status;
         p.k_new = a.has_new ? k_new->data : nullptr;
@@ -520,7 +482,7 @@ int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor
         p.vc = s3(a.vc);
         p.q = q->data;
         p.qs = s3(a.q);
-        p.q_rot = pl.rotate_q_to_ws ? workspace : nullptr;
+        p.q_rot = q_rot;
         p.cos = a.r ? cos->data : nullptr;
         p.sin = a.r ? sin->data : nullptr;
         p.cs_row = cs_row;
@@ -537,8 +499,60 @@ int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor
         p.r = a.r;
         p.interleaved = interleaved ? 1 : 0;
         p.cap = a.cap;
+        p.zero_word = zero_word;
         cudaError_t e = launch_rope_append(p, a.dtype, st);
         if (e != cudaSuccess) return cuda_fail(e, "rope/append launch");
+        return FA_OK;
+    };
+
+    if (pl.decode) {
+        char *ws = static_cast<char *>(workspace);
+        int32_t *pool = reinterpret_cast<int32_t *>(ws + pl.off_pool);
+        if ((rc = rope_append(workspace, pool))) return rc;
+        // q rows in the workspace: contiguous [b, s_q, h_q, d_qk]
+        fa_tensor qr = *q;
+        qr.data = workspace;
+        qr.stride[3] = 1;
+        qr.stride[2] = a.d_qk;
+        qr.stride[1] = a.h_q * a.d_qk;
+        qr.stride[0] = a.s_q * a.h_q * a.d_qk;
+        CUtensorMap tmQ, tmK, tmV;
+        if ((rc = make_rows_map(&tmQ, &qr, (int)a.s_q, "q_rot", (int)(a.h_q / a.h_kv)))) return rc;
+        if ((rc = make_rows_map(&tmK, k_cache, 64, "k_cache"))) return rc;
+        if ((rc = make_rows_map(&tmV, v_cache, 64, "v_cache"))) return rc;
+        DecodeParams p{};
+        p.status = status;
+        p.cs_rows = a.s_ro;
+        p.seqlens = cache_seqlens;
+        p.seqlen_scalar = cache_seqlens_scalar;
+        p.out = out->data;
+        p.os = s3(od);
+        p.lse = lse;
+        p.pool = pool;
+        p.o_part = pl.n_splits > 1 ? reinterpret_cast<float *>(ws + pl.off_o_part) : nullptr;
+        p.lse_part = pl.n_splits > 1 ? reinterpret_cast<float *>(ws + pl.off_lse_part) : nullptr;
+        p.b = (int)a.b;
+        p.s_q = (int)a.s_q;
+        p.s_new = (int)a.s_new;
+        p.h_q = (int)a.h_q;
+        p.h_kv = (int)a.h_kv;
+        p.g = (int)(a.h_q / a.h_kv);
+        p.r = a.r;
+        p.causal = causal ? 1 : 0;
+        p.cap = a.cap;
+        p.scale_log2 = sc * 1.4426950408889634f;
+        p.chunk = pl.chunk;
+        p.n_splits = pl.n_splits;
+        cudaError_t e = launch_decode(p, tmQ, tmK, tmV, a.dtype, (int)a.d_qk, (int)a.d_v, pl.mt, st);
+        if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+        return FA_OK;
+    }
+
+    // prefill / chunked path: rotate + append, then attention over the cache
+    void *q_att = q->data;
+    Strides3 q_att_s = s3(a.q);
+    if (a.has_new || pl.rotate_q_to_ws) {
+        if ((rc = rope_append(pl.rotate_q_to_ws ? workspace : nullptr, nullptr))) return rc;
         if (pl.rotate_q_to_ws) {
             q_att = workspace;
             q_att_s = Strides3{a.s_q * a.h_q * a.d_qk, a.h_q * a.d_qk, a.d_qk};

@@ -15,7 +15,8 @@ struct Strides3 {
     int64_t b, s, h;
 };
 
-// Rotary + append (+ optional rotated copy of q) for the prefill path.
+// Rotary + append (+ optional rotated copy of q), before the decode or the
+// prefill attention kernel.
 struct RopeAppendParams {
     int32_t *status;  // device status word (see fa_device_status)
     const void *k_new;
@@ -36,37 +37,28 @@ struct RopeAppendParams {
     int32_t seqlen_scalar;
     int b, s_q, s_new, h_q, h_kv, d_qk, d_v, r, interleaved;
     int64_t cap;
+    int32_t *zero_word;  // set to 0 by the kernel when not null (the decode work-pool counter)
 };
 
-// Split-KV decode with fused RoPE/append (s_q * h_q / h_kv <= 32 query rows
-// per kv head).
+// Split-KV decode over the cache after the RoPE/append kernel (s_q * h_q / h_kv
+// <= 32 query rows per kv head).
 struct DecodeParams {
     int32_t *status;  // device status word (see fa_device_status)
-    const void *q;
-    Strides3 qs;
-    const void *k_new;
-    Strides3 kn;
-    const void *v_new;
-    Strides3 vn;
-    void *k_cache;
-    Strides3 kc;
-    void *v_cache;
-    Strides3 vc;
-    const void *cos, *sin;
-    int64_t cs_row, cs_rows;
+    int64_t cs_rows;  // rows of the cos/sin table (precondition check only)
     const int32_t *seqlens;
     int32_t seqlen_scalar;
     void *out;
     Strides3 os;
     float *lse;      // [b, h_q, s_q] or nullptr
-    float *o_part;   // [n_splits, b, h_q, s_q, d_v]
-    float *lse_part; // [n_splits, b, h_q, s_q]
-    int b, s_q, s_new, h_q, h_kv, g, r, interleaved, causal;
+    float *o_part;   // [b, h_q, s_q, n_splits, d_v]
+    float *lse_part; // [b, h_q, s_q, n_splits]
+    int b, s_q, s_new, h_q, h_kv, g, r, causal;
     int64_t cap;
     float scale_log2;
     int chunk;     // key rows per split, multiple of 64
     int n_stages;  // K/V ring depth (set by the launcher from the shared-memory budget)
-    int n_splits;  // splits per (batch, kv head) = grid.x
+    int n_splits;  // slots per output row (one per 64-row item of the longest segment)
+    int *pool;     // work-pool counter (zeroed by the RoPE/append kernel)
 };
 
 // Generic attention (any supported head dim): keys from k/v (dense) or
@@ -121,8 +113,10 @@ bool prefill_supported(int d_qk, int d_v);
 int prefill_block_n(int d_qk, int d_v, int tiles_per_cta);  // key rows per K/V tile (TMA box rows)
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &tmQ, const CUtensorMap &tmK,
                            const CUtensorMap &tmV, int dtype, int d_qk, int d_v, cudaStream_t st);
-cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmK, const CUtensorMap &tmV,
-                          int dtype, int d_qk, int d_v, int mt, cudaStream_t st);
+// tmQ: the rotated q rows in the workspace, box (64 cols, g heads, s_q rows);
+// tmK / tmV: the caches, box (64 cols, 1 head, 64 rows).
+cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmQ, const CUtensorMap &tmK,
+                          const CUtensorMap &tmV, int dtype, int d_qk, int d_v, int mt, cudaStream_t st);
 bool decode_supported(int d_qk, int d_v, int mt);
 cudaError_t launch_simt_attn(const SimtAttnParams &p, int dtype, cudaStream_t st);
 

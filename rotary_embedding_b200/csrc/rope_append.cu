@@ -1,4 +1,5 @@
-// rope_append.cu -- fused RoPE + KV-cache append for the prefill path.
+// rope_append.cu -- fused RoPE + KV-cache append, ahead of the decode or the
+// prefill attention kernel.
 //
 // One thread per 16-byte chunk (8 elements) of a row.  Rows are, in order:
 // the new key rows (rotated at position L_b + i, rounded, written to
@@ -12,13 +13,20 @@
 // rotary_dim/2), int or per-batch SEQLEN_OFFSET, INTERLEAVED) and s2.cpp
 // PR #40 (write the new k/v rows at their offsets before attention reads
 // them; the attention kernel is enqueued after this one on the same stream).
+// The decode kernel is launched as this kernel's programmatic dependent: every
+// CTA releases it at once, and it waits for this grid's completion (and the
+// visibility of its writes) before it reads q or new cache rows.
 #include "fa_common.cuh"
 #include "fa_internal.h"
 
 namespace fa {
 
+// At most 40 registers per thread, so that one of these blocks and two CTAs
+// of the decode kernel (its programmatic dependent) fit on an SM together.
 template <typename T>
-__global__ void __launch_bounds__(256) rope_append_kernel(RopeAppendParams p) {
+__global__ void __launch_bounds__(256, 6) rope_append_kernel(RopeAppendParams p) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (p.zero_word && blockIdx.x == 0 && threadIdx.x == 0) *p.zero_word = 0;
     const int ck = p.d_qk / 8, cv = p.d_v / 8;
     const int64_t n_k = (int64_t)p.b * p.s_new * p.h_kv * ck;
     const int64_t n_v = (int64_t)p.b * p.s_new * p.h_kv * cv;
@@ -81,8 +89,8 @@ __global__ void __launch_bounds__(256) rope_append_kernel(RopeAppendParams p) {
 cudaError_t launch_rope_append(const RopeAppendParams &p, int dtype, cudaStream_t st) {
     const int64_t total = (int64_t)p.b * p.s_new * p.h_kv * (p.d_qk / 8 + p.d_v / 8) +
                           (p.q_rot ? (int64_t)p.b * p.s_q * p.h_q * (p.d_qk / 8) : 0);
-    if (total == 0) return cudaSuccess;
-    int64_t blocks = (total + 255) / 256;
+    if (total == 0 && !p.zero_word) return cudaSuccess;
+    int64_t blocks = total > 0 ? (total + 255) / 256 : 1;
     if (blocks > 148 * 16) blocks = 148 * 16;
     if (dtype == FA_DTYPE_F16)
         rope_append_kernel<__half><<<(unsigned)blocks, 256, 0, st>>>(p);

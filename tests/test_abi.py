@@ -93,7 +93,11 @@ def test_accepts_transposed_views_in_validation():
     # head-dim stride must be 1; the call then fails later only for lack of a GPU
     q = torch.zeros(2, 4, 3, 64, dtype=torch.float16).transpose(1, 2)
     _, kc, vc, kn, vn, out = _kv_tensors()
-    rc = _call(q, kc, vc, kn, vn, out)
+    # a workspace of the planned size at a 256-byte boundary (never touched here)
+    need = fa.fa_kvcache_workspace_size(q, kc, vc, kn)
+    buf = torch.zeros(need + 256, dtype=torch.uint8)
+    ws = (buf.data_ptr() + 255) // 256 * 256
+    rc = _call(q, kc, vc, kn, vn, out, ws=ws, ws_bytes=need)
     assert rc in (fa.FA_OK, fa.FA_ERR_CUDA)
 
 
