@@ -1,12 +1,15 @@
 // rope_append.cu -- fused RoPE + KV-cache append, ahead of the decode or the
 // prefill attention kernel.
 //
-// One thread per 16-byte chunk (8 elements) of a row.  Rows are, in order:
-// the new key rows (rotated at position L_b + i, rounded, written to
-// k_cache row L_b + i), the new value rows (bit copy to v_cache row
-// L_b + i) and, when a rotated copy of q is requested, the query rows
-// (rotated at position L_b + i into a contiguous buffer).  Loads and stores
-// are 128-bit and consecutive threads touch consecutive chunks of a row.
+// One 128-thread block per (batch entry b, row i) and group of 256 16-byte
+// chunks of that row's work: the new key row of every kv head (rotated at
+// position L_b + i, rounded, written to k_cache row L_b + i), the new value
+// row of every kv head (bit copy to v_cache row L_b + i) and, when a rotated
+// copy of q is requested, the query row of every head (rotated at position
+// L_b + i into a contiguous buffer).  Each thread first issues the 128-bit
+// loads of its two chunks (they do not depend on cache_seqlens), then the
+// block reads L_b and stages the cos/sin row of position L_b + i in shared
+// memory once for all heads, and the thread rotates and stores.
 //
 // Follows flash-attention issue #1402 (apply_rotary_emb / rotate_half,
 // cache_seqlens offsets), ROCm/flash-attention PR #99 (COS/SIN (seqlen,
@@ -21,81 +24,140 @@
 
 namespace fa {
 
-// At most 40 registers per thread, so that one of these blocks and two CTAs
+constexpr int kRopeThreads = 128;
+constexpr int kRopeOps = 2;   // 16-byte chunks per thread
+
+// At most 64 registers per thread, so that one of these blocks and two CTAs
 // of the decode kernel (its programmatic dependent) fit on an SM together.
 template <typename T>
-__global__ void __launch_bounds__(256, 6) rope_append_kernel(RopeAppendParams p) {
+__global__ void __launch_bounds__(kRopeThreads, 8) rope_append_kernel(RopeAppendParams p) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (p.zero_word && blockIdx.x == 0 && threadIdx.x == 0) *p.zero_word = 0;
-    const int ck = p.d_qk / 8, cv = p.d_v / 8;
-    const int64_t n_k = (int64_t)p.b * p.s_new * p.h_kv * ck;
-    const int64_t n_v = (int64_t)p.b * p.s_new * p.h_kv * cv;
-    const int64_t n_q = p.q_rot ? (int64_t)p.b * p.s_q * p.h_q * ck : 0;
-    const int64_t total = n_k + n_v + n_q;
+    if (p.zero_word && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.zero_word = 0;
+    __shared__ float cs_s[128], sn_s[128];
+    const int rows = max(1, max(p.q_rot ? p.s_q : 0, p.s_new));
+    const int b = blockIdx.x / rows, i = blockIdx.x % rows;
+    const int ck = p.d_qk >> 3, cv = p.d_v >> 3;
+    const bool has_new = i < p.s_new;
+    const bool has_q = p.q_rot != nullptr && i < p.s_q;
+    const int n_k = has_new ? p.h_kv * ck : 0;
+    const int n_v = has_new ? p.h_kv * cv : 0;
+    const int n_q = has_q ? p.h_q * ck : 0;
+    const int total = n_k + n_v + n_q;
+    if ((int)blockIdx.y * kRopeOps * kRopeThreads >= total) return;
     const bool inter = p.interleaved != 0;
-    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
-         idx += (int64_t)gridDim.x * blockDim.x) {
-        int64_t t = idx;
-        int kind;  // 0 = k_new, 1 = v_new, 2 = q
-        int c, h, i, b;
+    const int half = p.r >> 1;
+    const bool chunk_partner = !inter && (half & 7) == 0;
+
+    // this thread's chunks: kind 0 = k_new, 1 = v_new, 2 = q; source loads first
+    int kind[kRopeOps], head[kRopeOps], chunk[kRopeOps];
+    const T *srow[kRopeOps];
+    uint4 raw[kRopeOps], praw[kRopeOps];
+#pragma unroll
+    for (int u = 0; u < kRopeOps; ++u) {
+        const int t = ((int)blockIdx.y * kRopeOps + u) * kRopeThreads + (int)threadIdx.x;
+        kind[u] = -1;
+        head[u] = chunk[u] = 0;
+        srow[u] = nullptr;
+        raw[u] = praw[u] = make_uint4(0, 0, 0, 0);
+        if (t >= total) continue;
+        int c, h, kd;
         if (t < n_k) {
-            kind = 0;
-            c = (int)(t % ck); t /= ck;
-            h = (int)(t % p.h_kv); t /= p.h_kv;
-            i = (int)(t % p.s_new); b = (int)(t / p.s_new);
-        } else if ((t -= n_k) < n_v) {
-            kind = 1;
-            c = (int)(t % cv); t /= cv;
-            h = (int)(t % p.h_kv); t /= p.h_kv;
-            i = (int)(t % p.s_new); b = (int)(t / p.s_new);
+            kd = 0; h = t / ck; c = t - h * ck;
+            srow[u] = static_cast<const T *>(p.k_new) + b * p.kn.b + i * p.kn.s + h * p.kn.h;
+        } else if (t < n_k + n_v) {
+            const int t2 = t - n_k;
+            kd = 1; h = t2 / cv; c = t2 - h * cv;
+            srow[u] = static_cast<const T *>(p.v_new) + b * p.vn.b + i * p.vn.s + h * p.vn.h;
         } else {
-            t -= n_v;
-            kind = 2;
-            c = (int)(t % ck); t /= ck;
-            h = (int)(t % p.h_q); t /= p.h_q;
-            i = (int)(t % p.s_q); b = (int)(t / p.s_q);
+            const int t2 = t - n_k - n_v;
+            kd = 2; h = t2 / ck; c = t2 - h * ck;
+            srow[u] = static_cast<const T *>(p.q) + b * p.qs.b + i * p.qs.s + h * p.qs.h;
         }
-        const int L = seqlen_of(p.seqlens, p.seqlen_scalar, b);
-        // device-side preconditions: the new rows fit the cache and the table
-        if (L < 0 || (int64_t)L + p.s_new > p.cap ||
-            (p.r > 0 && (int64_t)L + (kind == 2 ? p.s_q : p.s_new) > p.cs_rows)) {
-            if (c == 0 && h == 0 && i == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
-            continue;
+        kind[u] = kd;
+        head[u] = h;
+        chunk[u] = c;
+        raw[u] = __ldg(reinterpret_cast<const uint4 *>(srow[u]) + c);
+        if (kd != 1 && chunk_partner && 8 * c < p.r) {
+            const int pc = (8 * c < half) ? c + (half >> 3) : c - (half >> 3);
+            praw[u] = __ldg(reinterpret_cast<const uint4 *>(srow[u]) + pc);
         }
-        const int64_t pos = (int64_t)L + i;
-        const T *cos_row = p.r > 0 ? static_cast<const T *>(p.cos) + pos * p.cs_row : nullptr;
-        const T *sin_row = p.r > 0 ? static_cast<const T *>(p.sin) + pos * p.cs_row : nullptr;
-        if (kind == 1) {
-            const T *src = static_cast<const T *>(p.v_new) + b * p.vn.b + i * p.vn.s + h * p.vn.h;
-            T *dst = static_cast<T *>(p.v_cache) + b * p.vc.b + pos * p.vc.s + h * p.vc.h;
-            reinterpret_cast<uint4 *>(dst)[c] = __ldg(reinterpret_cast<const uint4 *>(src) + c);
-            continue;
+    }
+
+    const int L = seqlen_of(p.seqlens, p.seqlen_scalar, b);
+    // device-side preconditions: the new rows fit the cache and the table
+    if (L < 0 || (int64_t)L + p.s_new > p.cap ||
+        (p.r > 0 && (int64_t)L + rows > p.cs_rows)) {
+        if (threadIdx.x == 0 && blockIdx.y == 0 && i == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
+        return;
+    }
+    const int64_t pos = (int64_t)L + i;
+    if (p.r > 0) {
+        const T *cos_row = static_cast<const T *>(p.cos) + pos * p.cs_row;
+        const T *sin_row = static_cast<const T *>(p.sin) + pos * p.cs_row;
+        for (int j = threadIdx.x; j < half; j += kRopeThreads) {
+            cs_s[j] = Elem<T>::to_f(cos_row[j]);
+            sn_s[j] = Elem<T>::to_f(sin_row[j]);
         }
-        const T *src;
+    }
+    __syncthreads();
+
+#pragma unroll
+    for (int u = 0; u < kRopeOps; ++u) {
+        if (kind[u] < 0) continue;
+        const int c = chunk[u], h = head[u];
         T *dst;
-        if (kind == 0) {
-            src = static_cast<const T *>(p.k_new) + b * p.kn.b + i * p.kn.s + h * p.kn.h;
+        if (kind[u] == 0)
             dst = static_cast<T *>(p.k_cache) + b * p.kc.b + pos * p.kc.s + h * p.kc.h;
-        } else {
-            src = static_cast<const T *>(p.q) + b * p.qs.b + i * p.qs.s + h * p.qs.h;
+        else if (kind[u] == 1)
+            dst = static_cast<T *>(p.v_cache) + b * p.vc.b + pos * p.vc.s + h * p.vc.h;
+        else
             dst = static_cast<T *>(p.q_rot) + (((int64_t)b * p.s_q + i) * p.h_q + h) * p.d_qk;
+        const int t0 = 8 * c;
+        if (kind[u] == 1 || t0 >= p.r) {
+            reinterpret_cast<uint4 *>(dst)[c] = raw[u];   // unrotated dims: bit copy
+            continue;
         }
-        float f[8];
-        load_rotated_chunk<T>(src, c, p.r, inter, cos_row, sin_row, f);
+        float f[8], pf[8];
+        unpack8<T>(raw[u], f);
+        if (inter) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) pf[k] = f[k ^ 1];
+        } else if (chunk_partner) {
+            unpack8<T>(praw[u], pf);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int t = t0 + k;
+                const int partner = t < half ? t + half : t - half;
+                pf[k] = t < p.r ? Elem<T>::to_f(srow[u][partner]) : 0.f;
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int t = t0 + k;
+            if (t < p.r) {
+                int partner, j;
+                bool first;
+                rope_pair_index(t, p.r, inter, partner, j, first);
+                f[k] = rope_elem(f[k], pf[k], cs_s[j], sn_s[j], first);
+            }
+        }
         reinterpret_cast<uint4 *>(dst)[c] = pack8<T>(f);
     }
 }
 
 cudaError_t launch_rope_append(const RopeAppendParams &p, int dtype, cudaStream_t st) {
-    const int64_t total = (int64_t)p.b * p.s_new * p.h_kv * (p.d_qk / 8 + p.d_v / 8) +
-                          (p.q_rot ? (int64_t)p.b * p.s_q * p.h_q * (p.d_qk / 8) : 0);
-    if (total == 0 && !p.zero_word) return cudaSuccess;
-    int64_t blocks = total > 0 ? (total + 255) / 256 : 1;
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    const int rows = std::max(p.q_rot ? p.s_q : 0, p.s_new);
+    const int64_t per_row = (int64_t)p.h_kv * (p.d_qk / 8 + p.d_v / 8) + (p.q_rot ? (int64_t)p.h_q * (p.d_qk / 8) : 0);
+    const int64_t grid_x = (int64_t)p.b * std::max(rows, 1);
+    if ((rows == 0 || p.b == 0) && !p.zero_word) return cudaSuccess;
+    const int64_t grid_y = std::max<int64_t>(1, (per_row + kRopeOps * kRopeThreads - 1) / (kRopeOps * kRopeThreads));
+    if (grid_x > 0x7fffffff || grid_y > 65535) return cudaErrorInvalidConfiguration;
+    dim3 grid((unsigned)std::max<int64_t>(grid_x, 1), (unsigned)grid_y);
     if (dtype == FA_DTYPE_F16)
-        rope_append_kernel<__half><<<(unsigned)blocks, 256, 0, st>>>(p);
+        rope_append_kernel<__half><<<grid, kRopeThreads, 0, st>>>(p);
     else
-        rope_append_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(p);
+        rope_append_kernel<__nv_bfloat16><<<grid, kRopeThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
 
