@@ -50,6 +50,8 @@ def _bind(lib):
     lib.oracle_round.restype = None
     lib.oracle_rope.argtypes = [P, P, i64, i32, P, P, P, i64, i32, i32]
     lib.oracle_rope.restype = i32
+    lib.oracle_rotary.argtypes = [P, P, i64, i32, P, P, P, i64, i32, i32, i32, i32]
+    lib.oracle_rotary.restype = ctypes.c_int
     lib.oracle_kvcache_fwd.argtypes = [i64, i64, i64, i64, i64, i32, i32, i64,
                                        P, P, P, P, P, P, P, i64, i32, i32, P,
                                        i32, d, i32, P, P]
@@ -101,6 +103,51 @@ def rope(x, pos, cos_tab, sin_tab, rotary_dim, interleaved, lib=None):
     tab_rows = cos_tab.shape[0] if cos_tab.ndim == 2 else 0
     rc = lib.oracle_rope(_ptr(x), _ptr(y), rows, d, _ptr(pos), _ptr(cos_tab), _ptr(sin_tab),
                          tab_rows, int(rotary_dim), int(bool(interleaved)))
+    if rc != 0:
+        raise ValueError("position outside the rotary table")
+    return y
+
+
+def rotary_positions(batch, seqlen, seqlen_offsets, cu_seqlens=None):
+    """Table row of every row of a rotary input ([P2] SEQLEN_OFFSET, an int or
+    one value per batch entry; IS_VARLEN).  Batched input [b, s, ...]: row i
+    of entry k is at offset_k + i, returned as [b, s].  Packed input [total,
+    ...] with cu_seqlens [b + 1]: row t of entry k (cu[k] <= t < cu[k+1]) is
+    at offset_k + t - cu[k], returned as [total]."""
+    if cu_seqlens is None:
+        off = np.broadcast_to(np.asarray(seqlen_offsets, dtype=np.int64).reshape(-1, 1)
+                              if np.ndim(seqlen_offsets) else np.int64(seqlen_offsets), (batch, 1))
+        return off + np.arange(seqlen, dtype=np.int64)[None, :]
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    nb = len(cu) - 1
+    off = np.broadcast_to(np.asarray(seqlen_offsets, dtype=np.int64), (nb,))
+    pos = np.empty(cu[-1], dtype=np.int64)
+    for k in range(nb):
+        for t in range(cu[k], cu[k + 1]):
+            pos[t] = off[k] + t - cu[k]
+    return pos
+
+
+def rotary(x, cos_tab, sin_tab, seqlen_offsets=0, rotary_dim=0, interleaved=False, conjugate=False,
+           cu_seqlens=None, fmt=None, lib=None):
+    """Standalone rotary of x ([b, s, h, d], or packed [total, h, d] with
+    cu_seqlens): every head of a row rotated at the row's table position,
+    by the negated angle when `conjugate`, rounded to `fmt`.  float64."""
+    lib = lib or load()
+    x = _f64(x)
+    d = x.shape[-1]
+    if cu_seqlens is None:
+        pos = rotary_positions(x.shape[0], x.shape[1], seqlen_offsets)
+    else:
+        pos = rotary_positions(None, None, seqlen_offsets, cu_seqlens)
+    pos = np.ascontiguousarray(np.broadcast_to(pos[..., None], x.shape[:-1]))
+    cos_tab = _f64(cos_tab)
+    sin_tab = _f64(sin_tab)
+    tab_rows = cos_tab.shape[0] if cos_tab.ndim == 2 else 0
+    y = np.empty_like(x)
+    rows = x.size // d if d else 0
+    rc = lib.oracle_rotary(_ptr(x), _ptr(y), rows, d, _ptr(pos), _ptr(cos_tab), _ptr(sin_tab), tab_rows,
+                           int(rotary_dim), int(bool(interleaved)), int(bool(conjugate)), _FMT[fmt])
     if rc != 0:
         raise ValueError("position outside the rotary table")
     return y

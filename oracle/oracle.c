@@ -144,6 +144,38 @@ int oracle_rope(const double *x, double *y, int64_t rows, int d, const int64_t *
 }
 
 /* ------------------------------------------------------------------ */
+/* Standalone rotary ([P2] "both non-fused and fused kernel": COS/SIN, */
+/* SEQLEN_OFFSET, INTERLEAVED, CONJUGATE).  Row i of x (length d) is   */
+/* rotated at table row pos[i]; with `conjugate` every pair is rotated */
+/* by the negated angle (sin replaced by -sin: the inverse rotation),   */
+/* then the result is rounded to `fmt`.  Returns -1 if a position is   */
+/* outside the table.                                                  */
+/* ------------------------------------------------------------------ */
+int oracle_rotary(const double *x, double *y, int64_t rows, int d, const int64_t *pos,
+                  const double *cos_tab, const double *sin_tab, int64_t tab_rows,
+                  int r, int interleaved, int conjugate, int fmt)
+{
+    int half = r / 2;
+    double *neg = half > 0 ? (double *)malloc(sizeof(double) * half) : NULL;
+    for (int64_t i = 0; i < rows; ++i) {
+        if (r > 0 && (pos[i] < 0 || pos[i] >= tab_rows)) { free(neg); return -1; }
+        const double *cr = r > 0 ? cos_tab + pos[i] * half : NULL;
+        const double *sr = r > 0 ? sin_tab + pos[i] * half : NULL;
+#if ORACLE_PLANT == 11           /* planted: the conjugate flag ignored */
+        conjugate = 0;
+#endif
+        if (r > 0 && conjugate) {
+            for (int j = 0; j < half; ++j) neg[j] = -sr[j];
+            sr = neg;
+        }
+        oracle_rope_row(x + i * d, y + i * d, d, r, interleaved, cr, sr);
+        oracle_round(y + i * d, d, fmt);
+    }
+    free(neg);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* Exact masked softmax attention for one (batch, query head) pair     */
 /* ([P5] Workflow 1 Step 2; causal flag of Workflow 2 Step 2).         */
 /*   q_rows  [s_q, d_qk] with row stride q_ld                          */

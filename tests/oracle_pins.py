@@ -391,4 +391,84 @@ def pin_issue_1402_double_rotation(lib):
         assert np.allclose(sdpa, once, atol=1e-3, rtol=0)
 
 
+def pin_rotary_conjugate_inverts(lib):
+    """CONJUGATE ([P2] standalone rotary) undoes the rotation: in float64 the
+    conjugate of the rotated rows gives the rows back, for both pairings and
+    a partial rotary_dim."""
+    rng = np.random.default_rng(31)
+    c, s, _ = _tables(40, 12)
+    x = rng.standard_normal((3, 5, 2, 16))
+    for inter in (False, True):
+        y = oracle.rotary(x, c, s, [0, 7, 20], 12, inter, False, lib=lib)
+        assert not np.allclose(y, x)
+        back = oracle.rotary(y, c, s, [0, 7, 20], 12, inter, True, lib=lib)
+        assert np.allclose(back, x, atol=1e-13, rtol=0)
+        back = oracle.rotary(oracle.rotary(x, c, s, [0, 7, 20], 12, inter, True, lib=lib), c, s,
+                             [0, 7, 20], 12, inter, False, lib=lib)
+        assert np.allclose(back, x, atol=1e-13, rtol=0)
+
+
+def pin_rotary_conjugate_is_adjoint(lib):
+    """The conjugate rotation is the transpose of the rotation:
+    <R x, y> = <x, R* y> for every row."""
+    rng = np.random.default_rng(32)
+    c, s, _ = _tables(30, 16)
+    x = rng.standard_normal((2, 6, 3, 16))
+    y = rng.standard_normal((2, 6, 3, 16))
+    for inter in (False, True):
+        rx = oracle.rotary(x, c, s, 5, 16, inter, False, lib=lib)
+        cy = oracle.rotary(y, c, s, 5, 16, inter, True, lib=lib)
+        assert np.allclose((rx * y).sum(-1), (x * cy).sum(-1), atol=1e-12, rtol=0)
+
+
+def pin_rotary_conjugate_composes_as_negative_angle(lib):
+    """Rotations compose by adding angles: the conjugate rotation at position p
+    followed by the rotation at position p + q equals the rotation at q
+    (tables built in float64 from base^(-2j/r) angles)."""
+    rng = np.random.default_rng(33)
+    c, s, _ = _tables(64, 8)
+    x = rng.standard_normal((1, 1, 1, 8))
+    for inter in (False, True):
+        for p, q in ((3, 5), (17, 0), (30, 21)):
+            a = oracle.rotary(oracle.rotary(x, c, s, p, 8, inter, True, lib=lib), c, s, p + q, 8, inter,
+                              False, lib=lib)
+            b = oracle.rotary(x, c, s, q, 8, inter, False, lib=lib)
+            assert np.allclose(a, b, atol=1e-12, rtol=0)
+
+
+def pin_rotary_equals_attention_rope_and_rounds(lib):
+    """Without CONJUGATE the standalone rotary is the attention path's RoPE of
+    every head at position offset + i, and the fp16/bf16 results are the
+    float64 ones rounded to nearest even."""
+    rng = np.random.default_rng(34)
+    c, s, _ = _tables(50, 16)
+    x = oracle.round_to(rng.standard_normal((2, 4, 3, 16)), "bf16")
+    offs = np.array([2, 9])
+    y = oracle.rotary(x, c, s, offs, 16, False, False, lib=lib)
+    pos = (offs[:, None] + np.arange(4)[None, :])[:, :, None].repeat(3, axis=2)
+    assert np.array_equal(y, oracle.rope(x, pos, c, s, 16, False, lib=lib))
+    for fmt in ("fp16", "bf16"):
+        assert np.array_equal(oracle.rotary(x, c, s, offs, 16, False, False, fmt=fmt, lib=lib),
+                              oracle.round_to(y, fmt))
+
+
+def pin_rotary_varlen_positions(lib):
+    """Packed rows ([P2] IS_VARLEN): entry k holds rows cu[k] .. cu[k+1] - 1 and
+    row t sits at offset_k + t - cu[k], so the packed result equals the
+    batched result of each entry; an int offset equals the same value per
+    entry."""
+    rng = np.random.default_rng(35)
+    c, s, _ = _tables(40, 8)
+    lens = [3, 1, 5]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    offs = np.array([4, 0, 11])
+    xp = rng.standard_normal((cu[-1], 2, 8))
+    yp = oracle.rotary(xp, c, s, offs, 8, True, True, cu_seqlens=cu, lib=lib)
+    for k, n in enumerate(lens):
+        yb = oracle.rotary(xp[None, cu[k]:cu[k + 1]], c, s, int(offs[k]), 8, True, True, lib=lib)
+        assert np.array_equal(yp[cu[k]:cu[k + 1]], yb[0])
+    assert np.array_equal(oracle.rotary(xp, c, s, 6, 8, False, False, cu_seqlens=cu, lib=lib),
+                          oracle.rotary(xp, c, s, [6, 6, 6], 8, False, False, cu_seqlens=cu, lib=lib))
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -19,6 +19,7 @@ PLANTS = {
     8: "kv head chosen modulo",
     9: "every query row rotated at position L",
     10: "v rows appended one row late",
+    11: "rotary conjugate flag ignored",
 }
 
 
