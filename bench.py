@@ -65,6 +65,8 @@ def is_decode(w: W.Workload) -> bool:
 
 def work_units(w: W.Workload, seqlens):
     """(algorithmic amount per step, unit, bound) for the workload."""
+    if w.mode == "rotary":
+        return W.rotary_bytes(w) / 1e9, "GB/s", "hbm"
     if is_decode(w):
         return W.kvcache_bytes(w, seqlens) / 1e9, "GB/s", "hbm"
     return W.flops(w, seqlens) / 1e12, "TFLOP/s", "tensor"
@@ -139,7 +141,7 @@ def traffic_record(config_key: str, kernel_tag: str):
     """DRAM traffic per launch of the attention kernel on this workload, from
     the committed ncu summary profiles/traffic_<workload>.md, if it was taken
     on the current kernel source (its sha256 prefix must match)."""
-    src = {"decode": "decode.cu", "prefill": "prefill_sm100.cu"}.get(kernel_tag)
+    src = {"decode": "decode.cu", "prefill": "prefill_sm100.cu", "rotary": "rotary.cu"}.get(kernel_tag)
     summ = os.path.join(ROOT, "profiles", f"traffic_{config_key}.md")
     if not src or not os.path.exists(summ):
         return None
@@ -157,6 +159,15 @@ def traffic_record(config_key: str, kernel_tag: str):
 
 # ----------------------------------------------------------------------------- our arm
 def make_step(w, inp_dev, fa):
+    if w.mode == "rotary":
+        x, offs = inp_dev["q"], inp_dev["cache_seqlens"]
+        out = torch.empty_like(x)
+
+        def step():
+            fa.fa_rotary(x, inp_dev["cos"], inp_dev["sin"], offs, w.rotary_dim, w.interleaved, w.conjugate,
+                         out=out)
+        plan = {"path": 0, "launches": 1, "n_splits": 1, "chunk": 0, "workspace_bytes": 0}
+        return step, plan, (out, None)
     if w.mode == "dense":
         q, k, v = inp_dev["q"], inp_dev["k"], inp_dev["v"]
         out = torch.empty(q.shape[:3] + (w.d_v,), dtype=q.dtype, device=q.device)
@@ -217,20 +228,22 @@ def time_steps(step, steps, warmup, stream, flush_buf, barrier):
 def time_e2e(w, inp_host, inp_dev, step_fn_factory, steps, warmup, stream, flush_buf, barrier):
     """End-to-end through the public API: per step, copy the step's inputs from
     pinned host memory, run the call, read out + lse back to pinned host memory."""
-    names = ["q", "k", "v"] if w.mode == "dense" else ["q", "k_new", "v_new", "cache_seqlens"]
+    names = {"dense": ["q", "k", "v"], "rotary": ["q", "cache_seqlens"]}.get(
+        w.mode, ["q", "k_new", "v_new", "cache_seqlens"])
     pinned = {n: inp_host[n].pin_memory() for n in names}
     step, _, (out, lse) = step_fn_factory()
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory() if lse is not None else None
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    d2h = out_h.numel() * out_h.element_size() + (lse_h.numel() * lse_h.element_size() if lse is not None else 0)
 
     def e2e_step():
         for n in names:
             inp_dev[n].copy_(pinned[n], non_blocking=True)
         step()
         out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+        if lse is not None:
+            lse_h.copy_(lse, non_blocking=True)
     times = time_steps(e2e_step, steps, warmup, stream, flush_buf, barrier)
     return times, h2d, d2h
 
@@ -244,7 +257,18 @@ def cpu_sample(w, inp, budget_s):
     b = 0
     while not done or (t_total < budget_s and len(done) < 4 * w.batch):
         bi = b % w.batch
-        if w.mode == "dense":
+        if w.mode == "rotary":
+            # 64 rows of one batch entry, every head
+            i0 = (b // w.batch) * 64 % w.s_q
+            x = inp["q"][bi:bi + 1, i0:i0 + 64].double().numpy()
+            cs, sn = inp["cos"].double().numpy(), inp["sin"].double().numpy()
+            t0 = time.perf_counter()
+            oracle.rotary(x, cs, sn, int(inp["cache_seqlens"][bi]) + i0, w.rotary_dim, w.interleaved,
+                          w.conjugate, fmt=w.dtype)
+            dt = time.perf_counter() - t0
+            amount += W.rotary_bytes(w.scaled(batch=1, s_q=x.shape[1])) / 1e9
+            done.append(f"b{bi}rows{i0}")
+        elif w.mode == "dense":
             # one (batch, head) pair, every query row
             h = (b // w.batch) % w.h_q
             q = inp["q"][bi:bi + 1, :, h:h + 1].double().numpy()
@@ -274,8 +298,8 @@ def cpu_sample(w, inp, budget_s):
             done.append(f"b{bi}")
         t_total += dt
         b += 1
-    desc = (f"float64 oracle, single thread, on {len(done)} "
-            f"{'(batch, head) pairs' if w.mode == 'dense' else 'batch entries'} of the workload "
+    unit_desc = {"dense": "(batch, head) pairs", "rotary": "64-row blocks (all heads)"}.get(w.mode, "batch entries")
+    desc = (f"float64 oracle, single thread, on {len(done)} {unit_desc} of the workload "
             f"({', '.join(done[:8])}{'...' if len(done) > 8 else ''}); inputs converted to float64 "
             f"outside the timed region")
     return amount, t_total, desc
@@ -392,9 +416,9 @@ def run_ours(args):
     # algorithmic amount of one call / the attention kernel's own duration
     # (the whole call's duration if the kernel events could not be timed)
     achieved = amount / ((kernel_ms if kernel_ms else ms) / 1e3)
-    kernel_tag = "decode" if plan["path"] == fa.FA_PATH_DECODE else "prefill"
+    kernel_tag = "rotary" if w.mode == "rotary" else ("decode" if plan["path"] == fa.FA_PATH_DECODE else "prefill")
     kernel_name = {fa.FA_PATH_DECODE: "decode_kernel", fa.FA_PATH_PREFILL: "prefill2_kernel / prefill_kernel",
-                   fa.FA_PATH_DENSE: "prefill2_kernel / prefill_kernel"}.get(plan["path"], "attention kernel")
+                   fa.FA_PATH_DENSE: "prefill2_kernel / prefill_kernel"}.get(plan["path"], "rotary_kernel")
     traffic = traffic_record(args.config, kernel_tag)
     result = {
         "metric": METRIC,

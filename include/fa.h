@@ -213,15 +213,48 @@ int fa_fwd_plan(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, fa_p
  * synchronising `stream`; *status receives FA_OK or an FA_ERR_DEVICE_* code. */
 int fa_device_status(void *stream, int32_t *status);
 
+/* Standalone rotary embedding: the "non-fused" rotary kernel of
+ * ROCm/flash-attention PR #99 (COS/SIN of shape (seqlen, rotary_dim/2),
+ * SEQLEN_OFFSET as an int or one value per batch entry, INTERLEAVED,
+ * CONJUGATE, IS_VARLEN), with the pairing of the RoFormer rotation that
+ * page's "Motivation" describes.
+ *  - x: [b, s, h, d] (batched), or [1, total, h, d] holding packed sequences
+ *    when cu_seqlens is given.  fp16/bf16, head-dim stride 1, other strides
+ *    multiples of 16 bytes, d a multiple of 8 and <= 256.
+ *  - out: same shape and type as x; may be x itself (in place).
+ *  - cos, sin: [S_ro, rotary_dim/2] in x's type (row stride free).
+ *  - seqlen_offsets: int32 device array with one offset per batch entry (or
+ *    per packed sequence), or NULL to use seqlen_offset_scalar for all.
+ *  - cu_seqlens: NULL (batched: row i of entry b is at table row
+ *    offset_b + i), or an int32 device array [n_seqs + 1] of increasing row
+ *    starts (packed: row t of sequence k, cu_seqlens[k] <= t <
+ *    cu_seqlens[k+1], is at table row offset_k + t - cu_seqlens[k]).  Rows
+ *    outside every sequence are copied unchanged.
+ *  - rotary_dim: even, <= d; dims >= rotary_dim are copied.  0: plain copy.
+ *  - interleaved: 0 pairs (j, j + rotary_dim/2), 1 pairs (2j, 2j+1).
+ *  - conjugate: 1 rotates by the negated angle (sin replaced by -sin), the
+ *    inverse rotation.  Pairs are computed in fp32 and rounded to nearest
+ *    even.
+ *  - Device-side precondition: every position lies in [0, S_ro); a row that
+ *    does not is left as it is and FA_ERR_DEVICE_PRECONDITION is recorded
+ *    (fa_device_status).
+ * Allocates nothing; asynchronous on `stream`. */
+int fa_rotary(const fa_tensor *x, const fa_tensor *cos, const fa_tensor *sin,
+              const int32_t *seqlen_offsets, int32_t seqlen_offset_scalar,
+              const int32_t *cu_seqlens, int32_t n_seqs,
+              int32_t rotary_dim, int32_t interleaved, int32_t conjugate,
+              const fa_tensor *out, void *stream);
+
 /* Profiling hook; the pages have no counterpart (it exists so that a
  * benchmark can time the attention kernel alone, apart from the RoPE/append
  * kernel before it and the split-combine kernel after it).
  *  - start, stop: cudaEvent_t handles created by the caller with timing
  *    enabled, or both NULL to switch the hook off.  The library does not own
  *    them; the caller keeps them alive while the hook is on.
- *  - While set, every fa_kvcache_fwd / fa_kvcache_fwd_noalloc / fa_fwd call
- *    records `start` on its stream just before the launch of its attention
- *    kernel (decode, prefill or generic) and `stop` just after it (inside a
+ *  - While set, every fa_kvcache_fwd / fa_kvcache_fwd_noalloc / fa_fwd /
+ *    fa_rotary call records `start` on its stream just before the launch of
+ *    its main kernel (decode, prefill, generic attention or rotary) and
+ *    `stop` just after it (inside a
  *    stream capture as external event-record nodes).  The events sit between
  *    the decode and combine kernels, so while the hook is on the combine
  *    launch no longer overlaps the decode kernel's tail.

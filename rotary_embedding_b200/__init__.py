@@ -157,6 +157,36 @@ def fa_kvcache_fwd(q, k_cache, v_cache, k_new=None, v_new=None, rotary_cos=None,
     return out, lse
 
 
+lib.fa_rotary.argtypes = [_P, _P, _P, _v, _i32, _v, _i32, _i32, _i32, _i32, _P, _v]
+lib.fa_rotary.restype = ctypes.c_int
+
+
+def fa_rotary(x, cos, sin, seqlen_offsets=0, rotary_dim=None, interleaved=False, conjugate=False,
+              cu_seqlens=None, out=None, stream=None):
+    """Standalone rotary embedding of x ([b, s, h, d], or [total, h, d] packed
+    rows with cu_seqlens [n_seqs + 1]): every head of a row rotated at table
+    row offset + i (per batch entry / packed sequence), by the negated angle
+    when `conjugate`.  seqlen_offsets is an int or an int32 CUDA tensor.
+    out may be x (in place); a new tensor is allocated when it is None."""
+    packed = cu_seqlens is not None
+    xv = x.unsqueeze(0) if packed else x
+    if out is None:
+        out = torch.empty_like(x)
+    ov = out.unsqueeze(0) if packed else out
+    if rotary_dim is None:
+        rotary_dim = 2 * cos.shape[1] if cos is not None else 0
+    if isinstance(seqlen_offsets, torch.Tensor):
+        off_ptr, off_scalar = ctypes.c_void_p(seqlen_offsets.data_ptr()), 0
+    else:
+        off_ptr, off_scalar = None, int(seqlen_offsets)
+    cu_ptr = ctypes.c_void_p(cu_seqlens.data_ptr()) if packed else None
+    n_seqs = int(cu_seqlens.numel()) - 1 if packed else 0
+    _check(lib.fa_rotary(_ref(describe(xv)), _ref(describe(cos)), _ref(describe(sin)), off_ptr, off_scalar,
+                         cu_ptr, n_seqs, int(rotary_dim), int(bool(interleaved)), int(bool(conjugate)),
+                         _ref(describe(ov)), _stream_handle(stream, x.device)))
+    return out
+
+
 lib.fa_kvcache_fwd_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _v, _i32, _i32, _i32, _i32, ctypes.c_float,
                                         _P, _v, _v]
 lib.fa_kvcache_fwd_noalloc.restype = ctypes.c_int

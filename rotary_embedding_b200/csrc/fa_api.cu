@@ -354,6 +354,70 @@ extern "C" {
 
 int fa_version(void) { return 100; }
 
+int fa_rotary(const fa_tensor *x, const fa_tensor *cos, const fa_tensor *sin,
+              const int32_t *seqlen_offsets, int32_t seqlen_offset_scalar,
+              const int32_t *cu_seqlens, int32_t n_seqs,
+              int32_t rotary_dim, int32_t interleaved, int32_t conjugate,
+              const fa_tensor *out, void *stream) {
+    g_last_error[0] = 0;
+    Dims4 xd, od;
+    int rc;
+    if ((rc = check_tensor(x, "x", 4, 0, &xd))) return rc;
+    if ((rc = check_tensor(out, "out", 4, x->dtype, &od))) return rc;
+    for (int k = 0; k < 4; ++k)
+        if (xd.n[k] != od.n[k]) return fail(FA_ERR_INVALID_ARG, "out must have the shape of x");
+    const int64_t d = xd.n[3];
+    if (d % 8 || d > 256) return fail(FA_ERR_UNSUPPORTED, "rotary needs d a multiple of 8 and <= 256 (got %lld)",
+                                      (long long)d);
+    if (rotary_dim < 0 || rotary_dim % 2 || rotary_dim > d)
+        return fail(FA_ERR_INVALID_ARG, "rotary_dim must be even and <= d (got %d)", rotary_dim);
+    if (cu_seqlens && (xd.n[0] != 1 || n_seqs < 1))
+        return fail(FA_ERR_INVALID_ARG, "packed rows need x of shape [1, total, h, d] and n_seqs >= 1");
+    if (!cu_seqlens && n_seqs != 0) return fail(FA_ERR_INVALID_ARG, "n_seqs without cu_seqlens");
+    int64_t s_ro = 0, cs_row = 0;
+    if (rotary_dim > 0) {
+        if (!cos || !sin) return fail(FA_ERR_INVALID_ARG, "cos and sin are needed when rotary_dim > 0");
+        Dims4 dc, ds;
+        if ((rc = check_tensor(cos, "cos", 2, x->dtype, &dc, false))) return rc;
+        if ((rc = check_tensor(sin, "sin", 2, x->dtype, &ds, false))) return rc;
+        if (dc.n[0] != ds.n[0] || dc.n[1] != ds.n[1] || dc.s[0] != ds.s[0])
+            return fail(FA_ERR_INVALID_ARG, "cos and sin must have the same shape and strides");
+        if (dc.n[1] < rotary_dim / 2)
+            return fail(FA_ERR_INVALID_ARG, "cos/sin need rotary_dim/2 = %d columns (got %lld)", rotary_dim / 2,
+                        (long long)dc.n[1]);
+        s_ro = dc.n[0];
+        cs_row = dc.n[0] > 1 ? dc.s[0] : dc.n[1];
+    }
+    const int64_t rows = xd.n[0] * xd.n[1];
+    if (rows == 0 || xd.n[2] == 0 || d == 0) return FA_OK;
+    int32_t *status = status_word();
+    if (!status) return fail(FA_ERR_CUDA, "no CUDA device");
+    RotaryParams p{};
+    p.status = status;
+    p.x = x->data;
+    p.xs = s3(xd);
+    p.out = out->data;
+    p.os = s3(od);
+    p.cos = rotary_dim > 0 ? cos->data : nullptr;
+    p.sin = rotary_dim > 0 ? sin->data : nullptr;
+    p.cs_row = cs_row;
+    p.cs_rows = s_ro;
+    p.offsets = seqlen_offsets;
+    p.offset_scalar = seqlen_offset_scalar;
+    p.cu_seqlens = cu_seqlens;
+    p.n_seqs = cu_seqlens ? n_seqs : 0;
+    p.rows = rows;
+    p.s = (int)xd.n[1];
+    p.h = (int)xd.n[2];
+    p.d = (int)d;
+    p.r = rotary_dim;
+    p.interleaved = interleaved ? 1 : 0;
+    p.conjugate = conjugate ? 1 : 0;
+    cudaError_t e = launch_rotary(p, x->dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "rotary launch");
+    return FA_OK;
+}
+
 int fa_set_kernel_events(void *start, void *stop) {
     if ((start == nullptr) != (stop == nullptr))
         return fail(FA_ERR_INVALID_ARG, "fa_set_kernel_events: pass both events or neither");

@@ -61,6 +61,27 @@ struct DecodeParams {
     int *pool;     // work-pool counter (zeroed by the RoPE/append kernel)
 };
 
+// Standalone rotary (fa_rotary): x [b, s, h, d] with element strides xs
+// (batch, row, head), out likewise.  Row R = b * s + i; batched: position
+// offsets[b] + i.  Packed (b = 1): rows cu[k] .. cu[k+1]-1 are sequence k and
+// row R sits at offsets[k] + R - cu[k].
+struct RotaryParams {
+    int32_t *status;
+    const void *x;
+    Strides3 xs;
+    void *out;
+    Strides3 os;
+    const void *cos, *sin;
+    int64_t cs_row, cs_rows;
+    const int32_t *offsets;  // [b] or [n_seqs]; nullptr: offset_scalar
+    int32_t offset_scalar;
+    const int32_t *cu_seqlens;  // [n_seqs + 1] or nullptr (batched)
+    int n_seqs;
+    int64_t rows;   // b * s, or total packed rows
+    int s;          // batched: rows per batch entry
+    int h, d, r, interleaved, conjugate;
+};
+
 // Generic attention (any supported head dim): keys from k/v (dense) or
 // from the cache after the append kernel ran.
 struct SimtAttnParams {
@@ -109,6 +130,7 @@ int set_last_error(int code, const char *msg);
 void kernel_event(int which, cudaStream_t st);
 
 cudaError_t launch_rope_append(const RopeAppendParams &p, int dtype, cudaStream_t st);
+cudaError_t launch_rotary(const RotaryParams &p, int dtype, cudaStream_t st);
 bool prefill_supported(int d_qk, int d_v);
 int prefill_block_n(int d_qk, int d_v, int tiles_per_cta);  // key rows per K/V tile (TMA box rows)
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &tmQ, const CUtensorMap &tmK,

@@ -31,7 +31,7 @@ _DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    mode: str                 # "kvcache" (fa_kvcache_fwd) or "dense" (fa_fwd)
+    mode: str                 # "kvcache" (fa_kvcache_fwd), "dense" (fa_fwd) or "rotary" (fa_rotary)
     dtype: str                # "fp16" | "bf16"
     batch: int
     h_q: int
@@ -51,6 +51,7 @@ class Workload:
     dist: str = "randn"       # "randn" (N(0,1)) or "rand" (U[0,1))
     kv_is_q: bool = False     # the issue-#1402 reproducer passes key = value = query
     zero_cache: bool = False
+    conjugate: bool = False   # rotary mode: rotate by the negated angle
 
     @property
     def torch_dtype(self):
@@ -89,7 +90,15 @@ MLA_DECODE = Workload(
     dtype="bf16", batch=4, h_q=16, h_kv=16, d_qk=192, d_v=128, s_q=1, cap=16384,
     seqlens=(16383, 16383), causal=True)
 
+# The standalone rotary kernel (the next step widened from the path): q of a
+# long prefill, rotated in place of the attention kernel's fused RoPE.
+ROTARY_Q = Workload(
+    name="rotary-q bf16 b4 s4096 h32 d128 rope128 half-split offsets~U{0..4096}", mode="rotary",
+    dtype="bf16", batch=4, h_q=32, h_kv=32, d_qk=128, d_v=128, s_q=4096, cap=8192,
+    seqlens=(0, 4096), rotary_dim=128, interleaved=False)
+
 CONFIGS = {
+    "rotary-q": ROTARY_Q,
     "issue-repro": ISSUE_REPRO,
     "gqa-decode": GQA_DECODE,
     "chunked-prefill": CHUNKED_PREFILL,
@@ -121,6 +130,13 @@ def make_inputs(w: Workload, seed: int = 0) -> dict:
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     dt = w.torch_dtype
+    if w.mode == "rotary":
+        # x as "q" [b, s, h, d]; per-batch position offsets as "cache_seqlens"
+        q = _draw(g, (w.batch, w.s_q, w.h_q, w.d_qk), w.dist, dt)
+        lo, hi = w.seqlens
+        offs = torch.randint(lo, hi + 1, (w.batch,), generator=g, dtype=torch.int32)
+        cos, sin = rotary_tables(w.cap, w.rotary_dim, w.rotary_base, dt)
+        return {"q": q, "cache_seqlens": offs, "cos": cos, "sin": sin}
     if w.mode == "dense":
         q = _draw(g, (w.batch, w.s_q, w.h_q, w.d_qk), w.dist, dt)
         k = _draw(g, (w.batch, w.s_k, w.h_kv, w.d_qk), w.dist, dt)
@@ -145,6 +161,14 @@ def make_inputs(w: Workload, seed: int = 0) -> dict:
     if w.rotary_dim:
         out["cos"], out["sin"] = rotary_tables(w.cap, w.rotary_dim, w.rotary_base, dt)
     return out
+
+
+def rotary_bytes(w: Workload) -> int:
+    """Algorithmic bytes of one standalone rotary call: x read, out written,
+    and the cos/sin row of every row read."""
+    e = 2
+    return (2 * w.batch * w.s_q * w.h_q * w.d_qk * e
+            + w.batch * w.s_q * w.rotary_dim * e)
 
 
 def kvcache_bytes(w: Workload, seqlens) -> int:
