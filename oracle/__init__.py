@@ -54,9 +54,9 @@ def _bind(lib):
     lib.oracle_rotary.restype = ctypes.c_int
     lib.oracle_kvcache_fwd.argtypes = [i64, i64, i64, i64, i64, i32, i32, i64,
                                        P, P, P, P, P, P, P, i64, i32, i32, P,
-                                       i32, d, i32, P, P]
+                                       i32, d, i32, P, P, i64, i64]
     lib.oracle_kvcache_fwd.restype = i32
-    lib.oracle_fwd.argtypes = [i64, i64, i64, i64, i64, i32, i32, P, P, P, i32, d, P, P]
+    lib.oracle_fwd.argtypes = [i64, i64, i64, i64, i64, i32, i32, P, P, P, i32, d, P, P, i64, i64]
     lib.oracle_fwd.restype = i32
     return lib
 
@@ -155,6 +155,7 @@ def rotary(x, cos_tab, sin_tab, seqlen_offsets=0, rotary_dim=0, interleaved=Fals
 
 def kvcache_fwd(q, k_cache, v_cache, k_new, v_new, cos_tab, sin_tab, cache_seqlens,
                 rotary_dim=0, interleaved=False, causal=False, scale=None, fmt=None,
+                window=(-1, -1),
                 lib=None):
     """The whole attn_with_kvcache path in float64.
 
@@ -192,14 +193,16 @@ def kvcache_fwd(q, k_cache, v_cache, k_new, v_new, cos_tab, sin_tab, cache_seqle
                                 _ptr(q), _ptr(kc), _ptr(vc), _ptr(kn), _ptr(vn),
                                 _ptr(ct), _ptr(st), tab_rows, r, int(bool(interleaved)),
                                 _ptr(seql), int(bool(causal)), float(scale), _FMT[fmt],
-                                _ptr(out), _ptr(lse))
+                                _ptr(out), _ptr(lse), int(window[0]), int(window[1]))
     if rc != 0:
         raise ValueError(f"oracle_kvcache_fwd rejected its arguments (code {rc})")
     return out, lse, kc, vc
 
 
-def fwd(q, k, v, causal=False, scale=None, lib=None):
-    """Cache-less attention in float64: returns (out [b,s_q,h_q,d_v], lse [b,h_q,s_q])."""
+def fwd(q, k, v, causal=False, scale=None, lib=None, window=(-1, -1)):
+    """Cache-less attention in float64: returns (out [b,s_q,h_q,d_v], lse [b,h_q,s_q]).
+    window = (left, right): query i (at key position a = i + s_k - s_q) sees keys
+    a - left .. a + right; -1 leaves that side unbounded."""
     lib = lib or load()
     q, k, v = _f64(q), _f64(k), _f64(v)
     b, s_q, h_q, d_qk = q.shape
@@ -210,7 +213,8 @@ def fwd(q, k, v, causal=False, scale=None, lib=None):
     out = np.zeros((b, s_q, h_q, d_v))
     lse = np.zeros((b, h_q, s_q))
     rc = lib.oracle_fwd(b, s_q, s_k, h_q, h_kv, d_qk, d_v, _ptr(q), _ptr(k), _ptr(v),
-                        int(bool(causal)), float(scale), _ptr(out), _ptr(lse))
+                        int(bool(causal)), float(scale), _ptr(out), _ptr(lse), int(window[0]),
+                        int(window[1]))
     if rc != 0:
         raise ValueError(f"oracle_fwd rejected its arguments (code {rc})")
     return out, lse

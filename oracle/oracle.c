@@ -188,51 +188,60 @@ static void attend_one_head(const double *q_rows, int64_t q_ld,
                             const double *k_rows, int64_t k_ld,
                             const double *v_rows, int64_t v_ld,
                             int64_t s_q, int64_t N, int d_qk, int d_v,
-                            int causal, double scale,
+                            int causal, int64_t win_left, int64_t win_right, double scale,
                             double *out, int64_t o_ld, double *lse, double *scores)
 {
     for (int64_t i = 0; i < s_q; ++i) {
-        /* keys visible to query i: all N, or j <= i + N - s_q when causal */
-        int64_t n_vis = N;
+        /* keys visible to query i (aligned bottom-right at a = i + N - s_q):
+         * lo <= j <= hi with hi = a when causal, a + win_right when that
+         * bound is given, and lo = a - win_left when that bound is given
+         * ("optimizing-attention-flash", window_size=(left, right), -1 = none) */
+        int64_t a = i + N - s_q;
+        int64_t hi = N - 1, lo = 0;
         if (causal) {
-            int64_t last = i + N - s_q;          /* last visible key index */
+            int64_t last = a;                    /* last visible key index */
 #if ORACLE_PLANT == 4            /* planted: top-left instead of bottom-right alignment */
             last = i;
 #elif ORACLE_PLANT == 5          /* planted: diagonal excluded */
-            last = i + N - s_q - 1;
+            last = a - 1;
 #endif
-            n_vis = last + 1;
-            if (n_vis < 0) n_vis = 0;
-            if (n_vis > N) n_vis = N;
+            hi = last;
         }
+        if (win_right >= 0 && a + win_right < hi) hi = a + win_right;
+        if (win_left >= 0) lo = a - win_left;
+#if ORACLE_PLANT == 12           /* planted: left window one key short */
+        if (win_left >= 0) lo = a - win_left + 1;
+#endif
+        if (lo < 0) lo = 0;
+        if (hi > N - 1) hi = N - 1;
         double *o = out + i * o_ld;
-        if (n_vis == 0) {
+        if (hi < lo) {
             for (int t = 0; t < d_v; ++t) o[t] = 0.0;
             lse[i] = -INFINITY;
             continue;
         }
         const double *qi = q_rows + i * q_ld;
         double m = -INFINITY;
-        for (int64_t j = 0; j < n_vis; ++j) {
+        for (int64_t j = lo; j <= hi; ++j) {
             const double *kj = k_rows + j * k_ld;
             double dot = 0.0;
             for (int t = 0; t < d_qk; ++t) dot += qi[t] * kj[t];
 #if ORACLE_PLANT == 6            /* planted: scale dropped */
-            scores[j] = dot;
+            scores[j - lo] = dot;
 #else
-            scores[j] = scale * dot;
+            scores[j - lo] = scale * dot;
 #endif
-            if (scores[j] > m) m = scores[j];
+            if (scores[j - lo] > m) m = scores[j - lo];
         }
         double l = 0.0;
-        for (int64_t j = 0; j < n_vis; ++j) {
-            scores[j] = exp(scores[j] - m);
-            l += scores[j];
+        for (int64_t j = lo; j <= hi; ++j) {
+            scores[j - lo] = exp(scores[j - lo] - m);
+            l += scores[j - lo];
         }
         for (int t = 0; t < d_v; ++t) o[t] = 0.0;
-        for (int64_t j = 0; j < n_vis; ++j) {
+        for (int64_t j = lo; j <= hi; ++j) {
             const double *vj = v_rows + j * v_ld;
-            double p = scores[j] / l;
+            double p = scores[j - lo] / l;
             for (int t = 0; t < d_v; ++t) o[t] += p * vj[t];
         }
 #if ORACLE_PLANT == 7            /* planted: max term dropped from lse */
@@ -268,7 +277,7 @@ int oracle_kvcache_fwd(int64_t b, int64_t s_q, int64_t s_new, int64_t h_q, int64
                        const double *cos_tab, const double *sin_tab, int64_t tab_rows,
                        int r, int interleaved, const int32_t *cache_seqlens,
                        int causal, double scale, int fmt,
-                       double *out, double *lse)
+                       double *out, double *lse, int64_t win_left, int64_t win_right)
 {
     if (h_kv <= 0 || h_q % h_kv != 0) return -1;
     if (r < 0 || r % 2 != 0 || r > d_qk) return -2;
@@ -330,7 +339,7 @@ int oracle_kvcache_fwd(int64_t b, int64_t s_q, int64_t s_new, int64_t h_q, int64
             attend_one_head(qrot + h * d_qk, h_q * d_qk,
                             k_cache + (bi * cap * h_kv + hk) * d_qk, h_kv * d_qk,
                             v_cache + (bi * cap * h_kv + hk) * d_v, h_kv * d_v,
-                            s_q, N, d_qk, d_v, causal, scale,
+                            s_q, N, d_qk, d_v, causal, win_left, win_right, scale,
                             out + (bi * s_q * h_q + h) * d_v, h_q * d_v,
                             lse + (bi * h_q + h) * s_q, scores);
         }
@@ -347,7 +356,7 @@ int oracle_kvcache_fwd(int64_t b, int64_t s_q, int64_t s_new, int64_t h_q, int64
 /* ------------------------------------------------------------------ */
 int oracle_fwd(int64_t b, int64_t s_q, int64_t s_k, int64_t h_q, int64_t h_kv,
                int d_qk, int d_v, const double *q, const double *k, const double *v,
-               int causal, double scale, double *out, double *lse)
+               int causal, double scale, double *out, double *lse, int64_t win_left, int64_t win_right)
 {
     if (h_kv <= 0 || h_q % h_kv != 0) return -1;
     int64_t group = h_q / h_kv;
@@ -359,7 +368,7 @@ int oracle_fwd(int64_t b, int64_t s_q, int64_t s_k, int64_t h_q, int64_t h_kv,
             attend_one_head(q + (bi * s_q * h_q + h) * d_qk, h_q * d_qk,
                             k + (bi * s_k * h_kv + hk) * d_qk, h_kv * d_qk,
                             v + (bi * s_k * h_kv + hk) * d_v, h_kv * d_v,
-                            s_q, s_k, d_qk, d_v, causal, scale,
+                            s_q, s_k, d_qk, d_v, causal, win_left, win_right, scale,
                             out + (bi * s_q * h_q + h) * d_v, h_q * d_v,
                             lse + (bi * h_q + h) * s_q, scores);
         }

@@ -471,4 +471,71 @@ def pin_rotary_varlen_positions(lib):
                           oracle.rotary(xp, c, s, [6, 6, 6], 8, False, False, cu_seqlens=cu, lib=lib))
 
 
+def pin_window_covering_everything_is_no_window(lib):
+    """A window wider than the sequence ("optimizing-attention-flash",
+    window_size=(left, right)) changes nothing: equal to (-1, -1)."""
+    rng = np.random.default_rng(41)
+    q, k, v = (rng.standard_normal((2, 6, 2, 8)) for _ in range(3))
+    for causal in (False, True):
+        a = oracle.fwd(q, k, v, causal=causal, scale=0.5, lib=lib)
+        b = oracle.fwd(q, k, v, causal=causal, scale=0.5, lib=lib, window=(6, 6))
+        assert np.allclose(a[0], b[0], atol=1e-14) and np.allclose(a[1], b[1], atol=1e-14)
+
+
+def pin_window_zero_sees_only_the_aligned_key(lib):
+    """window (0, 0): query i sees only key a = i + s_k - s_q, so out = v[a]
+    exactly and lse = scale q.k[a] (the single-key case)."""
+    rng = np.random.default_rng(42)
+    q = rng.standard_normal((1, 3, 2, 8))
+    k = rng.standard_normal((1, 7, 2, 8))
+    v = rng.standard_normal((1, 7, 2, 5))
+    out, lse = oracle.fwd(q, k, v, causal=False, scale=0.3, lib=lib, window=(0, 0))
+    for i in range(3):
+        a = i + 7 - 3
+        assert np.array_equal(out[0, i], v[0, a])
+        for h in range(2):
+            assert np.isclose(lse[0, h, i], 0.3 * q[0, i, h] @ k[0, a, h], atol=1e-14)
+
+
+def pin_window_left_matches_slice_softmax(lib):
+    """Causal with a left window w: query i attends to keys a - w .. a, the
+    textbook softmax over that slice (scipy), and keys outside the window do
+    not matter."""
+    from scipy.special import softmax, logsumexp
+    rng = np.random.default_rng(43)
+    q = rng.standard_normal((1, 5, 1, 8))
+    k = rng.standard_normal((1, 9, 1, 8))
+    v = rng.standard_normal((1, 9, 1, 4))
+    w = 2
+    out, lse = oracle.fwd(q, k, v, causal=True, scale=0.4, lib=lib, window=(w, -1))
+    for i in range(5):
+        a = i + 9 - 5
+        lo = max(0, a - w)
+        sc = 0.4 * k[0, lo:a + 1, 0] @ q[0, i, 0]
+        assert np.allclose(out[0, i, 0], softmax(sc) @ v[0, lo:a + 1, 0], atol=1e-13)
+        assert np.isclose(lse[0, 0, i], logsumexp(sc), atol=1e-13)
+    # perturbing a key outside every window leaves the result unchanged
+    k2, v2 = k.copy(), v.copy()
+    k2[0, 0] += 5.0
+    v2[0, 0] -= 3.0
+    out2, lse2 = oracle.fwd(q, k2, v2, causal=True, scale=0.4, lib=lib, window=(w, -1))
+    assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
+
+
+def pin_window_in_kvcache_mode(lib):
+    """The window applies to the cache path too, on the keys now in the cache:
+    a decode row (s_new 1) with window (w, -1) equals plain attention over the
+    last w + 1 keys."""
+    rng = np.random.default_rng(44)
+    kc = rng.standard_normal((1, 12, 1, 8))
+    vc = rng.standard_normal((1, 12, 1, 8))
+    q = rng.standard_normal((1, 1, 1, 8))
+    kn = rng.standard_normal((1, 1, 1, 8))
+    vn = rng.standard_normal((1, 1, 1, 8))
+    out, lse, kc2, vc2 = oracle.kvcache_fwd(q, kc, vc, kn, vn, None, None, [9], causal=True, scale=0.5,
+                                            window=(3, -1), lib=lib)
+    ref, rlse = oracle.fwd(q, kc2[:, 6:10], vc2[:, 6:10], causal=False, scale=0.5, lib=lib)
+    assert np.allclose(out, ref, atol=1e-14) and np.allclose(lse, rlse, atol=1e-14)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

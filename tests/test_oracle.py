@@ -20,6 +20,7 @@ PLANTS = {
     9: "every query row rotated at position L",
     10: "v rows appended one row late",
     11: "rotary conjugate flag ignored",
+    12: "left window one key short",
 }
 
 
