@@ -174,7 +174,7 @@ def make_step(w, inp_dev, fa):
         lse = torch.empty((w.batch, w.h_q, w.s_q), dtype=torch.float32, device=q.device)
 
         def step():
-            fa.fa_fwd(q, k, v, causal=w.causal, softmax_scale=w.scale or None, out=out, lse=lse)
+            fa.fa_fwd(q, k, v, causal=w.causal, softmax_scale=w.scale or None, out=out, lse=lse, window=w.window)
         plan = fa.fa_fwd_plan(q, k, v)
         return step, plan, (out, lse)
     d = inp_dev
@@ -276,7 +276,7 @@ def cpu_sample(w, inp, budget_s):
             k = inp["k"][bi:bi + 1, :, hk:hk + 1].double().numpy()
             v = inp["v"][bi:bi + 1, :, hk:hk + 1].double().numpy()
             t0 = time.perf_counter()
-            oracle.fwd(q, k, v, causal=w.causal, scale=w.softmax_scale())
+            oracle.fwd(q, k, v, causal=w.causal, scale=w.softmax_scale(), window=w.window)
             dt = time.perf_counter() - t0
             sub = w.scaled(batch=1, h_q=1, h_kv=1)
             amount += W.flops(sub) / 1e12

@@ -186,6 +186,28 @@ int fa_fwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
            int32_t causal, float scale, const fa_tensor *out, float *lse,
            void *workspace, size_t workspace_bytes, void *stream);
 
+/* Sliding-window forms of fa_kvcache_fwd and fa_fwd: the window_size=(left,
+ * right) of the "optimizing-attention-flash" page (Workflow 2 Steps 2-3;
+ * (-1, -1) means no window).  Query row i, aligned bottom-right at key
+ * position a = i + N - s_q (N = keys), sees keys a - window_left ..
+ * a + window_right (each bound -1 = unbounded on that side), and with causal
+ * also no key past a.  Every other argument, and the behaviour with
+ * (-1, -1), is that of fa_kvcache_fwd / fa_fwd (which call these).  A row
+ * with no visible key gets out = 0 and lse = -inf.  Returns
+ * FA_ERR_INVALID_ARG for bounds below -1. */
+int fa_kvcache_fwd_window(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
+                          const fa_tensor *k_new, const fa_tensor *v_new,
+                          const fa_tensor *cos, const fa_tensor *sin,
+                          const int32_t *cache_seqlens, int32_t cache_seqlens_scalar,
+                          int32_t rotary_dim, int32_t interleaved, int32_t causal,
+                          int32_t window_left, int32_t window_right, float scale,
+                          const fa_tensor *out, float *lse,
+                          void *workspace, size_t workspace_bytes, void *stream);
+int fa_fwd_window(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
+                  int32_t causal, int32_t window_left, int32_t window_right, float scale,
+                  const fa_tensor *out, float *lse,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
 /* Workspace bytes fa_fwd needs for these shapes. */
 int fa_fwd_workspace_size(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
                           size_t *bytes);

@@ -61,6 +61,11 @@ lib.fa_kvcache_workspace_size.argtypes = [_P, _P, _P, _P, _i32, ctypes.POINTER(c
 lib.fa_kvcache_workspace_size.restype = ctypes.c_int
 lib.fa_fwd.argtypes = [_P, _P, _P, _i32, ctypes.c_float, _P, _v, _v, ctypes.c_size_t, _v]
 lib.fa_fwd.restype = ctypes.c_int
+lib.fa_fwd_window.argtypes = [_P, _P, _P, _i32, _i32, _i32, ctypes.c_float, _P, _v, _v, ctypes.c_size_t, _v]
+lib.fa_fwd_window.restype = ctypes.c_int
+lib.fa_kvcache_fwd_window.argtypes = [_P, _P, _P, _P, _P, _P, _P, _v, _i32, _i32, _i32, _i32, _i32, _i32,
+                                      ctypes.c_float, _P, _v, _v, ctypes.c_size_t, _v]
+lib.fa_kvcache_fwd_window.restype = ctypes.c_int
 lib.fa_fwd_workspace_size.argtypes = [_P, _P, _P, ctypes.POINTER(ctypes.c_size_t)]
 lib.fa_fwd_workspace_size.restype = ctypes.c_int
 lib.fa_device_status.argtypes = [_v, ctypes.POINTER(ctypes.c_int32)]
@@ -123,11 +128,12 @@ def fa_fwd_workspace_size(q, k, v) -> int:
 def fa_kvcache_fwd(q, k_cache, v_cache, k_new=None, v_new=None, rotary_cos=None, rotary_sin=None,
                    cache_seqlens=0, rotary_dim=None, rotary_interleaved=False, causal=False,
                    softmax_scale=None, out=None, lse=None, workspace=None, return_lse=True,
-                   stream=None):
+                   stream=None, window=(-1, -1)):
     """RoPE of q/k_new at positions cache_seqlens[b] + i, append of the rotated
     k and raw v into k_cache/v_cache (in place), then attention over cache and
     new rows.  Tensors are [batch, seq, heads, dim] CUDA tensors; cache_seqlens
-    is an int or an int32 CUDA tensor [batch].  Returns (out, lse)."""
+    is an int or an int32 CUDA tensor [batch]; window = (left, right) keys
+    around the query's aligned position (-1 = unbounded).  Returns (out, lse)."""
     b, s_q, h_q, _ = q.shape
     d_v = v_cache.shape[3]
     if rotary_cos is not None and rotary_dim is None:
@@ -146,11 +152,11 @@ def fa_kvcache_fwd(q, k_cache, v_cache, k_new=None, v_new=None, rotary_cos=None,
     else:
         seq_ptr, seq_scalar = None, int(cache_seqlens)
     dq = describe(q)
-    _check(lib.fa_kvcache_fwd(
+    _check(lib.fa_kvcache_fwd_window(
         _ref(dq), _ref(describe(k_cache)), _ref(describe(v_cache)), _ref(describe(k_new)),
         _ref(describe(v_new)), _ref(describe(rotary_cos)), _ref(describe(rotary_sin)), seq_ptr,
-        seq_scalar, rotary_dim, int(bool(rotary_interleaved)), int(bool(causal)),
-        float(softmax_scale or 0.0), _ref(describe(out)),
+        seq_scalar, rotary_dim, int(bool(rotary_interleaved)), int(bool(causal)), int(window[0]),
+        int(window[1]), float(softmax_scale or 0.0), _ref(describe(out)),
         ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
         ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None,
         workspace.numel() if workspace is not None else 0, _stream_handle(stream, q.device)))
@@ -226,8 +232,10 @@ def fa_kvcache_fwd_noalloc(q, k_cache, v_cache, k_new=None, v_new=None, rotary_c
 
 
 def fa_fwd(q, k, v, causal=False, softmax_scale=None, out=None, lse=None, workspace=None,
-           return_lse=True, stream=None):
-    """Cache-less attention: q [b, s_q, h_q, d_qk], k/v [b, s_k, h_kv, d]; returns (out, lse)."""
+           return_lse=True, stream=None, window=(-1, -1)):
+    """Cache-less attention: q [b, s_q, h_q, d_qk], k/v [b, s_k, h_kv, d]; window =
+    (left, right) keys around the query's aligned position (-1 = unbounded);
+    returns (out, lse)."""
     b, s_q, h_q, _ = q.shape
     d_v = v.shape[3]
     if out is None:
@@ -238,9 +246,9 @@ def fa_fwd(q, k, v, causal=False, softmax_scale=None, out=None, lse=None, worksp
         ws_bytes = fa_fwd_workspace_size(q, k, v)
         if ws_bytes > 0:
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    _check(lib.fa_fwd(
-        _ref(describe(q)), _ref(describe(k)), _ref(describe(v)), int(bool(causal)),
-        float(softmax_scale or 0.0), _ref(describe(out)),
+    _check(lib.fa_fwd_window(
+        _ref(describe(q)), _ref(describe(k)), _ref(describe(v)), int(bool(causal)), int(window[0]),
+        int(window[1]), float(softmax_scale or 0.0), _ref(describe(out)),
         ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
         ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None,
         workspace.numel() if workspace is not None else 0, _stream_handle(stream, q.device)))

@@ -89,9 +89,9 @@ struct DecodeCfg {
     __host__ __device__ static int qt(int M) { return (M + 7) / 8 * 8; }
     __host__ __device__ static int qbuf_bytes(int M) { return (qt(M) * D_QK * 2 + 1023) / 1024 * 1024; }
     static int merge_bytes(int M) { return 4 * M * (D_V + 2) * 4; }
-    // ring and q barriers, stage items, the 4-int64 schedule, the per-batch table
+    // ring and q barriers, stage items, the 4-int64 schedule, the 16-byte per-batch table
     static int tail_bytes(int B) {
-        return (2 * kDecodeMaxStages + 4) * 8 + kDecodeMaxStages * 16 + 32 + 12 * B + 16;
+        return (2 * kDecodeMaxStages + 4) * 8 + kDecodeMaxStages * 16 + 32 + 16 * B + 16;
     }
     static int stages(int M, int B) {
         const int raw =
@@ -103,11 +103,13 @@ struct DecodeCfg {
     }
 };
 
-// Per-batch facts every thread can recompute: rows N_b and items n_b (0 when
-// the batch entry violates the device-side preconditions, which the
+// Per-batch facts every thread can recompute: rows N_b, the first row `base`
+// of item 0 (0, or with a left window the first visible row of the first
+// query row rounded down to 64) and items n_b covering rows base .. N_b - 1
+// (0 when the batch entry violates the device-side preconditions, which the
 // RoPE/append kernel records and skips in the same way).
 struct SegInfo {
-    int L, N, n_items;
+    int L, N, base, n_items;
 };
 
 __device__ __forceinline__ SegInfo seg_info(const DecodeParams &p, int b) {
@@ -117,7 +119,10 @@ __device__ __forceinline__ SegInfo seg_info(const DecodeParams &p, int b) {
     const bool bad = s.L < 0 || N64 > p.cap ||
                      (p.r > 0 && (int64_t)s.L + (p.s_q > p.s_new ? p.s_q : p.s_new) > p.cs_rows);
     s.N = bad ? 0 : (int)N64;
-    s.n_items = bad ? 0 : (s.N + kDecodeTile - 1) / kDecodeTile;
+    int64_t first = 0, last = -1;
+    visible_keys(0, s.N, p.s_q, p.causal, p.win_left, p.win_right, first, last);
+    s.base = (int)(first < s.N ? first : s.N) & ~(kDecodeTile - 1);
+    s.n_items = bad ? 0 : (s.N - s.base + kDecodeTile - 1) / kDecodeTile;
     return s;
 }
 
@@ -126,7 +131,7 @@ __device__ __forceinline__ int pool_items(int n) { return n / kPoolDen; }
 __device__ __forceinline__ int static_items(int n) { return n - pool_items(n); }
 // Rows of a segment's static part (all of it when the pool holds none).
 __device__ __forceinline__ int static_rows(const SegInfo &sg) {
-    return pool_items(sg.n_items) > 0 ? static_items(sg.n_items) * kDecodeTile : sg.N;
+    return pool_items(sg.n_items) > 0 ? static_items(sg.n_items) * kDecodeTile : sg.N - sg.base;
 }
 
 // An item (b, hk, s) and its segment; POOL selects which items of a segment
@@ -338,7 +343,7 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS)
                         if (!issue_q(itm)) return false;
                     }
                 }
-                const int row0 = itm.s * C::TILE;
+                const int row0 = itm.seg.base + itm.s * C::TILE;
                 // rows >= L of this tile were written by the RoPE/append kernel
                 if (p.s_new > 0 && row0 + C::TILE > itm.seg.L) ensure_waited();
                 const int s = k % NST;
@@ -417,7 +422,7 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS)
     // ---------------- consumers ----------------
     float o[MT][D_V / 8][4];
     float m_r[MT][2], l_r[MT][2];
-    int last_vis[MT][2];
+    int last_vis[MT][2], first_vis[MT][2];
     int s_first = 0;
     int qi = 0;            // pieces started
     uint32_t sQa = 0;
@@ -446,7 +451,10 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS)
 #pragma unroll
                 for (int hr = 0; hr < 2; ++hr) {
                     const int r = mt * 16 + (lane >> 2) + hr * 8;
-                    last_vis[mt][hr] = r < M ? (p.causal ? min(N - 1, r / p.g + N - p.s_q) : N - 1) : -1;
+                    int64_t fv, lv;
+                    visible_keys(r / p.g, N, p.s_q, p.causal, p.win_left, p.win_right, fv, lv);
+                    last_vis[mt][hr] = r < M ? (int)lv : -1;
+                    first_vis[mt][hr] = (int)fv;
                 }
             }
         }
@@ -455,7 +463,7 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS)
         {
             uint8_t *sK = sStage + s * C::STAGE;
             uint8_t *sV = sK + C::KBYTES;
-            const int key0 = itm.s * C::TILE + warp * 16;
+            const int key0 = seg.base + itm.s * C::TILE + warp * 16;
             const bool tail = key0 + 16 > N;
             if (tail) {
                 // rows past the sequence: zero this warp's value rows
@@ -508,7 +516,7 @@ __global__ void __launch_bounds__(160, DecodeOcc<D_V, MT>::CTAS)
                         for (int e = 0; e < 2; ++e) {
                             const int j = key0 + nt * 8 + ((lane & 3) << 1) + e;
                             float v = sacc[mt][nt][hr * 2 + e] * p.scale_log2;
-                            if (j > last_vis[mt][hr]) v = -INFINITY;
+                            if (j > last_vis[mt][hr] || j < first_vis[mt][hr]) v = -INFINITY;
                             vals[nt][e] = v;
                             mx = fmaxf(mx, v);
                         }

@@ -174,7 +174,8 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // the 128-row tile when g divides 128.
 int run_tc_attention(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, const fa_tensor *out,
                      float *lse, bool kvcache, const int32_t *seqlens, int32_t seqlen_scalar, int64_t s_new,
-                     int64_t cap, int causal, float scale_log2, int32_t *status, cudaStream_t st) {
+                     int64_t cap, int causal, int win_left, int win_right, float scale_log2, int32_t *status,
+                     cudaStream_t st) {
     const int64_t b = q->shape[0], s_q = q->shape[1], h_q = q->shape[2], d_qk = q->shape[3];
     const int64_t h_kv = k->shape[2], d_v = v->shape[3];
     const int64_t g = h_q / h_kv;
@@ -197,6 +198,8 @@ int run_tc_attention(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
     p.g = (int)g;
     p.pack = pack;
     p.causal = causal ? 1 : 0;
+    p.win_left = win_left;
+    p.win_right = win_right;
     p.n_q_tiles = (int)((s_q * pack + 127) / 128);
     p.scale_log2 = scale_log2;
     // Two query tiles per CTA keep the tensor core busy during the softmax,
@@ -228,7 +231,7 @@ KvPlan plan_kvcache(int64_t b, int64_t s_q, int64_t h_q, int64_t h_kv, int64_t d
     const int64_t M = g * s_q;
     const int mt = M <= 16 ? 1 : 2;
     // the combine holds up to 512 split slots per output row in registers
-    // the decode kernel stages a 12-byte record per batch entry in shared memory
+    // the decode kernel stages a 16-byte record per batch entry in shared memory
     if (s_q <= 8 && M <= 32 && (s_new == 0 || s_new == s_q) && decode_supported((int)d_qk, (int)d_v, mt) &&
         cap >= 1 && cap <= 512 * 64 && b <= 1024) {
         pl.decode = true;
@@ -501,7 +504,20 @@ int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor
                    int32_t rotary_dim, int32_t interleaved, int32_t causal, float scale,
                    const fa_tensor *out, float *lse, void *workspace, size_t workspace_bytes,
                    void *stream) {
+    return fa_kvcache_fwd_window(q, k_cache, v_cache, k_new, v_new, cos, sin, cache_seqlens,
+                                 cache_seqlens_scalar, rotary_dim, interleaved, causal, -1, -1, scale, out, lse,
+                                 workspace, workspace_bytes, stream);
+}
+
+int fa_kvcache_fwd_window(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
+                          const fa_tensor *k_new, const fa_tensor *v_new, const fa_tensor *cos,
+                          const fa_tensor *sin, const int32_t *cache_seqlens, int32_t cache_seqlens_scalar,
+                          int32_t rotary_dim, int32_t interleaved, int32_t causal, int32_t window_left,
+                          int32_t window_right, float scale, const fa_tensor *out, float *lse, void *workspace,
+                          size_t workspace_bytes, void *stream) {
     g_last_error[0] = 0;
+    if (window_left < -1 || window_right < -1)
+        return fail(FA_ERR_INVALID_ARG, "window bounds must be >= -1 (-1 = unbounded)");
     KvArgs a;
     int rc = validate_kvcache(q, k_cache, v_cache, k_new, v_new, cos, sin, rotary_dim, &a);
     if (rc) return rc;
@@ -603,6 +619,8 @@ int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor
         p.g = (int)(a.h_q / a.h_kv);
         p.r = a.r;
         p.causal = causal ? 1 : 0;
+        p.win_left = window_left;
+        p.win_right = window_right;
         p.cap = a.cap;
         p.scale_log2 = sc * 1.4426950408889634f;
         p.chunk = pl.chunk;
@@ -630,7 +648,8 @@ int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor
         qd.stride[2] = q_att_s.h;
         qd.stride[3] = 1;
         return run_tc_attention(&qd, k_cache, v_cache, out, lse, true, cache_seqlens, cache_seqlens_scalar,
-                                a.s_new, a.cap, causal, sc * 1.4426950408889634f, status, st);
+                                a.s_new, a.cap, causal, window_left, window_right, sc * 1.4426950408889634f,
+                                status, st);
     }
     SimtAttnParams p{};
     p.status = status;
@@ -656,6 +675,8 @@ int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor
     p.d_qk = (int)a.d_qk;
     p.d_v = (int)a.d_v;
     p.causal = causal ? 1 : 0;
+    p.win_left = window_left;
+    p.win_right = window_right;
     p.scale_log2 = sc * 1.4426950408889634f;
     cudaError_t e = launch_simt_attn(p, a.dtype, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
@@ -674,7 +695,15 @@ int fa_fwd_workspace_size(const fa_tensor *q, const fa_tensor *k, const fa_tenso
 
 int fa_fwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, int32_t causal, float scale,
            const fa_tensor *out, float *lse, void *workspace, size_t workspace_bytes, void *stream) {
+    return fa_fwd_window(q, k, v, causal, -1, -1, scale, out, lse, workspace, workspace_bytes, stream);
+}
+
+int fa_fwd_window(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, int32_t causal, int32_t window_left,
+                  int32_t window_right, float scale, const fa_tensor *out, float *lse, void *workspace,
+                  size_t workspace_bytes, void *stream) {
     g_last_error[0] = 0;
+    if (window_left < -1 || window_right < -1)
+        return fail(FA_ERR_INVALID_ARG, "window bounds must be >= -1 (-1 = unbounded)");
     (void)workspace;
     (void)workspace_bytes;
     Dims4 qd, kd, vd, od;
@@ -699,8 +728,8 @@ int fa_fwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, int32_t c
     if (!status) return fail(FA_ERR_CUDA, "no CUDA device");
     const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)d_qk);
     if (prefill_supported((int)d_qk, (int)d_v))
-        return run_tc_attention(q, k, v, out, lse, false, nullptr, 0, 0, 0, causal, sc * 1.4426950408889634f,
-                                status, static_cast<cudaStream_t>(stream));
+        return run_tc_attention(q, k, v, out, lse, false, nullptr, 0, 0, 0, causal, window_left, window_right,
+                                sc * 1.4426950408889634f, status, static_cast<cudaStream_t>(stream));
     SimtAttnParams p{};
     p.status = status;
     p.q = q->data;
@@ -723,6 +752,8 @@ int fa_fwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, int32_t c
     p.d_qk = (int)d_qk;
     p.d_v = (int)d_v;
     p.causal = causal ? 1 : 0;
+    p.win_left = window_left;
+    p.win_right = window_right;
     p.scale_log2 = sc * 1.4426950408889634f;
     cudaError_t e = launch_simt_attn(p, q->dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");

@@ -59,6 +59,7 @@ struct DecodeParams {
     int n_stages;  // K/V ring depth (set by the launcher from the shared-memory budget)
     int n_splits;  // slots per output row (one per 64-row item of the longest segment)
     int *pool;     // work-pool counter (zeroed by the RoPE/append kernel)
+    int win_left, win_right;  // sliding window (keys a - left .. a + right); -1 = unbounded
 };
 
 // Standalone rotary (fa_rotary): x [b, s, h, d] with element strides xs
@@ -101,6 +102,7 @@ struct SimtAttnParams {
     int64_t s_k;   // dense mode key rows
     int64_t cap;   // kvcache mode capacity (precondition check)
     int b, s_q, h_q, h_kv, g, d_qk, d_v, causal;
+    int win_left, win_right;  // sliding window; -1 = unbounded
     float scale_log2;
 };
 
@@ -117,8 +119,22 @@ struct PrefillParams {
     int64_t cap;   // kvcache mode capacity (precondition check)
     int kvcache, b, s_q, h_q, h_kv, g, pack, causal, n_q_tiles;
     int tiles_per_cta;  // 1: one 128-row tile per CTA; 2: two tiles, two softmax warpgroups
+    int win_left, win_right;  // sliding window; -1 = unbounded
     float scale_log2;
 };
+
+// Visible keys of query row i (of s_q) over N keys, aligned bottom-right at
+// a = i + N - s_q: first .. last (first > last: none).  Causal caps the last
+// key at a; a sliding window (left, right) keeps a - left .. a + right.
+__host__ __device__ __forceinline__ void visible_keys(int64_t i, int64_t N, int64_t s_q, int causal, int left,
+                                                      int right, int64_t &first, int64_t &last) {
+    const int64_t a = i + N - s_q;
+    last = N - 1;
+    if (causal && a < last) last = a;
+    if (right >= 0 && a + right < last) last = a + right;
+    first = left >= 0 ? a - left : 0;
+    if (first < 0) first = 0;
+}
 
 int sm_count();
 

@@ -103,10 +103,19 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
     } else {
         N = (int)p.s_k;
     }
-    const int kv_end = p.causal ? max(0, min(N, i_last + N - p.s_q + 1)) : N;
+    // visible keys of the tile's first and last query rows (causal, window)
+    int64_t f_first, l_first, f_last, l_last;
+    visible_keys(i0, N, p.s_q, p.causal, p.win_left, p.win_right, f_first, l_first);
+    visible_keys(i_last, N, p.s_q, p.causal, p.win_left, p.win_right, f_last, l_last);
+    const int kv_end = (int)max((int64_t)0, min((int64_t)N, l_last + 1));
     const int n_kv = (kv_end + kBN - 1) / kBN;
-    // first key index that needs an element mask (diagonal band or sequence end)
-    const int mask_from = p.causal ? max(0, min(N, i0 + N - p.s_q + 1)) : N;
+    const int kb = min((int)(f_first / kBN), n_kv);        // first key tile any row sees
+    const int nblk = n_kv - kb;                             // key tiles kb .. n_kv - 1
+    // key tiles that need an element mask: past the first row's last visible
+    // key (diagonal band, right window or sequence end) or before the last
+    // row's first visible key (left window)
+    const int mask_from = (int)max((int64_t)0, min((int64_t)N, l_first + 1));
+    const int lo_max = (int)f_last;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -135,16 +144,17 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0 && n_kv > 0) {
+        if (lane == 0 && nblk > 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             mbar_arrive_expect_tx(q_full, C::QBYTES);
 #pragma unroll
             for (int c = 0; c < D_QK / 64; ++c) tma_load_4d(sQ + c * C::QBOX, &tmQ, q_full, c * 64, hq0, i0, b);
-            for (int j = 0; j < n_kv; ++j) {
-                const int st = j % C::KST;
-                if (j >= C::KST && !mbar_wait(&kv_empty[st], ((j / C::KST) - 1) & 1, p.status)) break;
+            for (int t = 0; t < nblk; ++t) {
+                const int j = kb + t;
+                const int st = t % C::KST;
+                if (t >= C::KST && !mbar_wait(&kv_empty[st], ((t / C::KST) - 1) & 1, p.status)) break;
                 mbar_arrive_expect_tx(&k_full[st], C::KBYTES);
 #pragma unroll
                 for (int c = 0; c < D_QK / 64; ++c)
@@ -157,29 +167,30 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0 && n_kv > 0) {
+        if (lane == 0 && nblk > 0) {
             const uint32_t idesc_qk = tc::idesc_f16(bf16, kBM, kBN, false);
             const uint32_t idesc_pv = tc::idesc_f16(bf16, kBM, D_V, true);
             const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
             bool ok = mbar_wait(q_full, 0, p.status);
-            auto issue_pv = [&](int jj) -> bool {
-                const int st = jj % C::KST;
-                if (!mbar_wait(p_full, jj & 1, p.status)) return false;
-                if (!mbar_wait(&v_full[st], (jj / C::KST) & 1, p.status)) return false;
+            // tt: index of the key tile relative to kb (stages, parities)
+            auto issue_pv = [&](int tt) -> bool {
+                const int st = tt % C::KST;
+                if (!mbar_wait(p_full, tt & 1, p.status)) return false;
+                if (!mbar_wait(&v_full[st], (tt / C::KST) & 1, p.status)) return false;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int k = 0; k < kBN / 16; ++k) {
                     const uint64_t bdesc = tc::smem_desc(aV + st * C::VBYTES + k * 16 * 128, C::VBOX, 1024);
-                    tc::mma_ts(tmem + C::T_O, tmem + C::T_P + k * 8, bdesc, idesc_pv, (jj > 0 || k > 0) ? 1u : 0u);
+                    tc::mma_ts(tmem + C::T_O, tmem + C::T_P + k * 8, bdesc, idesc_pv, (tt > 0 || k > 0) ? 1u : 0u);
                 }
                 tc::commit(&kv_empty[st]);
                 tc::commit(pv_done);
                 return true;
             };
-            for (int j = 0; j < n_kv && ok; ++j) {
-                const int st = j % C::KST, sb = j & 1;
-                if (!mbar_wait(&k_full[st], (j / C::KST) & 1, p.status)) break;
-                if (j >= 2 && !mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1, p.status)) break;
+            for (int t = 0; t < nblk && ok; ++t) {
+                const int st = t % C::KST, sb = t & 1;
+                if (!mbar_wait(&k_full[st], (t / C::KST) & 1, p.status)) break;
+                if (t >= 2 && !mbar_wait(&s_free[sb], ((t >> 1) - 1) & 1, p.status)) break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int k = 0; k < D_QK / 16; ++k) {
@@ -189,12 +200,12 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
                     tc::mma_ss(tmem + (sb ? C::T_S1 : C::T_S0), adesc, bdesc, idesc_qk, k > 0 ? 1u : 0u);
                 }
                 tc::commit(&s_full[sb]);
-                if (j >= 1 && !issue_pv(j - 1)) {
+                if (t >= 1 && !issue_pv(t - 1)) {
                     ok = false;
                     break;
                 }
             }
-            if (ok) issue_pv(n_kv - 1);
+            if (ok) issue_pv(nblk - 1);
         }
     } else if (warp >= 4) {
         // ------------------------------------------------ softmax warpgroup
@@ -205,14 +216,18 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
         const int i = prow / pack;                     // query position
         const int hq = hq0 + (prow % pack);
         const bool row_valid = i < p.s_q;
-        const int last_vis = row_valid ? (p.causal ? min(N - 1, i + N - p.s_q) : N - 1) : -1;
+        int64_t fv64, lv64;
+        visible_keys(i, N, p.s_q, p.causal, p.win_left, p.win_right, fv64, lv64);
+        const int last_vis = row_valid ? (int)lv64 : -1;
+        const int first_vis = (int)fv64;
         const float c = p.scale_log2;
         float m_ref = -INFINITY;   // raw-score max used as the exponent reference
         float l = 0.f;
         bool ok = true;
-        for (int j = 0; j < n_kv && ok; ++j) {
-            const int sb = j & 1;
-            if (!mbar_wait(&s_full[sb], (j >> 1) & 1, p.status)) {
+        for (int t = 0; t < nblk && ok; ++t) {
+            const int j = kb + t;
+            const int sb = t & 1;
+            if (!mbar_wait(&s_full[sb], (t >> 1) & 1, p.status)) {
                 ok = false;
                 break;
             }
@@ -230,14 +245,14 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
 
             const int j0 = j * kBN;
             float mt = -INFINITY;
-            if (j0 + kBN > mask_from) {
+            if (j0 + kBN > mask_from || j0 < lo_max) {
 #pragma unroll
                 for (int h = 0; h < 4; ++h)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int key = j0 + h * 32 + e;
                         float v = __uint_as_float(sr[h][e]);
-                        v = key <= last_vis ? v : -INFINITY;
+                        v = (key <= last_vis && key >= first_vis) ? v : -INFINITY;
                         sr[h][e] = __float_as_uint(v);
                         mt = fmaxf(mt, v);
                     }
@@ -269,9 +284,9 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
                 }
             l = l * alpha + rs;
 
-            if (j > 0) {
+            if (t > 0) {
                 // O is stable and the P buffer free once PV_{j-1} has completed
-                if (!mbar_wait(pv_done, (j - 1) & 1, p.status)) {
+                if (!mbar_wait(pv_done, (t - 1) & 1, p.status)) {
                     ok = false;
                     break;
                 }
@@ -292,10 +307,10 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
             tc::st32(tmem + lane_addr + C::T_P, pk[0]);
             tc::st32(tmem + lane_addr + C::T_P + 32, pk[1]);
             tc::wait_st();
-            if (p.kvcache && j == n_kv - 1 && j0 + kBN > N) {
+            if (p.kvcache && t == nblk - 1 && j0 + kBN > N) {
                 // cache rows past N_b may hold anything: zero them in the V tile
-                const int st = j % C::KST;
-                if (!mbar_wait(&v_full[st], (j / C::KST) & 1, p.status)) {
+                const int st = t % C::KST;
+                if (!mbar_wait(&v_full[st], (t / C::KST) & 1, p.status)) {
                     ok = false;
                     break;
                 }
@@ -315,7 +330,7 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
             if (lane == 0) mbar_arrive(p_full);
         }
         // ------------------------------------------------ epilogue
-        if (ok && n_kv > 0 && !mbar_wait(pv_done, (n_kv - 1) & 1, p.status)) ok = false;
+        if (ok && nblk > 0 && !mbar_wait(pv_done, (nblk - 1) & 1, p.status)) ok = false;
         tc::fence_after_sync();
         // every lane takes part in the (warp-collective) TMEM loads; only rows
         // inside the sequence are stored
@@ -324,7 +339,7 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
 #pragma unroll
         for (int h = 0; h < D_V / 32; ++h) {
             uint32_t orr[32];
-            if (n_kv > 0) {
+            if (nblk > 0) {
                 tc::ld32(tmem + lane_addr + C::T_O + h * 32, orr);
                 tc::wait_ld();
             } else {
@@ -441,16 +456,26 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
     } else {
         N = (int)p.s_k;
     }
-    int i0[2], n_kv[2], mask_from[2];
+    // per tile: key tiles kb[x] .. n_kv[x] - 1 (causal, window), and the
+    // bounds past which a key tile needs an element mask (see prefill_kernel)
+    int i0[2], n_kv[2], kb[2], mask_from[2], lo_max[2];
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
         i0[x] = (2 * blk + x) * rows_per_tile;
         const int i_last = min(p.s_q, i0[x] + rows_per_tile) - 1;
-        const int kv_end = i0[x] >= p.s_q ? 0 : (p.causal ? max(0, min(N, i_last + N - p.s_q + 1)) : N);
+        int64_t f_first, l_first, f_last, l_last;
+        visible_keys(i0[x], N, p.s_q, p.causal, p.win_left, p.win_right, f_first, l_first);
+        visible_keys(i_last, N, p.s_q, p.causal, p.win_left, p.win_right, f_last, l_last);
+        const int kv_end = i0[x] >= p.s_q ? 0 : (int)max((int64_t)0, min((int64_t)N, l_last + 1));
         n_kv[x] = (kv_end + BN - 1) / BN;
-        mask_from[x] = p.causal ? max(0, min(N, i0[x] + N - p.s_q + 1)) : N;
+        kb[x] = min((int)(f_first / BN), n_kv[x]);
+        mask_from[x] = (int)max((int64_t)0, min((int64_t)N, l_first + 1));
+        lo_max[x] = (int)f_last;
     }
-    const int n_all = max(n_kv[0], n_kv[1]);
+    // key tiles loaded: kb0 .. n_all - 1 (the union of both tiles' ranges)
+    const bool any0 = kb[0] < n_kv[0], any1 = kb[1] < n_kv[1];
+    const int kb0 = any0 && any1 ? min(kb[0], kb[1]) : (any0 ? kb[0] : (any1 ? kb[1] : 0));
+    const int n_all = max(any0 ? n_kv[0] : 0, any1 ? n_kv[1] : 0);
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -482,7 +507,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
     if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0 && n_all > 0) {
+        if (lane == 0 && n_all > kb0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
@@ -492,14 +517,15 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
 #pragma unroll
                 for (int c = 0; c < D_QK / 64; ++c)
                     tma_load_4d(sQ + x * C::QBYTES + c * C::QBOX, &tmQ, q_full, c * 64, hq0, i0[x], b);
-            for (int j = 0; j < n_all; ++j) {
-                const int ks = j % KST, vs = j % VST;
-                if (j >= KST && !mbar_wait(&k_empty[ks], ((j / KST) - 1) & 1, p.status)) break;
+            for (int j = kb0; j < n_all; ++j) {
+                const int u = j - kb0;   // loaded tile index (stages, parities)
+                const int ks = u % KST, vs = u % VST;
+                if (u >= KST && !mbar_wait(&k_empty[ks], ((u / KST) - 1) & 1, p.status)) break;
                 mbar_arrive_expect_tx(&k_full[ks], C::KBYTES);
 #pragma unroll
                 for (int c = 0; c < D_QK / 64; ++c)
                     tma_load_4d(sK + ks * C::KBYTES + c * C::KBOX, &tmK, &k_full[ks], c * 64, hk, j * BN, b);
-                if (j >= VST && !mbar_wait(&v_empty[vs], ((j / VST) - 1) & 1, p.status)) break;
+                if (u >= VST && !mbar_wait(&v_empty[vs], ((u / VST) - 1) & 1, p.status)) break;
                 mbar_arrive_expect_tx(&v_full[vs], C::VBYTES);
 #pragma unroll
                 for (int c = 0; c < D_V / 64; ++c)
@@ -510,7 +536,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         // ------------------------------------------------ MMA issuer
         // The whole warp runs the loop (waits, warp-uniform descriptors); one
         // elected lane issues the MMAs and the commits that track them.
-        if (n_all > 0) {
+        if (n_all > kb0) {
             const bool leader = tc::elect_one();
             const uint32_t idesc_qk = tc::idesc_f16(bf16, kBM, BN, false);
             const uint32_t idesc_pv = tc::idesc_f16(bf16, kBM, D_V, true);
@@ -521,9 +547,10 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             const uint64_t dK0 = tc::smem_desc(smem_addr(sK), 16, 1024);
             const uint64_t dV0 = tc::smem_desc(smem_addr(sV), C::KBOX, 1024);
             bool ok = mbar_wait(q_full, 0, p.status);
+            // key tile j sits in stage (j - kb0) % KST / VST
             auto issue_qk = [&](int x, int j) {
                 const uint64_t dq = dQ0 + (uint64_t)((x * C::QBYTES) >> 4);
-                const uint64_t dk = dK0 + (uint64_t)(((j % KST) * C::KBYTES) >> 4);
+                const uint64_t dk = dK0 + (uint64_t)((((j - kb0) % KST) * C::KBYTES) >> 4);
                 const uint32_t ts = tmem + C::t_s(x);
                 if (leader) {
 #pragma unroll
@@ -537,9 +564,9 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                 __syncwarp();
             };
             auto issue_pv = [&](int x, int j) {
-                const uint64_t dv = dV0 + (uint64_t)(((j % VST) * C::VBYTES) >> 4);
+                const uint64_t dv = dV0 + (uint64_t)((((j - kb0) % VST) * C::VBYTES) >> 4);
                 const uint32_t to = tmem + C::t_o(x), tp = tmem + C::t_s(x);
-                const uint32_t acc0 = j > 0 ? 1u : 0u;
+                const uint32_t acc0 = j > kb[x] ? 1u : 0u;
                 if (leader) {
 #pragma unroll
                     for (int k = 0; k < BN / 16; ++k)
@@ -551,27 +578,30 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                 if (leader) tc::commit(bar);
                 __syncwarp();
             };
-            // prologue: QK of both tiles on key tile 0
+            // prologue: QK of the tiles whose range starts at the first loaded key tile
             if (ok && (ok = mbar_wait(&k_full[0], 0, p.status))) {
                 tc::fence_after_sync();
-                if (n_kv[0] > 0) issue_qk(0, 0);
-                if (n_kv[1] > 0) issue_qk(1, 0);
+                if (any0 && kb[0] == kb0) issue_qk(0, kb0);
+                if (any1 && kb[1] == kb0) issue_qk(1, kb0);
                 commit(&k_empty[0]);
             }
-            for (int j = 0; j < n_all && ok; ++j) {
-                const int vs = j % VST;
+            for (int j = kb0; j < n_all && ok; ++j) {
+                const int u = j - kb0;
+                const int vs = u % VST;
                 const bool next = j + 1 < n_all;
-                const int ks1 = (j + 1) % KST;
-                if (!(ok = mbar_wait(&v_full[vs], (j / VST) & 1, p.status))) break;
-                if (next && !(ok = mbar_wait(&k_full[ks1], ((j + 1) / KST) & 1, p.status))) break;
+                const int ks1 = (u + 1) % KST;
+                if (!(ok = mbar_wait(&v_full[vs], (u / VST) & 1, p.status))) break;
+                if (next && !(ok = mbar_wait(&k_full[ks1], ((u + 1) / KST) & 1, p.status))) break;
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    if (j < n_kv[x]) {
-                        if (!(ok = mbar_wait(&p_full[x], j & 1, p.status))) break;
+                    if (j >= kb[x] && j < n_kv[x]) {
+                        if (!(ok = mbar_wait(&p_full[x], (j - kb[x]) & 1, p.status))) break;
                         tc::fence_after_sync();
                         issue_pv(x, j);
                         if (j + 1 == n_kv[x]) commit(&o_full[x]);
                         if (j + 1 < n_kv[x]) issue_qk(x, j + 1);
+                    } else if (j + 1 == kb[x] && kb[x] < n_kv[x]) {
+                        issue_qk(x, j + 1);   // this tile's range starts at the next key tile
                     }
                 }
                 if (!ok) break;
@@ -590,16 +620,19 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         const int i = prow / pack;
         const int hq = hq0 + (prow % pack);
         const bool row_valid = i < p.s_q;
-        const int last_vis = row_valid ? (p.causal ? min(N - 1, i + N - p.s_q) : N - 1) : -1;
+        int64_t fv64, lv64;
+        visible_keys(i, N, p.s_q, p.causal, p.win_left, p.win_right, fv64, lv64);
+        const int last_vis = row_valid ? (int)lv64 : -1;
+        const int first_vis = (int)fv64;
         const float c = p.scale_log2;
         const uint64_t c2 = f2_pack(c, c);
         const uint32_t s_addr = tmem + lane_addr + C::t_s(x);
         const uint32_t o_addr = tmem + lane_addr + C::t_o(x);
-        const int nk = n_kv[x];
+        const int nk = n_kv[x], jb = kb[x];
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < nk && ok; ++j) {
-            if (!(ok = mbar_wait(&s_full[x], j & 1, p.status))) break;
+        for (int j = jb; j < nk && ok; ++j) {
+            if (!(ok = mbar_wait(&s_full[x], (j - jb) & 1, p.status))) break;
             tc::fence_after_sync();
             const int j0 = j * BN;
             constexpr int NCH = BN / 32;               // 32-column chunks of the S row
@@ -607,14 +640,17 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
 #pragma unroll
             for (int h = 0; h < NCH; ++h) tc::ld32(s_addr + h * 32, sr[h]);
             tc::wait_ld();
-            if (j0 + BN > mask_from[x]) {
-                // diagonal band or sequence end: -inf outside the visible keys
-                // (only these tiles pay for the comparisons)
+            const bool masked = j0 + BN > mask_from[x] || j0 < lo_max[x];
+            if (masked) {
+                // diagonal band, window edge or sequence end: -inf outside the
+                // visible keys (only these tiles pay for the comparisons)
 #pragma unroll
                 for (int h = 0; h < NCH; ++h)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (j0 + h * 32 + e > last_vis) sr[h][e] = __float_as_uint(-INFINITY);
+                    for (int e = 0; e < 32; ++e) {
+                        const int key = j0 + h * 32 + e;
+                        if (key > last_vis || key < first_vis) sr[h][e] = __float_as_uint(-INFINITY);
+                    }
             }
             // row max: one independent three-input chain per chunk
             float mx[NCH];
@@ -669,7 +705,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                     tc::st16(s_addr + h * 16, pk);
                 }
             };
-            if (j0 + BN > mask_from[x])
+            if (masked)
                 exp_row(std::integral_constant<bool, false>());
             else
                 exp_row(std::integral_constant<bool, true>());
@@ -688,8 +724,8 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             if (p.kvcache && j == nk - 1 && j0 + BN > N) {
                 // cache rows past N_b may hold anything: zero them in the V tile
                 // (both tiles' warpgroups do it; the writes are identical)
-                const int vs = j % VST;
-                if (!(ok = mbar_wait(&v_full[vs], (j / VST) & 1, p.status))) break;
+                const int vs = (j - kb0) % VST;
+                if (!(ok = mbar_wait(&v_full[vs], ((j - kb0) / VST) & 1, p.status))) break;
                 uint8_t *vt = sV + vs * C::VBYTES;
                 const int first = N - j0;
                 const int n16 = (BN - first) * 8 * (D_V / 64);
@@ -720,14 +756,14 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             l = l * alpha + (((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7)));
         }
         // ------------------------------------------------ epilogue
-        if (ok && nk > 0 && !mbar_wait(&o_full[x], 0, p.status)) ok = false;
+        if (ok && nk > jb && !mbar_wait(&o_full[x], 0, p.status)) ok = false;
         tc::fence_after_sync();
         T *orow = static_cast<T *>(p.out) + b * p.os.b + (int64_t)i * p.os.s + hq * p.os.h;
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
         for (int h = 0; h < D_V / 32; ++h) {
             uint32_t orr[32];
-            if (nk > 0) {
+            if (nk > jb) {
                 tc::ld32(o_addr + h * 32, orr);
                 tc::wait_ld();
             } else {

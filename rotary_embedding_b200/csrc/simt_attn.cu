@@ -36,7 +36,9 @@ __global__ void __launch_bounds__(256) simt_attn_kernel(const SimtAttnParams p) 
     } else {
         n_keys = p.s_k;
     }
-    const int64_t n_vis = p.causal ? min(n_keys, max((int64_t)0, i + n_keys - p.s_q + 1)) : n_keys;
+    int64_t first_vis, last_vis;
+    visible_keys(i, n_keys, p.s_q, p.causal, p.win_left, p.win_right, first_vis, last_vis);
+    const int64_t n_vis = max((int64_t)0, last_vis + 1);   // keys first_vis .. n_vis - 1
 
     float *sq = sq_all + warp_in_block * p.d_qk;
     const T *qrow = static_cast<const T *>(p.q) + b * p.qs.b + i * p.qs.s + hq * p.qs.h;
@@ -50,7 +52,7 @@ __global__ void __launch_bounds__(256) simt_attn_kernel(const SimtAttnParams p) 
     float m = -INFINITY, l = 0.f;
     const T *kbase = static_cast<const T *>(p.k) + b * p.ks.b + hk * p.ks.h;
     const T *vbase = static_cast<const T *>(p.v) + b * p.vs.b + hk * p.vs.h;
-    for (int64_t j0 = 0; j0 < n_vis; j0 += 32) {
+    for (int64_t j0 = first_vis; j0 < n_vis; j0 += 32) {
         const int64_t j = j0 + lane;
         float s = -INFINITY;
         if (j < n_vis) {

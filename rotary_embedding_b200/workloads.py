@@ -52,6 +52,7 @@ class Workload:
     kv_is_q: bool = False     # the issue-#1402 reproducer passes key = value = query
     zero_cache: bool = False
     conjugate: bool = False   # rotary mode: rotate by the negated angle
+    window: tuple = (-1, -1)  # sliding window (left, right) keys around the aligned position; -1 = none
 
     @property
     def torch_dtype(self):
@@ -97,8 +98,15 @@ ROTARY_Q = Workload(
     dtype="bf16", batch=4, h_q=32, h_kv=32, d_qk=128, d_v=128, s_q=4096, cap=8192,
     seqlens=(0, 4096), rotary_dim=128, interleaved=False)
 
+# Sliding-window prefill (the window_size=(left, right) of the
+# "optimizing-attention-flash" page): causal, 1024 keys to the left.
+WINDOW_PREFILL = Workload(
+    name="window-prefill bf16 b2 h16 s8192 d128 causal window(1024,0)", mode="dense", dtype="bf16",
+    batch=2, h_q=16, h_kv=16, d_qk=128, d_v=128, s_q=8192, s_k=8192, causal=True, window=(1024, 0))
+
 CONFIGS = {
     "rotary-q": ROTARY_Q,
+    "window-prefill": WINDOW_PREFILL,
     "issue-repro": ISSUE_REPRO,
     "gqa-decode": GQA_DECODE,
     "chunked-prefill": CHUNKED_PREFILL,
@@ -195,7 +203,19 @@ def visible_pairs(w: Workload, seqlens=None) -> int:
         s_q = w.s_q
         lens = [int(x) + w.s_q for x in seqlens]
     for n in lens:
-        if not w.causal:
+        if w.window != (-1, -1):
+            # query i at a = i + n - s_q sees keys max(0, a - left) .. min(n - 1, a [causal], a + right)
+            left, right = w.window
+            for i in range(s_q):
+                a = i + n - s_q
+                hi = n - 1
+                if w.causal:
+                    hi = min(hi, a)
+                if right >= 0:
+                    hi = min(hi, a + right)
+                lo = max(0, a - left) if left >= 0 else 0
+                total += max(0, hi - lo + 1)
+        elif not w.causal:
             total += s_q * n
         else:
             # query i sees keys j <= i + n - s_q
