@@ -199,6 +199,28 @@ def kvcache_fwd(q, k_cache, v_cache, k_new, v_new, cos_tab, sin_tab, cache_seqle
     return out, lse, kc, vc
 
 
+def fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal=False, scale=None, lib=None, window=(-1, -1)):
+    """Attention over packed sequences ([P2] IS_VARLEN): q [total_q, h_q, d_qk],
+    k/v [total_k, h_kv, d]; sequence s holds query rows cu_q[s] .. cu_q[s+1]-1
+    and key rows cu_k[s] .. cu_k[s+1]-1, each attended exactly as a batch of
+    one by fwd (bottom-right alignment inside the sequence).  Returns
+    (out [total_q, h_q, d_v], lse [h_q, total_q])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cq = np.asarray(cu_seqlens_q, dtype=np.int64)
+    ck = np.asarray(cu_seqlens_k, dtype=np.int64)
+    out = np.zeros((q.shape[0], q.shape[1], v.shape[2]))
+    lse = np.full((q.shape[1], q.shape[0]), -np.inf)
+    for sidx in range(len(cq) - 1):
+        q0, q1, k0, k1 = cq[sidx], cq[sidx + 1], ck[sidx], ck[sidx + 1]
+        if q1 == q0:
+            continue
+        o, l = fwd(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], causal=causal, scale=scale, lib=lib,
+                   window=window)
+        out[q0:q1] = o[0]
+        lse[:, q0:q1] = l[0]
+    return out, lse
+
+
 def fwd(q, k, v, causal=False, scale=None, lib=None, window=(-1, -1)):
     """Cache-less attention in float64: returns (out [b,s_q,h_q,d_v], lse [b,h_q,s_q]).
     window = (left, right): query i (at key position a = i + s_k - s_q) sees keys

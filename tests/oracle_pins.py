@@ -538,4 +538,26 @@ def pin_window_in_kvcache_mode(lib):
     assert np.allclose(out, ref, atol=1e-14) and np.allclose(lse, rlse, atol=1e-14)
 
 
+def pin_varlen_sequences_are_independent(lib):
+    """Packed sequences ([P2] IS_VARLEN) do not see each other: changing one
+    sequence's keys and values leaves every other sequence's output and lse
+    bit-identical, and a single packed sequence equals the batched call."""
+    rng = np.random.default_rng(51)
+    cq = [0, 3, 3, 10]
+    ck = [0, 5, 9, 21]
+    q = rng.standard_normal((10, 2, 8))
+    k = rng.standard_normal((21, 1, 8))
+    v = rng.standard_normal((21, 1, 4))
+    out, lse = oracle.fwd_varlen(q, k, v, cq, ck, causal=True, lib=lib)
+    k2, v2 = k.copy(), v.copy()
+    k2[9:] += 1.0
+    v2[9:] -= 2.0
+    out2, lse2 = oracle.fwd_varlen(q, k2, v2, cq, ck, causal=True, lib=lib)
+    assert np.array_equal(out[:3], out2[:3]) and np.array_equal(lse[:, :3], lse2[:, :3])
+    assert not np.allclose(out[3:], out2[3:])
+    one, l1 = oracle.fwd_varlen(q[:3], k[:5], v[:5], [0, 3], [0, 5], causal=True, lib=lib)
+    ref, rl = oracle.fwd(q[None, :3], k[None, :5], v[None, :5], causal=True, lib=lib)
+    assert np.array_equal(one, ref[0]) and np.array_equal(l1, rl[0])
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
