@@ -159,6 +159,16 @@ def traffic_record(config_key: str, kernel_tag: str):
 
 # ----------------------------------------------------------------------------- our arm
 def make_step(w, inp_dev, fa):
+    if w.mode == "varlen":
+        q, k, v, cu = inp_dev["q"], inp_dev["k"], inp_dev["v"], inp_dev["cu_seqlens"]
+        out = torch.empty((q.shape[0], q.shape[1], v.shape[2]), dtype=q.dtype, device=q.device)
+        lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
+
+        def step():
+            fa.fa_fwd_varlen(q, k, v, cu, cu, w.s_q, causal=w.causal, softmax_scale=w.scale or None,
+                             window=w.window, out=out, lse=lse)
+        plan = {"path": fa.FA_PATH_DENSE, "launches": 1, "n_splits": 1, "chunk": 0, "workspace_bytes": 0}
+        return step, plan, (out, lse)
     if w.mode == "rotary":
         x, offs = inp_dev["q"], inp_dev["cache_seqlens"]
         out = torch.empty_like(x)
@@ -228,7 +238,8 @@ def time_steps(step, steps, warmup, stream, flush_buf, barrier):
 def time_e2e(w, inp_host, inp_dev, step_fn_factory, steps, warmup, stream, flush_buf, barrier):
     """End-to-end through the public API: per step, copy the step's inputs from
     pinned host memory, run the call, read out + lse back to pinned host memory."""
-    names = {"dense": ["q", "k", "v"], "rotary": ["q", "cache_seqlens"]}.get(
+    names = {"dense": ["q", "k", "v"], "rotary": ["q", "cache_seqlens"],
+             "varlen": ["q", "k", "v", "cu_seqlens"]}.get(
         w.mode, ["q", "k_new", "v_new", "cache_seqlens"])
     pinned = {n: inp_host[n].pin_memory() for n in names}
     step, _, (out, lse) = step_fn_factory()
@@ -257,7 +268,21 @@ def cpu_sample(w, inp, budget_s):
     b = 0
     while not done or (t_total < budget_s and len(done) < 4 * w.batch):
         bi = b % w.batch
-        if w.mode == "rotary":
+        if w.mode == "varlen":
+            # one (sequence, head) pair, every query row
+            cu = inp["cu_seqlens"]
+            h = (b // w.batch) % w.h_q
+            q0, q1 = int(cu[bi]), int(cu[bi + 1])
+            hk = h // (w.h_q // w.h_kv)
+            q = inp["q"][None, q0:q1, h:h + 1].double().numpy()
+            k = inp["k"][None, q0:q1, hk:hk + 1].double().numpy()
+            v = inp["v"][None, q0:q1, hk:hk + 1].double().numpy()
+            t0 = time.perf_counter()
+            oracle.fwd(q, k, v, causal=w.causal, scale=w.softmax_scale(), window=w.window)
+            dt = time.perf_counter() - t0
+            amount += W.flops(w.scaled(mode="dense", batch=1, h_q=1, h_kv=1, s_q=q1 - q0, s_k=q1 - q0)) / 1e12
+            done.append(f"s{bi}h{h}")
+        elif w.mode == "rotary":
             # 64 rows of one batch entry, every head
             i0 = (b // w.batch) * 64 % w.s_q
             x = inp["q"][bi:bi + 1, i0:i0 + 64].double().numpy()
@@ -298,7 +323,8 @@ def cpu_sample(w, inp, budget_s):
             done.append(f"b{bi}")
         t_total += dt
         b += 1
-    unit_desc = {"dense": "(batch, head) pairs", "rotary": "64-row blocks (all heads)"}.get(w.mode, "batch entries")
+    unit_desc = {"dense": "(batch, head) pairs", "rotary": "64-row blocks (all heads)",
+                 "varlen": "(sequence, head) pairs"}.get(w.mode, "batch entries")
     desc = (f"float64 oracle, single thread, on {len(done)} {unit_desc} of the workload "
             f"({', '.join(done[:8])}{'...' if len(done) > 8 else ''}); inputs converted to float64 "
             f"outside the timed region")
@@ -367,7 +393,8 @@ def run_ours(args):
     w = W.CONFIGS[args.config]
     inp = W.make_inputs(w, seed=0)
     inp_dev = {k: v.to(device) for k, v in inp.items()}
-    seqlens = inp["cache_seqlens"].tolist() if w.mode == "kvcache" else None
+    seqlens = (inp["cache_seqlens"].tolist() if w.mode == "kvcache"
+               else (inp["cu_seqlens"].diff().tolist() if w.mode == "varlen" else None))
     amount, unit, bound = work_units(w, seqlens)
     stream = torch.cuda.current_stream(device)
     flush_buf = L2Flush(device)
@@ -473,7 +500,8 @@ def run_reference(args):
         return 0
     w = W.CONFIGS[args.config]
     inp = W.make_inputs(w, seed=0)
-    seqlens = inp["cache_seqlens"].tolist() if w.mode == "kvcache" else None
+    seqlens = (inp["cache_seqlens"].tolist() if w.mode == "kvcache"
+               else (inp["cu_seqlens"].diff().tolist() if w.mode == "varlen" else None))
     _, unit, _ = work_units(w, seqlens)
     # each step is one bounded sample; the whole run stays within a few minutes
     per_step = max(0.2, min(5.0, 60.0 / max(args.steps, 1)))

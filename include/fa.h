@@ -208,6 +208,30 @@ int fa_fwd_window(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
                   const fa_tensor *out, float *lse,
                   void *workspace, size_t workspace_bytes, void *stream);
 
+/* Attention over packed sequences (the IS_VARLEN option of ROCm/flash-
+ * attention PR #99): sequences of different lengths stored back to back.
+ *  - q [total_q, h_q, d_qk], k [total_k, h_kv, d_qk], v [total_k, h_kv, d_v],
+ *    out [total_q, h_q, d_v]: fp16/bf16, head-dim stride 1, other strides and
+ *    base multiples of 16 bytes.  Head dims: the pairs the tcgen05 kernel
+ *    takes (64/64, 128/128, 192/128, 128/64, 64/128, 192/64), else
+ *    FA_ERR_UNSUPPORTED.
+ *  - cu_seqlens_q, cu_seqlens_k: int32 DEVICE arrays [n_seqs + 1] of
+ *    non-decreasing row starts; sequence s owns query rows cu_q[s] ..
+ *    cu_q[s+1]-1 and key rows cu_k[s] .. cu_k[s+1]-1, and is attended as a
+ *    batch of one (bottom-right causal alignment, window as in
+ *    fa_fwd_window, inside the sequence).
+ *  - max_seqlen_q: an upper bound of cu_q[s+1] - cu_q[s] (sizes the grid;
+ *    rows past it are not computed).
+ *  - lse: fp32 DEVICE array [h_q, total_q] (contiguous) or NULL.
+ *  - Device-side precondition: every sequence lies inside the packed rows;
+ *    a sequence that does not is skipped and FA_ERR_DEVICE_PRECONDITION is
+ *    recorded (fa_device_status).
+ * Allocates nothing; asynchronous on `stream`. */
+int fa_fwd_varlen(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
+                  const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t n_seqs,
+                  int32_t max_seqlen_q, int32_t causal, int32_t window_left, int32_t window_right,
+                  float scale, const fa_tensor *out, float *lse, void *stream);
+
 /* Workspace bytes fa_fwd needs for these shapes. */
 int fa_fwd_workspace_size(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
                           size_t *bytes);

@@ -66,6 +66,8 @@ lib.fa_fwd_window.restype = ctypes.c_int
 lib.fa_kvcache_fwd_window.argtypes = [_P, _P, _P, _P, _P, _P, _P, _v, _i32, _i32, _i32, _i32, _i32, _i32,
                                       ctypes.c_float, _P, _v, _v, ctypes.c_size_t, _v]
 lib.fa_kvcache_fwd_window.restype = ctypes.c_int
+lib.fa_fwd_varlen.argtypes = [_P, _P, _P, _v, _v, _i32, _i32, _i32, _i32, _i32, ctypes.c_float, _P, _v, _v]
+lib.fa_fwd_varlen.restype = ctypes.c_int
 lib.fa_fwd_workspace_size.argtypes = [_P, _P, _P, ctypes.POINTER(ctypes.c_size_t)]
 lib.fa_fwd_workspace_size.restype = ctypes.c_int
 lib.fa_device_status.argtypes = [_v, ctypes.POINTER(ctypes.c_int32)]
@@ -252,6 +254,25 @@ def fa_fwd(q, k, v, causal=False, softmax_scale=None, out=None, lse=None, worksp
         ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
         ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None,
         workspace.numel() if workspace is not None else 0, _stream_handle(stream, q.device)))
+    return out, lse
+
+
+def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, causal=False, softmax_scale=None,
+                  window=(-1, -1), out=None, lse=None, return_lse=True, stream=None):
+    """Attention over packed sequences: q [total_q, h_q, d_qk], k/v [total_k,
+    h_kv, d]; cu_seqlens_q/k int32 CUDA tensors [n_seqs + 1] of row starts.
+    Returns (out [total_q, h_q, d_v], lse [h_q, total_q])."""
+    total_q, h_q, _ = q.shape
+    d_v = v.shape[2]
+    if out is None:
+        out = torch.empty((total_q, h_q, d_v), dtype=q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((h_q, total_q), dtype=torch.float32, device=q.device)
+    _check(lib.fa_fwd_varlen(
+        _ref(describe(q)), _ref(describe(k)), _ref(describe(v)), ctypes.c_void_p(cu_seqlens_q.data_ptr()),
+        ctypes.c_void_p(cu_seqlens_k.data_ptr()), int(cu_seqlens_q.numel()) - 1, int(max_seqlen_q),
+        int(bool(causal)), int(window[0]), int(window[1]), float(softmax_scale or 0.0), _ref(describe(out)),
+        ctypes.c_void_p(lse.data_ptr()) if lse is not None else None, _stream_handle(stream, q.device)))
     return out, lse
 
 

@@ -23,7 +23,7 @@ LIB = os.path.join(HERE, "libfa.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "-I", INCLUDE, "-I", CSRC,
-         "--expt-relaxed-constexpr", "-Xptxas", "-warn-spills"]
+         "--expt-relaxed-constexpr", "-Xptxas", "-warn-spills", "-diag-error", "549"]
 
 
 def _sources():

@@ -175,8 +175,13 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int run_tc_attention(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, const fa_tensor *out,
                      float *lse, bool kvcache, const int32_t *seqlens, int32_t seqlen_scalar, int64_t s_new,
                      int64_t cap, int causal, int win_left, int win_right, float scale_log2, int32_t *status,
-                     cudaStream_t st) {
-    const int64_t b = q->shape[0], s_q = q->shape[1], h_q = q->shape[2], d_qk = q->shape[3];
+                     cudaStream_t st, const int32_t *cu_q = nullptr, const int32_t *cu_k = nullptr,
+                     int64_t n_seqs = 0, int64_t max_seqlen_q = 0) {
+    // packed sequences: q/k/v/out are [1, total, h, d] views, the grid runs
+    // over n_seqs sequences of at most max_seqlen_q query rows
+    const bool varlen = cu_q != nullptr;
+    const int64_t b = varlen ? n_seqs : q->shape[0], s_q = varlen ? max_seqlen_q : q->shape[1];
+    const int64_t h_q = q->shape[2], d_qk = q->shape[3];
     const int64_t h_kv = k->shape[2], d_v = v->shape[3];
     const int64_t g = h_q / h_kv;
     const int pack = (128 % g == 0) ? (int)g : 1;
@@ -200,6 +205,10 @@ int run_tc_attention(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
     p.causal = causal ? 1 : 0;
     p.win_left = win_left;
     p.win_right = win_right;
+    p.cu_q = cu_q;
+    p.cu_k = cu_k;
+    p.total_q = varlen ? q->shape[1] : 0;
+    p.total_k = varlen ? k->shape[1] : 0;
     p.n_q_tiles = (int)((s_q * pack + 127) / 128);
     p.scale_log2 = scale_log2;
     // Two query tiles per CTA keep the tensor core busy during the softmax,
@@ -758,6 +767,56 @@ int fa_fwd_window(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, in
     cudaError_t e = launch_simt_attn(p, q->dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
     return FA_OK;
+}
+
+int fa_fwd_varlen(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, const int32_t *cu_seqlens_q,
+                  const int32_t *cu_seqlens_k, int32_t n_seqs, int32_t max_seqlen_q, int32_t causal,
+                  int32_t window_left, int32_t window_right, float scale, const fa_tensor *out, float *lse,
+                  void *stream) {
+    g_last_error[0] = 0;
+    if (window_left < -1 || window_right < -1)
+        return fail(FA_ERR_INVALID_ARG, "window bounds must be >= -1 (-1 = unbounded)");
+    Dims4 qd, kd, vd, od;
+    int rc;
+    if ((rc = check_tensor(q, "q", 3, 0, &qd))) return rc;
+    if ((rc = check_tensor(k, "k", 3, q->dtype, &kd))) return rc;
+    if ((rc = check_tensor(v, "v", 3, q->dtype, &vd))) return rc;
+    if ((rc = check_tensor(out, "out", 3, q->dtype, &od))) return rc;
+    const int64_t total_q = qd.n[0], h_q = qd.n[1], d_qk = qd.n[2];
+    const int64_t total_k = kd.n[0], h_kv = kd.n[1], d_v = vd.n[2];
+    if (kd.n[2] != d_qk) return fail(FA_ERR_INVALID_ARG, "k head dim differs from q");
+    if (vd.n[0] != total_k || vd.n[1] != h_kv) return fail(FA_ERR_INVALID_ARG, "v shape differs from k");
+    if (h_kv <= 0 || h_q % h_kv) return fail(FA_ERR_INVALID_ARG, "h_q must be a multiple of h_kv");
+    if (od.n[0] != total_q || od.n[1] != h_q || od.n[2] != d_v)
+        return fail(FA_ERR_INVALID_ARG, "out shape must be [total_q, h_q, d_v]");
+    if (!cu_seqlens_q || !cu_seqlens_k || n_seqs < 0 || max_seqlen_q < 0)
+        return fail(FA_ERR_INVALID_ARG, "cu_seqlens_q/k, n_seqs >= 0 and max_seqlen_q >= 0 are required");
+    if (!prefill_supported((int)d_qk, (int)d_v))
+        return fail(FA_ERR_UNSUPPORTED, "packed sequences need head dims the tcgen05 kernel takes "
+                    "(d_qk/d_v in 64/64, 128/128, 192/128, 128/64, 64/128, 192/64)");
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) return fail(FA_ERR_LAYOUT, "lse not 4-byte aligned");
+    if (n_seqs == 0 || max_seqlen_q == 0 || total_q == 0 || h_q == 0) return FA_OK;
+    int32_t *status = status_word();
+    if (!status) return fail(FA_ERR_CUDA, "no CUDA device");
+    // [total, h, d] as a batch of one [1, total, h, d]
+    auto as4 = [](const fa_tensor *t) {
+        fa_tensor r = *t;
+        r.ndim = 4;
+        r.shape[3] = t->shape[2];
+        r.shape[2] = t->shape[1];
+        r.shape[1] = t->shape[0];
+        r.shape[0] = 1;
+        r.stride[3] = 1;
+        r.stride[2] = t->stride[1];
+        r.stride[1] = t->stride[0];
+        r.stride[0] = t->stride[0] * t->shape[0];
+        return r;
+    };
+    const fa_tensor q4 = as4(q), k4 = as4(k), v4 = as4(v), o4 = as4(out);
+    const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)d_qk);
+    return run_tc_attention(&q4, &k4, &v4, &o4, lse, false, nullptr, 0, 0, 0, causal, window_left, window_right,
+                            sc * 1.4426950408889634f, status, static_cast<cudaStream_t>(stream), cu_seqlens_q,
+                            cu_seqlens_k, n_seqs, max_seqlen_q);
 }
 
 int fa_device_status(void *stream, int32_t *status) {

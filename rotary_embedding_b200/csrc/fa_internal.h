@@ -120,6 +120,11 @@ struct PrefillParams {
     int kvcache, b, s_q, h_q, h_kv, g, pack, causal, n_q_tiles;
     int tiles_per_cta;  // 1: one 128-row tile per CTA; 2: two tiles, two softmax warpgroups
     int win_left, win_right;  // sliding window; -1 = unbounded
+    // packed sequences (varlen): grid z = sequence s with query rows
+    // cu_q[s] .. cu_q[s+1]-1 and key rows cu_k[s] .. of batch entry 0;
+    // lse is [h_q, total_q].  nullptr: batched.
+    const int32_t *cu_q, *cu_k;
+    int64_t total_q, total_k;
     float scale_log2;
 };
 

@@ -90,10 +90,24 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
     const int hq0 = hgrp * pack;                           // first query head of the tile
     const int hk = hq0 / p.g;
     const int i0 = qt * (kBM / pack);                      // first query position
-    const int i_last = min(p.s_q, i0 + kBM / pack) - 1;
 
-    int N;
-    if (p.kvcache) {
+    // keys N, query rows sq of this CTA's sequence, and the row offsets of a
+    // packed (varlen) sequence: blockIdx.z is then the sequence, whose rows
+    // qoff .. and koff .. sit in batch entry 0 of the packed tensors
+    int N, sq = p.s_q, qoff = 0, koff = 0, tb = b;
+    if (p.cu_q) {
+        qoff = __ldg(p.cu_q + b);
+        sq = __ldg(p.cu_q + b + 1) - qoff;
+        koff = __ldg(p.cu_k + b);
+        N = __ldg(p.cu_k + b + 1) - koff;
+        tb = 0;
+        // device-side preconditions: the sequence lies inside the packed rows
+        if (qoff < 0 || sq < 0 || (int64_t)qoff + sq > p.total_q || koff < 0 || N < 0 ||
+            (int64_t)koff + N > p.total_k) {
+            if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
+            return;
+        }
+    } else if (p.kvcache) {
         const int L = seqlen_of(p.seqlens, p.seqlen_scalar, b);
         if (L < 0 || (int64_t)L + p.s_new > p.cap) {
             if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
@@ -103,10 +117,12 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
     } else {
         N = (int)p.s_k;
     }
+    if (i0 >= sq) return;                                  // past this sequence's rows
+    const int i_last = min(sq, i0 + kBM / pack) - 1;
     // visible keys of the tile's first and last query rows (causal, window)
     int64_t f_first, l_first, f_last, l_last;
-    visible_keys(i0, N, p.s_q, p.causal, p.win_left, p.win_right, f_first, l_first);
-    visible_keys(i_last, N, p.s_q, p.causal, p.win_left, p.win_right, f_last, l_last);
+    visible_keys(i0, N, sq, p.causal, p.win_left, p.win_right, f_first, l_first);
+    visible_keys(i_last, N, sq, p.causal, p.win_left, p.win_right, f_last, l_last);
     const int kv_end = (int)max((int64_t)0, min((int64_t)N, l_last + 1));
     const int n_kv = (kv_end + kBN - 1) / kBN;
     const int kb = min((int)(f_first / kBN), n_kv);        // first key tile any row sees
@@ -150,7 +166,7 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
             tma_prefetch_desc(&tmV);
             mbar_arrive_expect_tx(q_full, C::QBYTES);
 #pragma unroll
-            for (int c = 0; c < D_QK / 64; ++c) tma_load_4d(sQ + c * C::QBOX, &tmQ, q_full, c * 64, hq0, i0, b);
+            for (int c = 0; c < D_QK / 64; ++c) tma_load_4d(sQ + c * C::QBOX, &tmQ, q_full, c * 64, hq0, qoff + i0, tb);
             for (int t = 0; t < nblk; ++t) {
                 const int j = kb + t;
                 const int st = t % C::KST;
@@ -158,11 +174,11 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
                 mbar_arrive_expect_tx(&k_full[st], C::KBYTES);
 #pragma unroll
                 for (int c = 0; c < D_QK / 64; ++c)
-                    tma_load_4d(sK + st * C::KBYTES + c * C::KBOX, &tmK, &k_full[st], c * 64, hk, j * kBN, b);
+                    tma_load_4d(sK + st * C::KBYTES + c * C::KBOX, &tmK, &k_full[st], c * 64, hk, koff + j * kBN, tb);
                 mbar_arrive_expect_tx(&v_full[st], C::VBYTES);
 #pragma unroll
                 for (int c = 0; c < D_V / 64; ++c)
-                    tma_load_4d(sV + st * C::VBYTES + c * C::VBOX, &tmV, &v_full[st], c * 64, hk, j * kBN, b);
+                    tma_load_4d(sV + st * C::VBYTES + c * C::VBOX, &tmV, &v_full[st], c * 64, hk, koff + j * kBN, tb);
             }
         }
     } else if (warp == 1) {
@@ -215,9 +231,9 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
         const int prow = qt * kBM + r;                 // packed row
         const int i = prow / pack;                     // query position
         const int hq = hq0 + (prow % pack);
-        const bool row_valid = i < p.s_q;
+        const bool row_valid = i < sq;
         int64_t fv64, lv64;
-        visible_keys(i, N, p.s_q, p.causal, p.win_left, p.win_right, fv64, lv64);
+        visible_keys(i, N, sq, p.causal, p.win_left, p.win_right, fv64, lv64);
         const int last_vis = row_valid ? (int)lv64 : -1;
         const int first_vis = (int)fv64;
         const float c = p.scale_log2;
@@ -334,7 +350,7 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
         tc::fence_after_sync();
         // every lane takes part in the (warp-collective) TMEM loads; only rows
         // inside the sequence are stored
-        T *orow = static_cast<T *>(p.out) + b * p.os.b + (int64_t)i * p.os.s + hq * p.os.h;
+        T *orow = static_cast<T *>(p.out) + tb * p.os.b + (int64_t)(qoff + i) * p.os.s + hq * p.os.h;
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
         for (int h = 0; h < D_V / 32; ++h) {
@@ -357,7 +373,7 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
             }
         }
         if (row_valid && p.lse)
-            p.lse[((int64_t)b * p.h_q + hq) * p.s_q + i] = l > 0.f ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
+            p.lse[p.cu_q ? (int64_t)hq * p.total_q + qoff + i : ((int64_t)b * p.h_q + hq) * sq + i] = l > 0.f ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -445,8 +461,23 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
     const int hk = hq0 / p.g;
     const int rows_per_tile = kBM / pack;                   // query positions per tile
 
-    int N;
-    if (p.kvcache) {
+    // keys N, query rows sq of this CTA's sequence, and the row offsets of a
+    // packed (varlen) sequence: blockIdx.z is then the sequence, whose rows
+    // qoff .. and koff .. sit in batch entry 0 of the packed tensors
+    int N, sq = p.s_q, qoff = 0, koff = 0, tb = b;
+    if (p.cu_q) {
+        qoff = __ldg(p.cu_q + b);
+        sq = __ldg(p.cu_q + b + 1) - qoff;
+        koff = __ldg(p.cu_k + b);
+        N = __ldg(p.cu_k + b + 1) - koff;
+        tb = 0;
+        // device-side preconditions: the sequence lies inside the packed rows
+        if (qoff < 0 || sq < 0 || (int64_t)qoff + sq > p.total_q || koff < 0 || N < 0 ||
+            (int64_t)koff + N > p.total_k) {
+            if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
+            return;
+        }
+    } else if (p.kvcache) {
         const int L = seqlen_of(p.seqlens, p.seqlen_scalar, b);
         if (L < 0 || (int64_t)L + p.s_new > p.cap) {
             if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
@@ -456,17 +487,18 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
     } else {
         N = (int)p.s_k;
     }
+    if (2 * blk * rows_per_tile >= sq) return;             // past this sequence's rows
     // per tile: key tiles kb[x] .. n_kv[x] - 1 (causal, window), and the
     // bounds past which a key tile needs an element mask (see prefill_kernel)
     int i0[2], n_kv[2], kb[2], mask_from[2], lo_max[2];
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
         i0[x] = (2 * blk + x) * rows_per_tile;
-        const int i_last = min(p.s_q, i0[x] + rows_per_tile) - 1;
+        const int i_last = min(sq, i0[x] + rows_per_tile) - 1;
         int64_t f_first, l_first, f_last, l_last;
-        visible_keys(i0[x], N, p.s_q, p.causal, p.win_left, p.win_right, f_first, l_first);
-        visible_keys(i_last, N, p.s_q, p.causal, p.win_left, p.win_right, f_last, l_last);
-        const int kv_end = i0[x] >= p.s_q ? 0 : (int)max((int64_t)0, min((int64_t)N, l_last + 1));
+        visible_keys(i0[x], N, sq, p.causal, p.win_left, p.win_right, f_first, l_first);
+        visible_keys(i_last, N, sq, p.causal, p.win_left, p.win_right, f_last, l_last);
+        const int kv_end = i0[x] >= sq ? 0 : (int)max((int64_t)0, min((int64_t)N, l_last + 1));
         n_kv[x] = (kv_end + BN - 1) / BN;
         kb[x] = min((int)(f_first / BN), n_kv[x]);
         mask_from[x] = (int)max((int64_t)0, min((int64_t)N, l_first + 1));
@@ -516,7 +548,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             for (int x = 0; x < 2; ++x)
 #pragma unroll
                 for (int c = 0; c < D_QK / 64; ++c)
-                    tma_load_4d(sQ + x * C::QBYTES + c * C::QBOX, &tmQ, q_full, c * 64, hq0, i0[x], b);
+                    tma_load_4d(sQ + x * C::QBYTES + c * C::QBOX, &tmQ, q_full, c * 64, hq0, qoff + i0[x], tb);
             for (int j = kb0; j < n_all; ++j) {
                 const int u = j - kb0;   // loaded tile index (stages, parities)
                 const int ks = u % KST, vs = u % VST;
@@ -524,12 +556,12 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                 mbar_arrive_expect_tx(&k_full[ks], C::KBYTES);
 #pragma unroll
                 for (int c = 0; c < D_QK / 64; ++c)
-                    tma_load_4d(sK + ks * C::KBYTES + c * C::KBOX, &tmK, &k_full[ks], c * 64, hk, j * BN, b);
+                    tma_load_4d(sK + ks * C::KBYTES + c * C::KBOX, &tmK, &k_full[ks], c * 64, hk, koff + j * BN, tb);
                 if (u >= VST && !mbar_wait(&v_empty[vs], ((u / VST) - 1) & 1, p.status)) break;
                 mbar_arrive_expect_tx(&v_full[vs], C::VBYTES);
 #pragma unroll
                 for (int c = 0; c < D_V / 64; ++c)
-                    tma_load_4d(sV + vs * C::VBYTES + c * C::KBOX, &tmV, &v_full[vs], c * 64, hk, j * BN, b);
+                    tma_load_4d(sV + vs * C::VBYTES + c * C::KBOX, &tmV, &v_full[vs], c * 64, hk, koff + j * BN, tb);
             }
         }
     } else if (warp == 1) {
@@ -619,9 +651,9 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         const int prow = (2 * blk + x) * kBM + r;      // packed row
         const int i = prow / pack;
         const int hq = hq0 + (prow % pack);
-        const bool row_valid = i < p.s_q;
+        const bool row_valid = i < sq;
         int64_t fv64, lv64;
-        visible_keys(i, N, p.s_q, p.causal, p.win_left, p.win_right, fv64, lv64);
+        visible_keys(i, N, sq, p.causal, p.win_left, p.win_right, fv64, lv64);
         const int last_vis = row_valid ? (int)lv64 : -1;
         const int first_vis = (int)fv64;
         const float c = p.scale_log2;
@@ -758,7 +790,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         // ------------------------------------------------ epilogue
         if (ok && nk > jb && !mbar_wait(&o_full[x], 0, p.status)) ok = false;
         tc::fence_after_sync();
-        T *orow = static_cast<T *>(p.out) + b * p.os.b + (int64_t)i * p.os.s + hq * p.os.h;
+        T *orow = static_cast<T *>(p.out) + tb * p.os.b + (int64_t)(qoff + i) * p.os.s + hq * p.os.h;
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
         for (int h = 0; h < D_V / 32; ++h) {
@@ -781,7 +813,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             }
         }
         if (row_valid && p.lse)
-            p.lse[((int64_t)b * p.h_q + hq) * p.s_q + i] = l > 0.f ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
+            p.lse[p.cu_q ? (int64_t)hq * p.total_q + qoff + i : ((int64_t)b * p.h_q + hq) * sq + i] = l > 0.f ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
     }
     tc::fence_before_sync();
     __syncthreads();

@@ -31,7 +31,8 @@ _DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    mode: str                 # "kvcache" (fa_kvcache_fwd), "dense" (fa_fwd) or "rotary" (fa_rotary)
+    mode: str                 # "kvcache" (fa_kvcache_fwd), "dense" (fa_fwd), "rotary" (fa_rotary)
+                              # or "varlen" (fa_fwd_varlen: batch packed sequences, lengths ~ U{seqlens})
     dtype: str                # "fp16" | "bf16"
     batch: int
     h_q: int
@@ -104,8 +105,14 @@ WINDOW_PREFILL = Workload(
     name="window-prefill bf16 b2 h16 s8192 d128 causal window(1024,0)", mode="dense", dtype="bf16",
     batch=2, h_q=16, h_kv=16, d_qk=128, d_v=128, s_q=8192, s_k=8192, causal=True, window=(1024, 0))
 
+# Packed prefill of sequences of mixed lengths ([P2] IS_VARLEN).
+VARLEN_PREFILL = Workload(
+    name="varlen-prefill bf16 8 seqs len~U{256..4096} h16 d128 causal", mode="varlen", dtype="bf16",
+    batch=8, h_q=16, h_kv=16, d_qk=128, d_v=128, s_q=4096, seqlens=(256, 4096), causal=True)
+
 CONFIGS = {
     "rotary-q": ROTARY_Q,
+    "varlen-prefill": VARLEN_PREFILL,
     "window-prefill": WINDOW_PREFILL,
     "issue-repro": ISSUE_REPRO,
     "gqa-decode": GQA_DECODE,
@@ -145,6 +152,16 @@ def make_inputs(w: Workload, seed: int = 0) -> dict:
         offs = torch.randint(lo, hi + 1, (w.batch,), generator=g, dtype=torch.int32)
         cos, sin = rotary_tables(w.cap, w.rotary_dim, w.rotary_base, dt)
         return {"q": q, "cache_seqlens": offs, "cos": cos, "sin": sin}
+    if w.mode == "varlen":
+        lo, hi = w.seqlens
+        lens = torch.randint(lo, hi + 1, (w.batch,), generator=g, dtype=torch.int32)
+        total = int(lens.sum())
+        q = _draw(g, (total, w.h_q, w.d_qk), w.dist, dt)
+        k = _draw(g, (total, w.h_kv, w.d_qk), w.dist, dt)
+        v = _draw(g, (total, w.h_kv, w.d_v), w.dist, dt)
+        cu = torch.zeros(w.batch + 1, dtype=torch.int32)
+        cu[1:] = torch.cumsum(lens, 0)
+        return {"q": q, "k": k, "v": v, "cu_seqlens": cu}
     if w.mode == "dense":
         q = _draw(g, (w.batch, w.s_q, w.h_q, w.d_qk), w.dist, dt)
         k = _draw(g, (w.batch, w.s_k, w.h_kv, w.d_qk), w.dist, dt)
@@ -196,6 +213,10 @@ def kvcache_bytes(w: Workload, seqlens) -> int:
 def visible_pairs(w: Workload, seqlens=None) -> int:
     """Number of visible (query row, key) pairs summed over batch and query heads."""
     total = 0
+    if w.mode == "varlen":
+        # seqlens: the drawn lengths; each sequence is a batch of one with s_q = s_k
+        return sum(visible_pairs(w.scaled(mode="dense", batch=1, s_q=int(n), s_k=int(n)))
+                   for n in seqlens) if seqlens is not None else 0
     if w.mode == "dense":
         lens = [w.s_k] * w.batch
         s_q = w.s_q
