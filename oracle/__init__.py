@@ -58,6 +58,8 @@ def _bind(lib):
     lib.oracle_kvcache_fwd.restype = i32
     lib.oracle_fwd.argtypes = [i64, i64, i64, i64, i64, i32, i32, P, P, P, i32, d, P, P, i64, i64]
     lib.oracle_fwd.restype = i32
+    lib.oracle_bwd.argtypes = [i64, i64, i64, i64, i64, i32, i32, P, P, P, P, i32, d, i64, i64, P, P, P]
+    lib.oracle_bwd.restype = i32
     return lib
 
 
@@ -240,3 +242,24 @@ def fwd(q, k, v, causal=False, scale=None, lib=None, window=(-1, -1)):
     if rc != 0:
         raise ValueError(f"oracle_fwd rejected its arguments (code {rc})")
     return out, lse
+
+
+def bwd(q, k, v, dout, causal=False, scale=None, lib=None, window=(-1, -1)):
+    """Gradients of cache-less attention in float64 ([P4] d_qk != d_v
+    backward): the gradient of sum(dout * fwd(q, k, v)) with respect to q, k
+    and v, for the same mask, scale and GQA mapping.  Returns (dq, dk, dv)
+    shaped like q, k, v."""
+    lib = lib or load()
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    b, s_q, h_q, d_qk = q.shape
+    s_k, h_kv = k.shape[1], k.shape[2]
+    d_v = v.shape[3]
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(d_qk)
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    rc = lib.oracle_bwd(b, s_q, s_k, h_q, h_kv, d_qk, d_v, _ptr(q), _ptr(k), _ptr(v), _ptr(dout),
+                        int(bool(causal)), float(scale), int(window[0]), int(window[1]),
+                        _ptr(dq), _ptr(dk), _ptr(dv))
+    if rc != 0:
+        raise ValueError(f"oracle_bwd rejected its arguments (code {rc})")
+    return dq, dk, dv

@@ -176,6 +176,38 @@ int oracle_rotary(const double *x, double *y, int64_t rows, int d, const int64_t
 }
 
 /* ------------------------------------------------------------------ */
+/* Keys lo .. hi visible to query row i of s_q over N keys (hi < lo:   */
+/* none).  The rows are aligned bottom-right at a = i + N - s_q: with  */
+/* causal, hi = a; with a window ("optimizing-attention-flash",        */
+/* window_size=(left, right), -1 = unbounded), lo = a - left and hi is */
+/* at most a + right.                                                  */
+/* ------------------------------------------------------------------ */
+static void visible_range(int64_t i, int64_t N, int64_t s_q, int causal,
+                          int64_t win_left, int64_t win_right, int64_t *lo_out, int64_t *hi_out)
+{
+    int64_t a = i + N - s_q;
+    int64_t hi = N - 1, lo = 0;
+    if (causal) {
+        int64_t last = a;                    /* last visible key index */
+#if ORACLE_PLANT == 4            /* planted: top-left instead of bottom-right alignment */
+        last = i;
+#elif ORACLE_PLANT == 5          /* planted: diagonal excluded */
+        last = a - 1;
+#endif
+        hi = last;
+    }
+    if (win_right >= 0 && a + win_right < hi) hi = a + win_right;
+    if (win_left >= 0) lo = a - win_left;
+#if ORACLE_PLANT == 12           /* planted: left window one key short */
+    if (win_left >= 0) lo = a - win_left + 1;
+#endif
+    if (lo < 0) lo = 0;
+    if (hi > N - 1) hi = N - 1;
+    *lo_out = lo;
+    *hi_out = hi;
+}
+
+/* ------------------------------------------------------------------ */
 /* Exact masked softmax attention for one (batch, query head) pair     */
 /* ([P5] Workflow 1 Step 2; causal flag of Workflow 2 Step 2).         */
 /*   q_rows  [s_q, d_qk] with row stride q_ld                          */
@@ -192,28 +224,8 @@ static void attend_one_head(const double *q_rows, int64_t q_ld,
                             double *out, int64_t o_ld, double *lse, double *scores)
 {
     for (int64_t i = 0; i < s_q; ++i) {
-        /* keys visible to query i (aligned bottom-right at a = i + N - s_q):
-         * lo <= j <= hi with hi = a when causal, a + win_right when that
-         * bound is given, and lo = a - win_left when that bound is given
-         * ("optimizing-attention-flash", window_size=(left, right), -1 = none) */
-        int64_t a = i + N - s_q;
-        int64_t hi = N - 1, lo = 0;
-        if (causal) {
-            int64_t last = a;                    /* last visible key index */
-#if ORACLE_PLANT == 4            /* planted: top-left instead of bottom-right alignment */
-            last = i;
-#elif ORACLE_PLANT == 5          /* planted: diagonal excluded */
-            last = a - 1;
-#endif
-            hi = last;
-        }
-        if (win_right >= 0 && a + win_right < hi) hi = a + win_right;
-        if (win_left >= 0) lo = a - win_left;
-#if ORACLE_PLANT == 12           /* planted: left window one key short */
-        if (win_left >= 0) lo = a - win_left + 1;
-#endif
-        if (lo < 0) lo = 0;
-        if (hi > N - 1) hi = N - 1;
+        int64_t lo, hi;
+        visible_range(i, N, s_q, causal, win_left, win_right, &lo, &hi);
         double *o = out + i * o_ld;
         if (hi < lo) {
             for (int t = 0; t < d_v; ++t) o[t] = 0.0;
@@ -373,5 +385,101 @@ int oracle_fwd(int64_t b, int64_t s_q, int64_t s_k, int64_t h_q, int64_t h_kv,
                             lse + (bi * h_q + h) * s_q, scores);
         }
     free(scores);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Backward of cache-less attention ([P4] "Support hdimQK != hdimV     */
+/* backward": the gradients of q, k and v when d_qk != d_v).  The     */
+/* pages give no formula; this is the gradient of the forward's        */
+/* definition, out_i = sum_j P_ij v_j with P_i = softmax_j(scale q_i.k_j) */
+/* over the visible keys, for an upstream gradient dout:               */
+/*   dv_j  += P_ij dout_i                                              */
+/*   dP_ij  = dout_i . v_j                                             */
+/*   dS_ij  = P_ij (dP_ij - sum_t P_it dP_it)   (softmax Jacobian)     */
+/*   dq_i   = scale sum_j dS_ij k_j                                    */
+/*   dk_j  += scale dS_ij q_i                                          */
+/* with P recomputed exactly (two-pass softmax) from q and k.  A kv    */
+/* head's dk and dv sum over the query heads that read it (GQA).       */
+/* Layouts (contiguous): q, dq [b, s_q, h_q, d_qk]; k, dk              */
+/* [b, s_k, h_kv, d_qk]; v, dv [b, s_k, h_kv, d_v]; dout               */
+/* [b, s_q, h_q, d_v].  Returns 0, or a negative value for arguments   */
+/* the definition cannot evaluate.                                     */
+/* ------------------------------------------------------------------ */
+int oracle_bwd(int64_t b, int64_t s_q, int64_t s_k, int64_t h_q, int64_t h_kv,
+               int d_qk, int d_v, const double *q, const double *k, const double *v,
+               const double *dout, int causal, double scale, int64_t win_left, int64_t win_right,
+               double *dq, double *dk, double *dv)
+{
+    if (h_kv <= 0 || h_q % h_kv != 0) return -1;
+    int64_t group = h_q / h_kv;
+    double *P = (double *)malloc(sizeof(double) * (size_t)(s_k + 1));
+    double *dP = (double *)malloc(sizeof(double) * (size_t)(s_k + 1));
+    if (!P || !dP) {
+        free(P);
+        free(dP);
+        return -4;
+    }
+    memset(dq, 0, sizeof(double) * (size_t)(b * s_q * h_q * d_qk));
+    memset(dk, 0, sizeof(double) * (size_t)(b * s_k * h_kv * d_qk));
+    memset(dv, 0, sizeof(double) * (size_t)(b * s_k * h_kv * d_v));
+    for (int64_t bi = 0; bi < b; ++bi)
+        for (int64_t h = 0; h < h_q; ++h) {
+            int64_t hk = h / group;
+#if ORACLE_PLANT == 15           /* planted: only the group's last query head reaches dk, dv */
+            if (h % group != group - 1) continue;
+#endif
+            for (int64_t i = 0; i < s_q; ++i) {
+                int64_t lo, hi;
+                visible_range(i, s_k, s_q, causal, win_left, win_right, &lo, &hi);
+                if (hi < lo) continue;            /* no visible key: out is 0, no gradient */
+                const double *qi = q + ((bi * s_q + i) * h_q + h) * d_qk;
+                const double *doi = dout + ((bi * s_q + i) * h_q + h) * d_v;
+                double *dqi = dq + ((bi * s_q + i) * h_q + h) * d_qk;
+                /* P_i: exact softmax over the visible keys */
+                double m = -INFINITY;
+                for (int64_t j = lo; j <= hi; ++j) {
+                    const double *kj = k + ((bi * s_k + j) * h_kv + hk) * d_qk;
+                    double dot = 0.0;
+                    for (int t = 0; t < d_qk; ++t) dot += qi[t] * kj[t];
+                    P[j - lo] = scale * dot;
+                    if (P[j - lo] > m) m = P[j - lo];
+                }
+                double l = 0.0;
+                for (int64_t j = lo; j <= hi; ++j) {
+                    P[j - lo] = exp(P[j - lo] - m);
+                    l += P[j - lo];
+                }
+                for (int64_t j = lo; j <= hi; ++j) P[j - lo] /= l;
+                /* dP_ij = dout_i . v_j and the Jacobian's row term */
+                double rowterm = 0.0;
+                for (int64_t j = lo; j <= hi; ++j) {
+                    const double *vj = v + ((bi * s_k + j) * h_kv + hk) * d_v;
+                    double dot = 0.0;
+                    for (int t = 0; t < d_v; ++t) dot += doi[t] * vj[t];
+                    dP[j - lo] = dot;
+                    rowterm += P[j - lo] * dot;
+                }
+#if ORACLE_PLANT == 13           /* planted: the Jacobian's row term dropped */
+                rowterm = 0.0;
+#endif
+                for (int64_t j = lo; j <= hi; ++j) {
+                    const double *kj = k + ((bi * s_k + j) * h_kv + hk) * d_qk;
+                    double *dkj = dk + ((bi * s_k + j) * h_kv + hk) * d_qk;
+                    double *dvj = dv + ((bi * s_k + j) * h_kv + hk) * d_v;
+                    double pij = P[j - lo];
+                    double ds = pij * (dP[j - lo] - rowterm);
+                    for (int t = 0; t < d_v; ++t) dvj[t] += pij * doi[t];
+                    for (int t = 0; t < d_qk; ++t) dqi[t] += scale * ds * kj[t];
+#if ORACLE_PLANT == 14           /* planted: scale missing from dk */
+                    for (int t = 0; t < d_qk; ++t) dkj[t] += ds * qi[t];
+#else
+                    for (int t = 0; t < d_qk; ++t) dkj[t] += scale * ds * qi[t];
+#endif
+                }
+            }
+        }
+    free(P);
+    free(dP);
     return 0;
 }

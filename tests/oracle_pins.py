@@ -560,4 +560,111 @@ def pin_varlen_sequences_are_independent(lib):
     assert np.array_equal(one, ref[0]) and np.array_equal(l1, rl[0])
 
 
+def _loss_grad_fd(q, k, v, dout, causal, window, lib, eps=1e-5):
+    """Central finite differences of sum(dout * fwd(q, k, v)) in float64."""
+    def loss(qq, kk, vv):
+        out, _ = oracle.fwd(qq, kk, vv, causal=causal, window=window, lib=lib)
+        return float((out * dout).sum())
+    grads = []
+    for which in range(3):
+        args = [q.copy(), k.copy(), v.copy()]
+        g = np.zeros_like(args[which])
+        for idx in np.ndindex(*g.shape):
+            a = [x.copy() for x in args]
+            a[which][idx] += eps
+            up = loss(*a)
+            a[which][idx] -= 2 * eps
+            g[idx] = (up - loss(*a)) / (2 * eps)
+        grads.append(g)
+    return grads
+
+
+def pin_bwd_matches_finite_differences(lib):
+    """The backward ("Support hdimQK != hdimV backward") is the gradient of
+    the pinned forward: central differences of sum(dout * out) agree with
+    dq, dk, dv for d_qk != d_v, GQA, causal (with rows that see no key),
+    and a two-sided window."""
+    rng = np.random.default_rng(61)
+    for (s_q, s_k, h_q, h_kv, d_qk, d_v, causal, window) in (
+            (3, 5, 2, 1, 4, 3, True, (-1, -1)),
+            (4, 2, 2, 2, 3, 2, True, (-1, -1)),      # s_q > s_k: rows 0, 1 see no key
+            (4, 4, 3, 1, 3, 4, False, (1, 1))):
+        q = rng.standard_normal((1, s_q, h_q, d_qk))
+        k = rng.standard_normal((1, s_k, h_kv, d_qk))
+        v = rng.standard_normal((1, s_k, h_kv, d_v))
+        dout = rng.standard_normal((1, s_q, h_q, d_v))
+        got = oracle.bwd(q, k, v, dout, causal=causal, window=window, lib=lib)
+        fd = _loss_grad_fd(q, k, v, dout, causal, window, lib)
+        for name, a, e in zip(("dq", "dk", "dv"), got, fd):
+            assert np.abs(a - e).max() <= 1e-7 * max(1.0, np.abs(e).max()), name
+
+
+def pin_bwd_key_and_value_sums(lib):
+    """Softmax rows sum to one, so each row of dS sums to zero: the keys'
+    gradients sum to zero, and the values' gradients sum to the upstream
+    gradient of every row that sees a key, over the group's query heads."""
+    rng = np.random.default_rng(62)
+    b, s_q, s_k, h_q, h_kv = 2, 6, 9, 4, 2
+    q = rng.standard_normal((b, s_q, h_q, 8))
+    k = rng.standard_normal((b, s_k, h_kv, 8))
+    v = rng.standard_normal((b, s_k, h_kv, 5))
+    dout = rng.standard_normal((b, s_q, h_q, 5))
+    _, dk, dv = oracle.bwd(q, k, v, dout, causal=True, lib=lib)
+    assert np.abs(dk.sum(axis=1)).max() <= 1e-12
+    g = h_q // h_kv
+    want = dout.reshape(b, s_q, h_kv, g, 5).sum(axis=(1, 3))
+    assert np.abs(dv.sum(axis=1) - want).max() <= 1e-12
+
+
+def pin_bwd_single_key(lib):
+    """One key: P = 1 whatever the scores, so dq = dk = 0 and dv is the sum
+    of the upstream gradients."""
+    rng = np.random.default_rng(63)
+    q = rng.standard_normal((1, 3, 2, 4))
+    k = rng.standard_normal((1, 1, 1, 4))
+    v = rng.standard_normal((1, 1, 1, 2))
+    dout = rng.standard_normal((1, 3, 2, 2))
+    dq, dk, dv = oracle.bwd(q, k, v, dout, causal=False, lib=lib)
+    assert np.abs(dq).max() == 0.0 and np.abs(dk).max() == 0.0
+    assert np.allclose(dv[0, 0, 0], dout.sum(axis=(0, 1, 2)), rtol=0, atol=1e-14)
+
+
+def pin_bwd_zero_window_and_unseen_keys(lib):
+    """A (0, 0) window gives each query exactly its aligned key (P = 1): dq =
+    dk = 0 and dv_j = dout_j.  Keys no query sees (causal with a short left
+    window) get no gradient at all."""
+    rng = np.random.default_rng(64)
+    q = rng.standard_normal((1, 5, 1, 4))
+    k = rng.standard_normal((1, 5, 1, 4))
+    v = rng.standard_normal((1, 5, 1, 3))
+    dout = rng.standard_normal((1, 5, 1, 3))
+    dq, dk, dv = oracle.bwd(q, k, v, dout, causal=False, window=(0, 0), lib=lib)
+    assert np.abs(dq).max() == 0.0 and np.abs(dk).max() == 0.0
+    assert np.array_equal(dv, dout)
+    k2 = rng.standard_normal((1, 12, 1, 4))
+    v2 = rng.standard_normal((1, 12, 1, 3))
+    dq, dk, dv = oracle.bwd(q, k2, v2, dout, causal=True, window=(2, -1), lib=lib)
+    # query i sits at key 7 + i and sees keys 5 + i .. 7 + i: keys 0 .. 4 unseen
+    assert np.abs(dk[:, :5]).max() == 0.0 and np.abs(dv[:, :5]).max() == 0.0
+    assert np.abs(dk[:, 5:]).max() > 0.0 and np.abs(dv[:, 5:]).max() > 0.0
+
+
+def pin_bwd_gqa_equals_repeated_heads(lib):
+    """GQA backward: a kv head's gradient is the sum of the gradients of its
+    query heads' copies when every query head gets its own copy of k and v."""
+    rng = np.random.default_rng(65)
+    b, s_q, s_k, h_q, h_kv, d_qk, d_v = 1, 4, 7, 6, 2, 5, 3
+    g = h_q // h_kv
+    q = rng.standard_normal((b, s_q, h_q, d_qk))
+    k = rng.standard_normal((b, s_k, h_kv, d_qk))
+    v = rng.standard_normal((b, s_k, h_kv, d_v))
+    dout = rng.standard_normal((b, s_q, h_q, d_v))
+    dq, dk, dv = oracle.bwd(q, k, v, dout, causal=True, lib=lib)
+    kr, vr = np.repeat(k, g, axis=2), np.repeat(v, g, axis=2)
+    dq_r, dk_r, dv_r = oracle.bwd(q, kr, vr, dout, causal=True, lib=lib)
+    assert np.abs(dq - dq_r).max() <= 1e-13
+    assert np.abs(dk - dk_r.reshape(b, s_k, h_kv, g, d_qk).sum(axis=3)).max() <= 1e-13
+    assert np.abs(dv - dv_r.reshape(b, s_k, h_kv, g, d_v).sum(axis=3)).max() <= 1e-13
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

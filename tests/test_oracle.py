@@ -21,6 +21,9 @@ PLANTS = {
     10: "v rows appended one row late",
     11: "rotary conjugate flag ignored",
     12: "left window one key short",
+    13: "backward softmax Jacobian row term dropped",
+    14: "backward scale missing from dk",
+    15: "backward dk and dv from the group's last query head only",
 }
 
 
