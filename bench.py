@@ -141,7 +141,8 @@ def traffic_record(config_key: str, kernel_tag: str):
     """DRAM traffic per launch of the attention kernel on this workload, from
     the committed ncu summary profiles/traffic_<workload>.md, if it was taken
     on the current kernel source (its sha256 prefix must match)."""
-    src = {"decode": "decode.cu", "prefill": "prefill_sm100.cu", "rotary": "rotary.cu"}.get(kernel_tag)
+    src = {"decode": "decode.cu", "prefill": "prefill_sm100.cu", "rotary": "rotary.cu",
+           "backward": "backward.cu"}.get(kernel_tag)
     summ = os.path.join(ROOT, "profiles", f"traffic_{config_key}.md")
     if not src or not os.path.exists(summ):
         return None
@@ -159,6 +160,23 @@ def traffic_record(config_key: str, kernel_tag: str):
 
 # ----------------------------------------------------------------------------- our arm
 def make_step(w, inp_dev, fa):
+    """(step, plan, outputs): `step` enqueues one library call on the current
+    stream; `outputs` are the tensors it writes (None entries are skipped)."""
+    if w.mode == "bwd":
+        q, k, v, dout = (inp_dev[n] for n in ("q", "k", "v", "dout"))
+        if "out" not in inp_dev:
+            # the forward's out and lse, made once outside every timed region
+            inp_dev["out"], inp_dev["lse"] = fa.fa_fwd(q, k, v, causal=w.causal, softmax_scale=w.scale or None,
+                                                       window=w.window)
+        out, lse = inp_dev["out"], inp_dev["lse"]
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(max(fa.fa_bwd_workspace_size(q), 1), dtype=torch.uint8, device=q.device)
+
+        def step():
+            fa.fa_bwd(q, k, v, out, dout, lse, causal=w.causal, softmax_scale=w.scale or None, window=w.window,
+                      dq=dq, dk=dk, dv=dv, workspace=ws)
+        plan = {"path": 0, "launches": 3, "n_splits": 1, "chunk": 0, "workspace_bytes": ws.numel()}
+        return step, plan, (dq, dk, dv)
     if w.mode == "varlen":
         q, k, v, cu = inp_dev["q"], inp_dev["k"], inp_dev["v"], inp_dev["cu_seqlens"]
         out = torch.empty((q.shape[0], q.shape[1], v.shape[2]), dtype=q.dtype, device=q.device)
@@ -239,22 +257,21 @@ def time_e2e(w, inp_host, inp_dev, step_fn_factory, steps, warmup, stream, flush
     """End-to-end through the public API: per step, copy the step's inputs from
     pinned host memory, run the call, read out + lse back to pinned host memory."""
     names = {"dense": ["q", "k", "v"], "rotary": ["q", "cache_seqlens"],
-             "varlen": ["q", "k", "v", "cu_seqlens"]}.get(
+             "varlen": ["q", "k", "v", "cu_seqlens"], "bwd": ["q", "k", "v", "out", "dout", "lse"]}.get(
         w.mode, ["q", "k_new", "v_new", "cache_seqlens"])
     pinned = {n: inp_host[n].pin_memory() for n in names}
-    step, _, (out, lse) = step_fn_factory()
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory() if lse is not None else None
+    step, _, outs = step_fn_factory()
+    outs = [t for t in outs if t is not None]
+    outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-    d2h = out_h.numel() * out_h.element_size() + (lse_h.numel() * lse_h.element_size() if lse is not None else 0)
+    d2h = sum(t.numel() * t.element_size() for t in outs_h)
 
     def e2e_step():
         for n in names:
             inp_dev[n].copy_(pinned[n], non_blocking=True)
         step()
-        out_h.copy_(out, non_blocking=True)
-        if lse is not None:
-            lse_h.copy_(lse, non_blocking=True)
+        for t, th in zip(outs, outs_h):
+            th.copy_(t, non_blocking=True)
     times = time_steps(e2e_step, steps, warmup, stream, flush_buf, barrier)
     return times, h2d, d2h
 
@@ -293,6 +310,19 @@ def cpu_sample(w, inp, budget_s):
             dt = time.perf_counter() - t0
             amount += W.rotary_bytes(w.scaled(batch=1, s_q=x.shape[1])) / 1e9
             done.append(f"b{bi}rows{i0}")
+        elif w.mode == "bwd":
+            # one (batch, head) pair, every query and key row
+            h = (b // w.batch) % w.h_q
+            hk = h // (w.h_q // w.h_kv)
+            q = inp["q"][bi:bi + 1, :, h:h + 1].double().numpy()
+            k = inp["k"][bi:bi + 1, :, hk:hk + 1].double().numpy()
+            v = inp["v"][bi:bi + 1, :, hk:hk + 1].double().numpy()
+            do = inp["dout"][bi:bi + 1, :, h:h + 1].double().numpy()
+            t0 = time.perf_counter()
+            oracle.bwd(q, k, v, do, causal=w.causal, scale=w.softmax_scale(), window=w.window)
+            dt = time.perf_counter() - t0
+            amount += W.flops(w.scaled(batch=1, h_q=1, h_kv=1)) / 1e12
+            done.append(f"b{bi}h{h}")
         elif w.mode == "dense":
             # one (batch, head) pair, every query row
             h = (b // w.batch) % w.h_q
@@ -323,7 +353,7 @@ def cpu_sample(w, inp, budget_s):
             done.append(f"b{bi}")
         t_total += dt
         b += 1
-    unit_desc = {"dense": "(batch, head) pairs", "rotary": "64-row blocks (all heads)",
+    unit_desc = {"dense": "(batch, head) pairs", "bwd": "(batch, head) pairs", "rotary": "64-row blocks (all heads)",
                  "varlen": "(sequence, head) pairs"}.get(w.mode, "batch entries")
     desc = (f"float64 oracle, single thread, on {len(done)} {unit_desc} of the workload "
             f"({', '.join(done[:8])}{'...' if len(done) > 8 else ''}); inputs converted to float64 "
@@ -400,6 +430,9 @@ def run_ours(args):
     flush_buf = L2Flush(device)
 
     step, plan, _ = make_step(w, inp_dev, fa)
+    if w.mode == "bwd":
+        # the end-to-end leg copies the forward's results in from the host too
+        inp["out"], inp["lse"] = inp_dev["out"].cpu(), inp_dev["lse"].cpu()
     # The timed step replays a CUDA graph of the library call, so the host's
     # Python/ctypes overhead is not inside the device-timed region.
     step()
@@ -446,6 +479,9 @@ def run_ours(args):
     kernel_tag = "rotary" if w.mode == "rotary" else ("decode" if plan["path"] == fa.FA_PATH_DECODE else "prefill")
     kernel_name = {fa.FA_PATH_DECODE: "decode_kernel", fa.FA_PATH_PREFILL: "prefill2_kernel / prefill_kernel",
                    fa.FA_PATH_DENSE: "prefill2_kernel / prefill_kernel"}.get(plan["path"], "rotary_kernel")
+    if w.mode == "bwd":
+        kernel_tag, kernel_name = "backward", "bwd_dkdv_kernel + bwd_dq_kernel"
+
     traffic = traffic_record(args.config, kernel_tag)
     result = {
         "metric": METRIC,

@@ -232,6 +232,42 @@ int fa_fwd_varlen(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
                   int32_t max_seqlen_q, int32_t causal, int32_t window_left, int32_t window_right,
                   float scale, const fa_tensor *out, float *lse, void *stream);
 
+/*
+ * fa_bwd -- gradients of fa_fwd_window (flash-attention PR #1604 "Support
+ * hdimQK != hdimV backward": d_qk may differ from d_v).  For out =
+ * softmax(scale q k^T + mask) v and an upstream gradient dout it writes
+ *   dq = d sum(dout * out) / dq, and likewise dk and dv,
+ * with the forward's mask (causal aligned bottom-right, window as in
+ * fa_fwd_window) and GQA mapping; a kv head's dk and dv sum the gradients of
+ * its group's query heads.
+ *  - q, dq [b, s_q, h_q, d_qk]; k, dk [b, s_k, h_kv, d_qk]; v, dv
+ *    [b, s_k, h_kv, d_v]; out, dout [b, s_q, h_q, d_v]: fp16/bf16 (one type
+ *    for all), head-dim stride 1, other strides and base addresses multiples
+ *    of 16 bytes.  q, k, v, out, dout are read only; dq, dk, dv are written
+ *    in full (zeros where no visible pair reaches an element) and must not
+ *    overlap the inputs.
+ *  - out and lse are the forward's results for the same q, k, v, mask and
+ *    scale (fa_fwd_window): lse fp32 [b, h_q, s_q], natural log, 4-byte
+ *    aligned.  P is recomputed as exp(scale q.k - lse).
+ *  - Head dims (d_qk, d_v): 64/64, 128/128, 192/128, else
+ *    FA_ERR_UNSUPPORTED.  scale <= 0 means 1/sqrt(d_qk).
+ *  - workspace: caller-owned device memory of fa_bwd_workspace_size bytes,
+ *    16-byte aligned (FA_ERR_WORKSPACE if smaller); it holds D_i =
+ *    dout_i . out_i as fp32 [b, h_q, s_q] and is dead after the call.
+ *  - Enqueued on `stream`; returns without synchronising.  The result does
+ *    not depend on scheduling (no atomics).  Errors: FA_ERR_INVALID_ARG
+ *    (shapes, types, window bounds below -1, lse missing), FA_ERR_LAYOUT,
+ *    FA_ERR_UNSUPPORTED, FA_ERR_CUDA.
+ */
+int fa_bwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
+           const fa_tensor *out, const fa_tensor *dout, const float *lse,
+           int32_t causal, int32_t window_left, int32_t window_right, float scale,
+           const fa_tensor *dq, const fa_tensor *dk, const fa_tensor *dv,
+           void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes fa_bwd needs for q of shape [b, s_q, h_q, d_qk]. */
+int fa_bwd_workspace_size(const fa_tensor *q, size_t *bytes);
+
 /* Workspace bytes fa_fwd needs for these shapes. */
 int fa_fwd_workspace_size(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
                           size_t *bytes);
@@ -298,9 +334,10 @@ int fa_rotary(const fa_tensor *x, const fa_tensor *cos, const fa_tensor *sin,
  *    enabled, or both NULL to switch the hook off.  The library does not own
  *    them; the caller keeps them alive while the hook is on.
  *  - While set, every fa_kvcache_fwd / fa_kvcache_fwd_noalloc / fa_fwd /
- *    fa_rotary call records `start` on its stream just before the launch of
- *    its main kernel (decode, prefill, generic attention or rotary) and
- *    `stop` just after it (inside a
+ *    fa_fwd_varlen / fa_rotary call records `start` on its stream just before
+ *    the launch of its main kernel (decode, prefill, generic attention or
+ *    rotary) and `stop` just after it; fa_bwd records them around its dk/dv
+ *    and dq kernels (after the D_i kernel) (inside a
  *    stream capture as external event-record nodes).  The events sit between
  *    the decode and combine kernels, so while the hook is on the combine
  *    launch no longer overlaps the decode kernel's tail.

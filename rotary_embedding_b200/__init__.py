@@ -68,6 +68,11 @@ lib.fa_kvcache_fwd_window.argtypes = [_P, _P, _P, _P, _P, _P, _P, _v, _i32, _i32
 lib.fa_kvcache_fwd_window.restype = ctypes.c_int
 lib.fa_fwd_varlen.argtypes = [_P, _P, _P, _v, _v, _i32, _i32, _i32, _i32, _i32, ctypes.c_float, _P, _v, _v]
 lib.fa_fwd_varlen.restype = ctypes.c_int
+lib.fa_bwd.argtypes = [_P, _P, _P, _P, _P, _v, _i32, _i32, _i32, ctypes.c_float, _P, _P, _P, _v, ctypes.c_size_t,
+                       _v]
+lib.fa_bwd.restype = ctypes.c_int
+lib.fa_bwd_workspace_size.argtypes = [_P, ctypes.POINTER(ctypes.c_size_t)]
+lib.fa_bwd_workspace_size.restype = ctypes.c_int
 lib.fa_fwd_workspace_size.argtypes = [_P, _P, _P, ctypes.POINTER(ctypes.c_size_t)]
 lib.fa_fwd_workspace_size.restype = ctypes.c_int
 lib.fa_device_status.argtypes = [_v, ctypes.POINTER(ctypes.c_int32)]
@@ -274,6 +279,32 @@ def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, causal=Fals
         int(bool(causal)), int(window[0]), int(window[1]), float(softmax_scale or 0.0), _ref(describe(out)),
         ctypes.c_void_p(lse.data_ptr()) if lse is not None else None, _stream_handle(stream, q.device)))
     return out, lse
+
+
+def fa_bwd_workspace_size(q):
+    n = ctypes.c_size_t(0)
+    _check(lib.fa_bwd_workspace_size(_ref(describe(q)), ctypes.byref(n)))
+    return n.value
+
+
+def fa_bwd(q, k, v, out, dout, lse, causal=False, softmax_scale=None, window=(-1, -1), dq=None, dk=None,
+           dv=None, workspace=None, stream=None):
+    """Gradients of fa_fwd for an upstream gradient dout, given the forward's
+    out and lse [b, h_q, s_q]: returns (dq, dk, dv) shaped like q, k, v."""
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        ws_bytes = fa_bwd_workspace_size(q)
+        if ws_bytes > 0:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    _check(lib.fa_bwd(
+        _ref(describe(q)), _ref(describe(k)), _ref(describe(v)), _ref(describe(out)), _ref(describe(dout)),
+        ctypes.c_void_p(lse.data_ptr()) if lse is not None else None, int(bool(causal)), int(window[0]),
+        int(window[1]), float(softmax_scale or 0.0), _ref(describe(dq)), _ref(describe(dk)), _ref(describe(dv)),
+        ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None,
+        workspace.numel() if workspace is not None else 0, _stream_handle(stream, q.device)))
+    return dq, dk, dv
 
 
 class FaPlan(ctypes.Structure):

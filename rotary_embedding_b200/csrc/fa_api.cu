@@ -819,6 +819,97 @@ int fa_fwd_varlen(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, co
                             cu_seqlens_k, n_seqs, max_seqlen_q);
 }
 
+int fa_bwd_workspace_size(const fa_tensor *q, size_t *bytes) {
+    g_last_error[0] = 0;
+    if (!bytes) return fail(FA_ERR_INVALID_ARG, "bytes is NULL");
+    Dims4 qd;
+    int rc;
+    if ((rc = check_tensor(q, "q", 4, 0, &qd))) return rc;
+    *bytes = align_up((size_t)(qd.n[0] * qd.n[1] * qd.n[2]) * sizeof(float), 256);
+    return FA_OK;
+}
+
+int fa_bwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, const fa_tensor *out,
+           const fa_tensor *dout, const float *lse, int32_t causal, int32_t window_left, int32_t window_right,
+           float scale, const fa_tensor *dq, const fa_tensor *dk, const fa_tensor *dv, void *workspace,
+           size_t workspace_bytes, void *stream) {
+    g_last_error[0] = 0;
+    if (window_left < -1 || window_right < -1)
+        return fail(FA_ERR_INVALID_ARG, "window bounds must be >= -1 (-1 = unbounded)");
+    Dims4 qd, kd, vd, od, dod, dqd, dkd, dvd;
+    int rc;
+    if ((rc = check_tensor(q, "q", 4, 0, &qd))) return rc;
+    if ((rc = check_tensor(k, "k", 4, q->dtype, &kd))) return rc;
+    if ((rc = check_tensor(v, "v", 4, q->dtype, &vd))) return rc;
+    if ((rc = check_tensor(out, "out", 4, q->dtype, &od))) return rc;
+    if ((rc = check_tensor(dout, "dout", 4, q->dtype, &dod))) return rc;
+    if ((rc = check_tensor(dq, "dq", 4, q->dtype, &dqd))) return rc;
+    if ((rc = check_tensor(dk, "dk", 4, q->dtype, &dkd))) return rc;
+    if ((rc = check_tensor(dv, "dv", 4, q->dtype, &dvd))) return rc;
+    const int64_t b = qd.n[0], s_q = qd.n[1], h_q = qd.n[2], d_qk = qd.n[3];
+    const int64_t s_k = kd.n[1], h_kv = kd.n[2], d_v = vd.n[3];
+    if (kd.n[0] != b || vd.n[0] != b) return fail(FA_ERR_INVALID_ARG, "k/v batch differs from q");
+    if (kd.n[3] != d_qk) return fail(FA_ERR_INVALID_ARG, "k head dim differs from q");
+    if (vd.n[1] != s_k || vd.n[2] != h_kv) return fail(FA_ERR_INVALID_ARG, "v shape differs from k");
+    if (h_kv <= 0 || h_q % h_kv) return fail(FA_ERR_INVALID_ARG, "h_q must be a multiple of h_kv");
+    auto same = [](const Dims4 &a, int64_t n0, int64_t n1, int64_t n2, int64_t n3) {
+        return a.n[0] == n0 && a.n[1] == n1 && a.n[2] == n2 && a.n[3] == n3;
+    };
+    if (!same(od, b, s_q, h_q, d_v)) return fail(FA_ERR_INVALID_ARG, "out shape must be [b, s_q, h_q, d_v]");
+    if (!same(dod, b, s_q, h_q, d_v)) return fail(FA_ERR_INVALID_ARG, "dout shape must be [b, s_q, h_q, d_v]");
+    if (!same(dqd, b, s_q, h_q, d_qk)) return fail(FA_ERR_INVALID_ARG, "dq shape must be that of q");
+    if (!same(dkd, b, s_k, h_kv, d_qk)) return fail(FA_ERR_INVALID_ARG, "dk shape must be that of k");
+    if (!same(dvd, b, s_k, h_kv, d_v)) return fail(FA_ERR_INVALID_ARG, "dv shape must be that of v");
+    if (!bwd_supported((int)d_qk, (int)d_v))
+        return fail(FA_ERR_UNSUPPORTED, "backward head dims (d_qk, d_v) must be 64/64, 128/128 or 192/128");
+    if (s_q > INT32_MAX || s_k > INT32_MAX || b > 65535 || h_q > 65535)
+        return fail(FA_ERR_UNSUPPORTED, "sizes past the launch limits");
+    if (!lse && b * s_q * h_q > 0) return fail(FA_ERR_INVALID_ARG, "lse is NULL");
+    if (reinterpret_cast<uintptr_t>(lse) & 3) return fail(FA_ERR_LAYOUT, "lse not 4-byte aligned");
+    if (b == 0 || h_q == 0) return FA_OK;
+    size_t need = 0;
+    if ((rc = fa_bwd_workspace_size(q, &need))) return rc;
+    if (workspace_bytes < need || (need && !workspace))
+        return fail(FA_ERR_WORKSPACE, "workspace of %zu bytes needed", need);
+    if (reinterpret_cast<uintptr_t>(workspace) & 15) return fail(FA_ERR_LAYOUT, "workspace not 16-byte aligned");
+    const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)d_qk);
+    BwdParams p{};
+    p.q = q->data;
+    p.qs = s3(qd);
+    p.k = k->data;
+    p.ks = s3(kd);
+    p.v = v->data;
+    p.vs = s3(vd);
+    p.out = out->data;
+    p.os = s3(od);
+    p.dout = dout->data;
+    p.dos = s3(dod);
+    p.lse = lse;
+    p.dsum = static_cast<float *>(workspace);
+    p.dq = dq->data;
+    p.dqs = s3(dqd);
+    p.dk = dk->data;
+    p.dks = s3(dkd);
+    p.dv = dv->data;
+    p.dvs = s3(dvd);
+    p.b = (int)b;
+    p.s_q = (int)s_q;
+    p.s_k = (int)s_k;
+    p.h_q = (int)h_q;
+    p.h_kv = (int)h_kv;
+    p.g = (int)(h_q / h_kv);
+    p.d_qk = (int)d_qk;
+    p.d_v = (int)d_v;
+    p.causal = causal ? 1 : 0;
+    p.win_left = window_left;
+    p.win_right = window_right;
+    p.scale = sc;
+    p.scale_log2 = sc * 1.4426950408889634f;
+    cudaError_t e = launch_bwd(p, q->dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    return FA_OK;
+}
+
 int fa_device_status(void *stream, int32_t *status) {
     g_last_error[0] = 0;
     if (!status) return fail(FA_ERR_INVALID_ARG, "status is NULL");

@@ -150,6 +150,31 @@ int set_last_error(int code, const char *msg);
 // which = 0 before the attention kernel's launch, 1 after it.
 void kernel_event(int which, cudaStream_t st);
 
+// Attention backward (dq, dk, dv) over dense [b, s, h, d] tensors.
+struct BwdParams {
+    const void *q;
+    Strides3 qs;
+    const void *k;
+    Strides3 ks;
+    const void *v;
+    Strides3 vs;
+    const void *out;
+    Strides3 os;
+    const void *dout;
+    Strides3 dos;
+    const float *lse;  // [b, h_q, s_q], natural log, from the forward
+    float *dsum;       // [b, h_q, s_q] workspace: D_i = dout_i . out_i
+    void *dq;
+    Strides3 dqs;
+    void *dk;
+    Strides3 dks;
+    void *dv;
+    Strides3 dvs;
+    int b, s_q, s_k, h_q, h_kv, g, d_qk, d_v, causal;
+    int win_left, win_right;  // sliding window; -1 = unbounded
+    float scale, scale_log2;
+};
+
 cudaError_t launch_rope_append(const RopeAppendParams &p, int dtype, cudaStream_t st);
 cudaError_t launch_rotary(const RotaryParams &p, int dtype, cudaStream_t st);
 bool prefill_supported(int d_qk, int d_v);
@@ -162,5 +187,7 @@ cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmQ, const C
                           const CUtensorMap &tmV, int dtype, int d_qk, int d_v, int mt, cudaStream_t st);
 bool decode_supported(int d_qk, int d_v, int mt);
 cudaError_t launch_simt_attn(const SimtAttnParams &p, int dtype, cudaStream_t st);
+bool bwd_supported(int d_qk, int d_v);
+cudaError_t launch_bwd(const BwdParams &p, int dtype, cudaStream_t st);
 
 }  // namespace fa

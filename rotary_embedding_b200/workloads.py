@@ -31,8 +31,9 @@ _DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    mode: str                 # "kvcache" (fa_kvcache_fwd), "dense" (fa_fwd), "rotary" (fa_rotary)
-                              # or "varlen" (fa_fwd_varlen: batch packed sequences, lengths ~ U{seqlens})
+    mode: str                 # "kvcache" (fa_kvcache_fwd), "dense" (fa_fwd), "rotary" (fa_rotary),
+                              # "varlen" (fa_fwd_varlen: batch packed sequences, lengths ~ U{seqlens})
+                              # or "bwd" (fa_bwd over the dense shapes, with an upstream gradient dout)
     dtype: str                # "fp16" | "bf16"
     batch: int
     h_q: int
@@ -110,7 +111,11 @@ VARLEN_PREFILL = Workload(
     name="varlen-prefill bf16 8 seqs len~U{256..4096} h16 d128 causal", mode="varlen", dtype="bf16",
     batch=8, h_q=16, h_kv=16, d_qk=128, d_v=128, s_q=4096, seqlens=(256, 4096), causal=True)
 
+# Backward of the MLA prefill (flash-attention PR #1604: d_qk 192, d_v 128).
+MLA_BACKWARD = MLA_PREFILL.scaled(name="mla-backward bf16 b4 h16 s4096 dqk192 dv128 causal", mode="bwd")
+
 CONFIGS = {
+    "mla-backward": MLA_BACKWARD,
     "rotary-q": ROTARY_Q,
     "varlen-prefill": VARLEN_PREFILL,
     "window-prefill": WINDOW_PREFILL,
@@ -162,11 +167,14 @@ def make_inputs(w: Workload, seed: int = 0) -> dict:
         cu = torch.zeros(w.batch + 1, dtype=torch.int32)
         cu[1:] = torch.cumsum(lens, 0)
         return {"q": q, "k": k, "v": v, "cu_seqlens": cu}
-    if w.mode == "dense":
+    if w.mode in ("dense", "bwd"):
         q = _draw(g, (w.batch, w.s_q, w.h_q, w.d_qk), w.dist, dt)
         k = _draw(g, (w.batch, w.s_k, w.h_kv, w.d_qk), w.dist, dt)
         v = _draw(g, (w.batch, w.s_k, w.h_kv, w.d_v), w.dist, dt)
-        return {"q": q, "k": k, "v": v}
+        if w.mode == "dense":
+            return {"q": q, "k": k, "v": v}
+        dout = _draw(g, (w.batch, w.s_q, w.h_q, w.d_v), w.dist, dt)
+        return {"q": q, "k": k, "v": v, "dout": dout}
     q = _draw(g, (w.batch, w.s_q, w.h_q, w.d_qk), w.dist, dt)
     if w.kv_is_q:
         k_new, v_new = q.clone(), q.clone()
@@ -217,7 +225,7 @@ def visible_pairs(w: Workload, seqlens=None) -> int:
         # seqlens: the drawn lengths; each sequence is a batch of one with s_q = s_k
         return sum(visible_pairs(w.scaled(mode="dense", batch=1, s_q=int(n), s_k=int(n)))
                    for n in seqlens) if seqlens is not None else 0
-    if w.mode == "dense":
+    if w.mode in ("dense", "bwd"):
         lens = [w.s_k] * w.batch
         s_q = w.s_q
     else:
@@ -249,5 +257,8 @@ def visible_pairs(w: Workload, seqlens=None) -> int:
 
 
 def flops(w: Workload, seqlens=None) -> float:
-    """Algorithmic FLOPs: 2*(d_qk + d_v) per visible (query, key) pair."""
-    return 2.0 * (w.d_qk + w.d_v) * visible_pairs(w, seqlens)
+    """Algorithmic FLOPs per visible (query, key) pair: forward 2*(d_qk + d_v)
+    (q.k and p*v); backward 2*(3*d_qk + 2*d_v) (q.k, dout.v, p*dout into dv,
+    ds*q into dk, ds*k into dq)."""
+    per_pair = 2.0 * (3 * w.d_qk + 2 * w.d_v) if w.mode == "bwd" else 2.0 * (w.d_qk + w.d_v)
+    return per_pair * visible_pairs(w, seqlens)
