@@ -227,6 +227,12 @@ int run_tc_attention(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
         if (env[0] == '1') p.tiles_per_cta = 1;
         if (env[0] == '2') p.tiles_per_cta = 2;
     }
+    // Under a causal mask the work of query tile t grows with t.  When the
+    // two-tile grid is one wave, the slowest CTA sets the time, so pair tile
+    // k with tile n-1-k (every CTA then sees about the same number of key
+    // tiles); with several waves the heaviest-first launch order balances
+    // adjacent pairs, which keep both softmax warpgroups busy to the end.
+    p.pair_ends = (causal && !varlen && p.tiles_per_cta == 2 && ctas2 <= sms) ? 1 : 0;
     const int bn = prefill_block_n((int)d_qk, (int)d_v, p.tiles_per_cta);
     CUtensorMap tmQ, tmK, tmV;
     int rc;

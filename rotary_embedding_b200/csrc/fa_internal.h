@@ -119,6 +119,9 @@ struct PrefillParams {
     int64_t cap;   // kvcache mode capacity (precondition check)
     int kvcache, b, s_q, h_q, h_kv, g, pack, causal, n_q_tiles;
     int tiles_per_cta;  // 1: one 128-row tile per CTA; 2: two tiles, two softmax warpgroups
+    // two-tile kernel: 0 = CTA k takes query tiles 2k and 2k+1; 1 = tiles k
+    // and n_q_tiles-1-k (equal causal work per CTA, for single-wave grids)
+    int pair_ends;
     int win_left, win_right;  // sliding window; -1 = unbounded
     // packed sequences (varlen): grid z = sequence s with query rows
     // cu_q[s] .. cu_q[s+1]-1 and key rows cu_k[s] .. of batch entry 0;

@@ -487,13 +487,24 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
     } else {
         N = (int)p.s_k;
     }
-    if (2 * blk * rows_per_tile >= sq) return;             // past this sequence's rows
+    // the CTA's two query tiles: 2 blk and 2 blk + 1, or blk and
+    // n_q_tiles - 1 - blk (the middle tile of an odd count pairs with an
+    // empty tile past the rows); every tile index is taken exactly once
+    int tile[2];
+    if (p.pair_ends) {
+        tile[0] = blk;
+        tile[1] = p.n_q_tiles - 1 - blk > blk ? p.n_q_tiles - 1 - blk : p.n_q_tiles;
+    } else {
+        tile[0] = 2 * blk;
+        tile[1] = 2 * blk + 1;
+    }
+    if (tile[0] * rows_per_tile >= sq) return;             // past this sequence's rows (tile[1] > tile[0])
     // per tile: key tiles kb[x] .. n_kv[x] - 1 (causal, window), and the
     // bounds past which a key tile needs an element mask (see prefill_kernel)
     int i0[2], n_kv[2], kb[2], mask_from[2], lo_max[2];
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
-        i0[x] = (2 * blk + x) * rows_per_tile;
+        i0[x] = tile[x] * rows_per_tile;
         const int i_last = min(sq, i0[x] + rows_per_tile) - 1;
         int64_t f_first, l_first, f_last, l_last;
         visible_keys(i0[x], N, sq, p.causal, p.win_left, p.win_right, f_first, l_first);
@@ -648,7 +659,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         const int q4 = warp & 3;                       // TMEM lane quadrant this warp may access
         const int r = q4 * 32 + lane;                  // tile row = TMEM lane
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
-        const int prow = (2 * blk + x) * kBM + r;      // packed row
+        const int prow = tile[x] * kBM + r;            // packed row
         const int i = prow / pack;
         const int hq = hq0 + (prow % pack);
         const bool row_valid = i < sq;
