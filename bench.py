@@ -42,6 +42,9 @@ from rotary_embedding_b200 import workloads as W  # noqa: E402
 
 METRIC = "prefill attention TFLOP/s and decode KV-cache GB/s on 1 B200, % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Nominal B200 figures (HGX HBM3e bandwidth; dense bf16/fp16 tensor rate, no sparsity), reported beside
+# the measured peaks as a second ceiling.
+SPEC_PEAKS = {"hbm": (7700.0, "GB/s"), "tensor": (2250.0, "TFLOP/s")}
 DEFAULT_CONFIG = "gqa-decode"
 
 
@@ -361,6 +364,18 @@ def cpu_sample(w, inp, budget_s):
     return amount, t_total, desc
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (for the oracle baseline's record)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def aggregate_over_ranks(ms_local: float, amount: float, world: int, device):
     """Whole-job throughput: every rank processed `amount` units in its own
     device time; the job takes the slowest rank's time (max over ranks)."""
@@ -512,6 +527,8 @@ def run_ours(args):
                      "timing": ("CUDA events around the kernel's launch on its stream, graph replay, "
                                 "L2 flushed per step" if kernel_ms else "whole call (kernel events unavailable)"),
                      "call_ms": round(ms, 5),
+                     "spec_peak": SPEC_PEAKS[bound][0] if bound in SPEC_PEAKS else None,
+                     "frac_of_spec": (round(achieved / SPEC_PEAKS[bound][0], 4) if bound in SPEC_PEAKS else None),
                      "amount_per_launch": amount},
         "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -522,7 +539,8 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         amt, secs, desc = cpu_sample(w, inp, args.cpu_seconds)
         result["cpu_baseline"] = {"value": round(amt / secs, 6), "unit": unit, "cores": 1,
-                                  "kind": "oracle", "sample": desc, "seconds": round(secs, 2)}
+                                  "kind": "oracle", "sample": desc, "seconds": round(secs, 2),
+                                  "cpu": cpu_model(), "host_cores": os.cpu_count()}
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -557,7 +575,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)", "config": {"workload": w.name},
         "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": 1, "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc, "cpu": cpu_model(), "host_cores": os.cpu_count()},
         "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
