@@ -32,7 +32,7 @@
  *       [batch, seq, heads, dim], causal flag, softmax_scale=None means
  *       1/sqrt(d)) and Step 3 (fewer KV heads than query heads).
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *  - the query row i of batch b sits at position cache_seqlens[b] + i, the
  *    same position as new key row i;
  *  - half-split pairs (j, j + r/2) inside the first r dims, interleaved
