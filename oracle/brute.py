@@ -31,16 +31,26 @@ def rope_row(x, theta, rotary_dim, interleaved):
     return y
 
 
-def visible(i, j, s_q, n_keys, causal):
-    """Bottom-right causal visibility of key j to query i."""
+def visible(i, j, s_q, n_keys, causal, window=(-1, -1)):
+    """Visibility of key j to query i, stated through the signed distance
+    dist = (i + n_keys - s_q) - j from the query's bottom-right aligned key:
+    causal keeps dist >= 0; a sliding window ("optimizing-attention-flash",
+    window_size=(left, right), -1 = unbounded) keeps dist <= left and
+    -dist <= right."""
     if j >= n_keys:
         return False
-    if not causal:
-        return True
-    return j - (n_keys - s_q) <= i
+    dist = (i + n_keys - s_q) - j
+    if causal and dist < 0:
+        return False
+    left, right = window
+    if left >= 0 and dist > left:
+        return False
+    if right >= 0 and -dist > right:
+        return False
+    return True
 
 
-def attention(q, keys, vals, s_q, causal, scale):
+def attention(q, keys, vals, s_q, causal, scale, window=(-1, -1)):
     """q: [s_q][d_qk], keys: [N][d_qk], vals: [N][d_v] -> (out [s_q][d_v], lse [s_q])."""
     n = len(keys)
     d_v = len(vals[0]) if vals else 0
@@ -48,7 +58,7 @@ def attention(q, keys, vals, s_q, causal, scale):
     for i in range(s_q):
         weights = []
         for j in range(n):
-            if visible(i, j, s_q, n, causal):
+            if visible(i, j, s_q, n, causal, window):
                 s = scale * sum(a * b for a, b in zip(q[i], keys[j]))
                 weights.append((j, math.exp(s)))
         if not weights:

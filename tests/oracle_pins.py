@@ -538,6 +538,28 @@ def pin_window_in_kvcache_mode(lib):
     assert np.allclose(out, ref, atol=1e-14) and np.allclose(lse, rlse, atol=1e-14)
 
 
+def pin_brute_force_windows(lib):
+    """The oracle's window bounds agree with the brute force's distance
+    predicate ("optimizing-attention-flash", window_size=(left, right)) on
+    tiny shapes: causal and not, s_q below, equal to and above the key count,
+    one- and two-sided windows, GQA."""
+    rng = np.random.default_rng(71)
+    for s_q, s_k in ((3, 6), (5, 5), (6, 3)):
+        for causal in (True, False):
+            for window in ((1, -1), (0, 2), (2, 1), (-1, 0), (4, 3)):
+                q = rng.standard_normal((1, s_q, 2, 3))
+                k = rng.standard_normal((1, s_k, 1, 3))
+                v = rng.standard_normal((1, s_k, 1, 2))
+                out, lse = oracle.fwd(q, k, v, causal=causal, window=window, lib=lib)
+                for h in range(2):
+                    bo, bl = brute.attention([list(r) for r in q[0, :, h]], [list(r) for r in k[0, :, 0]],
+                                             [list(r) for r in v[0, :, 0]], s_q, causal, 1 / math.sqrt(3), window)
+                    assert np.allclose(out[0, :, h], np.array(bo), rtol=0, atol=1e-12)
+                    assert np.array_equal(np.isinf(lse[0, h]), np.isinf(np.array(bl)))
+                    fin = np.isfinite(lse[0, h])
+                    assert np.allclose(lse[0, h][fin], np.array(bl)[fin], rtol=0, atol=1e-12)
+
+
 def pin_varlen_sequences_are_independent(lib):
     """Packed sequences ([P2] IS_VARLEN) do not see each other: changing one
     sequence's keys and values leaves every other sequence's output and lse
