@@ -4,8 +4,9 @@ window masks) against the float64 oracle's gradient.
 Tolerance (normwise, per tensor): max|got - ref| <= TOL * max|ref|.  The
 kernels round P and dS to the element type as MMA operands, read D_i from
 the rounded out, and round dq, dk, dv; a numpy model of exactly those
-roundings differs from the float64 gradient by at most 5.1e-3 (bf16) and
-6.9e-4 (fp16) of max|ref| on these shapes.  TOL is four times that.
+roundings (_rounding_model) differs from the float64 gradient by at most
+5.1e-3 (bf16) and 6.9e-4 (fp16) of max|ref| on these shapes.  TOL is four
+times that; test_bwd_tolerance_covers_the_rounding_model keeps the margin.
 Gradients that no visible (query, key) pair reaches (a query row that sees no
 key, a key no query sees) must be exactly zero.  Gradients that are zero only
 by cancellation (a row with one visible key has P = 1, so dP - D = 0) are
@@ -83,6 +84,62 @@ def _check(got, ref, dtype, unreached=None):
         if unreached is not None:
             mask = np.broadcast_to(unreached[0] if x == 0 else unreached[1], a.shape)
             assert np.all(a[mask] == 0.0), f"{name}: nonzero where no visible pair reaches"
+
+
+def _rounding_model(q, k, v, do, out, lse, causal, window, dtype):
+    """The kernels' arithmetic with their roundings and nothing else: P from
+    the forward's lse in fp32, P and dS rounded to the element type as MMA
+    operands, D from the rounded out, dq/dk/dv rounded; products otherwise
+    exact.  Used only to derive TOL."""
+    def rnd(x):
+        return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(DT[dtype]).double().numpy()
+    b, s_q, h_q, d = q.shape
+    s_k, h_kv = k.shape[1], k.shape[2]
+    g = h_q // h_kv
+    sc = 1.0 / np.sqrt(d)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    i = np.arange(s_q)[:, None]
+    j = np.arange(s_k)[None, :]
+    dist = i + s_k - s_q - j
+    vis = np.ones((s_q, s_k), bool)
+    if causal:
+        vis &= dist >= 0
+    if window[0] >= 0:
+        vis &= dist <= window[0]
+    if window[1] >= 0:
+        vis &= -dist <= window[1]
+    for bi in range(b):
+        for h in range(h_q):
+            hk = h // g
+            s = (q[bi, :, h] @ k[bi, :, hk].T).astype(np.float32)
+            L = lse[bi, h][:, None].astype(np.float32)
+            p = np.where(vis, np.exp2(s * np.float32(sc * np.log2(np.e)) - L * np.float32(np.log2(np.e))), 0)
+            dp = (do[bi, :, h] @ v[bi, :, hk].T).astype(np.float32)
+            dsum = (do[bi, :, h] * out[bi, :, h]).sum(-1).astype(np.float32)[:, None]
+            ds = (p * (dp - dsum)).astype(np.float32)
+            dv[bi, :, hk] += rnd(p).T @ do[bi, :, h]
+            dk[bi, :, hk] += sc * (rnd(ds).T @ q[bi, :, h])
+            dq[bi, :, h] = sc * (rnd(ds) @ k[bi, :, hk])
+    return rnd(dq), rnd(dk), rnd(dv)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_bwd_tolerance_covers_the_rounding_model(dtype):
+    """TOL stays at least three times the normwise error that the kernels'
+    roundings alone cause, on shapes of the GPU parity cases."""
+    worst = 0.0
+    for (d_qk, d_v), (causal, window), shape in (((192, 128), (True, (-1, -1)), (2, 100, 170, 4, 1)),
+                                                ((64, 64), (False, (30, 20)), (1, 200, 64, 2, 1)),
+                                                ((128, 128), (True, (40, -1)), (1, 130, 130, 2, 2))):
+        b, s_q, s_k, h_q, h_kv = shape
+        q, k, v, do = (t.double().numpy() for t in _case(d_qk + s_q + s_k, b, s_q, s_k, h_q, h_kv, d_qk, d_v, dtype))
+        out, lse = oracle.fwd(q, k, v, causal=causal, window=window)
+        out = torch.from_numpy(out).to(DT[dtype]).double().numpy()
+        ref = oracle.bwd(q, k, v, do, causal=causal, window=window)
+        got = _rounding_model(q, k, v, do, out, lse, causal, window, dtype)
+        for a, r in zip(got, ref):
+            worst = max(worst, np.abs(a - r).max() / np.abs(r).max())
+    assert 3.0 * worst <= TOL[dtype], (worst, TOL[dtype])
 
 
 @pytest.mark.gpu
