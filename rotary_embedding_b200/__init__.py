@@ -105,6 +105,23 @@ def _ref(d):
     return ctypes.byref(d) if d is not None else None
 
 
+def _lse_ptr(lse, shape):
+    """Pointer to an fp32 lse buffer of exactly `shape`, contiguous (the C
+    ABI takes lse as a plain float array in that layout), or None."""
+    if lse is None:
+        return None
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != tuple(shape):
+        raise ValueError(f"lse must be a contiguous float32 tensor of shape {tuple(shape)}")
+    return ctypes.c_void_p(lse.data_ptr())
+
+
+def _i32_ptr(t, name, min_len):
+    """Pointer to a contiguous int32 tensor of at least `min_len` entries."""
+    if t.dtype != torch.int32 or not t.is_contiguous() or t.numel() < min_len:
+        raise ValueError(f"{name} must be a contiguous int32 tensor of at least {min_len} entries")
+    return ctypes.c_void_p(t.data_ptr())
+
+
 def _check(status: int):
     if status != FA_OK:
         msg = lib.fa_last_error().decode() or lib.fa_status_string(status).decode()
@@ -155,7 +172,7 @@ def fa_kvcache_fwd(q, k_cache, v_cache, k_new=None, v_new=None, rotary_cos=None,
         if ws_bytes > 0:
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     if isinstance(cache_seqlens, torch.Tensor):
-        seq_ptr, seq_scalar = ctypes.c_void_p(cache_seqlens.data_ptr()), 0
+        seq_ptr, seq_scalar = _i32_ptr(cache_seqlens, "cache_seqlens", b), 0
     else:
         seq_ptr, seq_scalar = None, int(cache_seqlens)
     dq = describe(q)
@@ -164,7 +181,7 @@ def fa_kvcache_fwd(q, k_cache, v_cache, k_new=None, v_new=None, rotary_cos=None,
         _ref(describe(v_new)), _ref(describe(rotary_cos)), _ref(describe(rotary_sin)), seq_ptr,
         seq_scalar, rotary_dim, int(bool(rotary_interleaved)), int(bool(causal)), int(window[0]),
         int(window[1]), float(softmax_scale or 0.0), _ref(describe(out)),
-        ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+        _lse_ptr(lse, (b, h_q, s_q)),
         ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None,
         workspace.numel() if workspace is not None else 0, _stream_handle(stream, q.device)))
     return out, lse
@@ -188,12 +205,12 @@ def fa_rotary(x, cos, sin, seqlen_offsets=0, rotary_dim=None, interleaved=False,
     ov = out.unsqueeze(0) if packed else out
     if rotary_dim is None:
         rotary_dim = 2 * cos.shape[1] if cos is not None else 0
+    n_seqs = int(cu_seqlens.numel()) - 1 if packed else 0
     if isinstance(seqlen_offsets, torch.Tensor):
-        off_ptr, off_scalar = ctypes.c_void_p(seqlen_offsets.data_ptr()), 0
+        off_ptr, off_scalar = _i32_ptr(seqlen_offsets, "seqlen_offsets", n_seqs if packed else x.shape[0]), 0
     else:
         off_ptr, off_scalar = None, int(seqlen_offsets)
-    cu_ptr = ctypes.c_void_p(cu_seqlens.data_ptr()) if packed else None
-    n_seqs = int(cu_seqlens.numel()) - 1 if packed else 0
+    cu_ptr = _i32_ptr(cu_seqlens, "cu_seqlens", 1) if packed else None
     _check(lib.fa_rotary(_ref(describe(xv)), _ref(describe(cos)), _ref(describe(sin)), off_ptr, off_scalar,
                          cu_ptr, n_seqs, int(rotary_dim), int(bool(interleaved)), int(bool(conjugate)),
                          _ref(describe(ov)), _stream_handle(stream, x.device)))
@@ -225,7 +242,7 @@ def fa_kvcache_fwd_noalloc(q, k_cache, v_cache, k_new=None, v_new=None, rotary_c
     if lse is None and return_lse:
         lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
     if isinstance(cache_seqlens, torch.Tensor):
-        seq_ptr, seq_scalar = ctypes.c_void_p(cache_seqlens.data_ptr()), 0
+        seq_ptr, seq_scalar = _i32_ptr(cache_seqlens, "cache_seqlens", b), 0
     else:
         seq_ptr, seq_scalar = None, int(cache_seqlens)
     _check(lib.fa_kvcache_fwd_noalloc(
@@ -233,7 +250,7 @@ def fa_kvcache_fwd_noalloc(q, k_cache, v_cache, k_new=None, v_new=None, rotary_c
         _ref(describe(v_new)), _ref(describe(rotary_cos)), _ref(describe(rotary_sin)), seq_ptr,
         seq_scalar, rotary_dim, int(bool(rotary_interleaved)), int(bool(causal)),
         float(softmax_scale or 0.0), _ref(describe(out)),
-        ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+        _lse_ptr(lse, (b, h_q, s_q)),
         _stream_handle(stream, q.device)))
     return out, lse
 
@@ -256,7 +273,7 @@ def fa_fwd(q, k, v, causal=False, softmax_scale=None, out=None, lse=None, worksp
     _check(lib.fa_fwd_window(
         _ref(describe(q)), _ref(describe(k)), _ref(describe(v)), int(bool(causal)), int(window[0]),
         int(window[1]), float(softmax_scale or 0.0), _ref(describe(out)),
-        ctypes.c_void_p(lse.data_ptr()) if lse is not None else None,
+        _lse_ptr(lse, (b, h_q, s_q)),
         ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None,
         workspace.numel() if workspace is not None else 0, _stream_handle(stream, q.device)))
     return out, lse
@@ -274,10 +291,11 @@ def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, causal=Fals
     if lse is None and return_lse:
         lse = torch.empty((h_q, total_q), dtype=torch.float32, device=q.device)
     _check(lib.fa_fwd_varlen(
-        _ref(describe(q)), _ref(describe(k)), _ref(describe(v)), ctypes.c_void_p(cu_seqlens_q.data_ptr()),
-        ctypes.c_void_p(cu_seqlens_k.data_ptr()), int(cu_seqlens_q.numel()) - 1, int(max_seqlen_q),
+        _ref(describe(q)), _ref(describe(k)), _ref(describe(v)),
+        _i32_ptr(cu_seqlens_q, "cu_seqlens_q", 2), _i32_ptr(cu_seqlens_k, "cu_seqlens_k", cu_seqlens_q.numel()),
+        int(cu_seqlens_q.numel()) - 1, int(max_seqlen_q),
         int(bool(causal)), int(window[0]), int(window[1]), float(softmax_scale or 0.0), _ref(describe(out)),
-        ctypes.c_void_p(lse.data_ptr()) if lse is not None else None, _stream_handle(stream, q.device)))
+        _lse_ptr(lse, (h_q, total_q)), _stream_handle(stream, q.device)))
     return out, lse
 
 
@@ -300,7 +318,7 @@ def fa_bwd(q, k, v, out, dout, lse, causal=False, softmax_scale=None, window=(-1
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     _check(lib.fa_bwd(
         _ref(describe(q)), _ref(describe(k)), _ref(describe(v)), _ref(describe(out)), _ref(describe(dout)),
-        ctypes.c_void_p(lse.data_ptr()) if lse is not None else None, int(bool(causal)), int(window[0]),
+        _lse_ptr(lse, (q.shape[0], q.shape[2], q.shape[1])), int(bool(causal)), int(window[0]),
         int(window[1]), float(softmax_scale or 0.0), _ref(describe(dq)), _ref(describe(dk)), _ref(describe(dv)),
         ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None,
         workspace.numel() if workspace is not None else 0, _stream_handle(stream, q.device)))
