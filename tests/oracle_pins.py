@@ -52,6 +52,31 @@ def pin_round_fp16_matches_numpy(lib):
     assert np.array_equal(got, want), "fp16 rounding differs from numpy's correctly rounded cast"
 
 
+def pin_round_bf16_matches_torch(lib):
+    """bf16 rounding equals torch's round-to-nearest-even cast from float32 on
+    4000 random float32 bit patterns (normals of every exponent, subnormals
+    down to 2^-149, values past the largest finite bf16) and on the edges:
+    the smallest bf16 subnormal 2^-133 and the ties around it, the largest
+    finite bf16 (2 - 2^-7) 2^127, and the midpoint above it, which rounds to
+    infinity.  Every value is a float32, so the float64 the oracle takes and
+    the float32 torch takes are the same number."""
+    import torch
+    rng = np.random.default_rng(7)
+    x32 = rng.integers(0, 2 ** 32, 4000, dtype=np.uint64).astype(np.uint32).view(np.float32)
+    x32 = x32[np.isfinite(x32)]
+    top = (2.0 - 2.0 ** -7) * 2.0 ** 127
+    edges = np.array([2.0 ** -133, 2.0 ** -134, 3 * 2.0 ** -134, 1.5 * 2.0 ** -133, 2.0 ** -126,
+                      2.0 ** -126 - 2.0 ** -134, 2.0 ** -127 + 2.0 ** -134, top, -top,
+                      (2.0 - 2.0 ** -8) * 2.0 ** 127, (2.0 - 2.0 ** -9) * 2.0 ** 127,
+                      -(2.0 - 2.0 ** -8) * 2.0 ** 127, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8], dtype=np.float32)
+    x = np.concatenate([x32, edges]).astype(np.float64)
+    got = oracle.round_to(x, "bf16")
+    want = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    bad = np.flatnonzero(got != want)
+    assert bad.size == 0, f"bf16 rounding differs from torch at {x[bad[:5]]}: {got[bad[:5]]} vs {want[bad[:5]]}"
+    assert np.isinf(oracle.round_to(np.array([(2.0 - 2.0 ** -8) * 2.0 ** 127]), "bf16")[0])
+
+
 def pin_round_bf16_ties_to_even(lib):
     # exact bf16 neighbours of 1.0 are 1.0 and 1 + 2^-7; the midpoint ties to the even one
     cases = {1.0 + 2.0 ** -8: 1.0, 1.0 + 3 * 2.0 ** -8: 1.0 + 2.0 ** -6,
