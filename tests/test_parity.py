@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import rotary_embedding_b200 as fa
-from rotary_embedding_b200 import workloads as W
+import workloads as W
 from parity_util import (LSE_TOL, OUT_TOL, check_dense, check_kvcache, run_gpu_dense,
                          run_gpu_kvcache, run_oracle_kvcache, to_dtype_cpu, ulp_distance)
 
@@ -169,13 +169,6 @@ def test_empty_batch(cuda_device):
 
 
 # ------------------------------------------------------------------ dense (fa_fwd)
-@pytest.fixture(params=["1", "2"], ids=["1tile", "2tiles"])
-def prefill_tiles(request, monkeypatch):
-    """Run the test with the one-tile and with the two-tile prefill kernel."""
-    monkeypatch.setenv("FA_PREFILL_TILES_PER_CTA", request.param)
-    return int(request.param)
-
-
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("dims", [(64, 64, "fp16"), (192, 128, "bf16"), (128, 128, "bf16"), (16, 16, "fp16")])
 def test_dense_small(dims, causal, prefill_tiles, cuda_device):
@@ -274,8 +267,16 @@ def test_full_size_dense_configs(name, cuda_device):
     w = W.CONFIGS[name]
     inp = W.make_inputs(w)
     out, lse = run_gpu_dense(w, inp, cuda_device)
-    # sampled (batch, head, query-row block) triples against the oracle on the keys they see
-    for b, h, r0, r1 in ((0, 0, 0, 64), (w.batch - 1, w.h_q - 1, w.s_q - 128, w.s_q), (0, 3, 1000, 1100)):
+    # sampled (batch, head, query-row block) triples against the oracle on the keys they see:
+    # the first and last rows, a block across a tile boundary, and one block inside every
+    # 128-row query tile (so every tile of every CTA, whichever tiles a CTA pairs, is
+    # checked), with the batch entry, head and offset inside the tile varying
+    blocks = [(0, 0, 0, 64), (w.batch - 1, w.h_q - 1, w.s_q - 128, w.s_q), (0, 3, 1000, 1100)]
+    n_tiles = (w.s_q + 127) // 128
+    for t in range(n_tiles):
+        r0 = t * 128 + (37 * t) % 112
+        blocks.append((t % w.batch, (5 * t + 1) % w.h_q, r0, min(r0 + 16, w.s_q)))
+    for b, h, r0, r1 in blocks:
         k1 = r1 if w.causal else w.s_k
         q = inp["q"][b:b + 1, r0:r1, h:h + 1].double().numpy()
         k = inp["k"][b:b + 1, :k1, h:h + 1].double().numpy()

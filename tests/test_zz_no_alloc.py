@@ -5,17 +5,18 @@ plug-in whose host application owns every allocation, or a loop that must
 never enter the CUDA allocator).  For them the library offers a variant of
 fa_kvcache_fwd whose scratch lives in a fixed array inside the library.
 These checks call it through the C ABI and compare it with the workspace
-entry point, on two calls in a row (the second call finds the first call's
-data in the shared scratch).  The file name sorts last so that a run that
-stops at the first failure has already run every other test.
+entry point and with the float64 oracle, on two calls in a row (the second
+call finds the first call's data in the shared scratch).  The file name
+sorts last so that a run that stops at the first failure has already run
+every other test.
 """
 import numpy as np
 import pytest
 import torch
 
 import rotary_embedding_b200 as fa
-from rotary_embedding_b200 import workloads as W
-from parity_util import LSE_TOL, OUT_TOL
+import workloads as W
+from parity_util import LSE_TOL, OUT_TOL, check_kvcache, run_oracle_kvcache
 
 pytestmark = pytest.mark.gpu
 
@@ -42,9 +43,11 @@ def test_noalloc_matches_workspace_entry_point(w, cuda_device):
     ws = fa.fa_kvcache_plan(inp["q"], inp["k_cache"], inp["v_cache"], inp["k_new"], w.rotary_dim)
     assert 0 < ws["workspace_bytes"] <= fa.FA_NOALLOC_SCRATCH_BYTES
     ref = _call(fa.fa_kvcache_fwd, w, inp, cuda_device)
+    oracle_ref = run_oracle_kvcache(w, inp)
     for _ in range(2):
         got = _call(fa.fa_kvcache_fwd_noalloc, w, inp, cuda_device)
         assert fa.fa_device_status() == 0
+        check_kvcache(w, inp, got, oracle_ref)
         assert np.abs(got[0].double().numpy() - ref[0].double().numpy()).max() <= OUT_TOL[w.dtype]
         assert np.abs(got[1].double().numpy() - ref[1].double().numpy()).max() <= LSE_TOL
         assert torch.equal(got[2].view(torch.int16), ref[2].view(torch.int16))
