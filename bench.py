@@ -1,25 +1,33 @@
 #!/usr/bin/env python
 """Benchmark of the attention-with-KV-cache hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--sub LIST]
+                    [--impl ours|reference]
 
-One step = one fa_kvcache_fwd (or fa_fwd) call over one batch of seeded
-synthetic input resident in HBM: RoPE of q and the new k rows, cache
-append, and attention over cache + new rows.  The default workload is the
-GQA decode with RoPE (bf16, batch 8, 32 query / 8 kv heads, head dim 128,
-cache capacity 8192, cache_seqlens ~ U{1024..8000}, rotary_dim 64
-half-split); --config picks another.  Decode workloads report HBM GB/s of
-algorithmic bytes, prefill/dense workloads TFLOP/s of algorithmic FLOPs.
+One step = one library call over one batch of seeded synthetic input resident
+in HBM.  The default line is the headline prefill workload, MLA-like causal
+attention (bf16, batch 4, 16 heads, 4096 query and key rows, d_qk 192,
+d_v 128; flash-attention PR #1604's head dims), in TFLOP/s of algorithmic
+FLOPs against the dense bf16 tensor peak.  Beside it, under "decode", the
+line carries one sub-record per decode workload (the MLA decode over a
+16384-row cache and the GQA decode with RoPE, bf16, 32 query / 8 kv heads,
+cache_seqlens ~ U{1024..8000}), each in HBM GB/s of algorithmic bytes
+against the copy bandwidth.  --config picks another headline workload (then
+no sub-records unless --sub names some); --sub none drops them.
 
 Timing: W untimed warm-up steps, then K steps, each timed with CUDA events on
-the launching stream; the L2 is flushed (a 512 MiB write) before every timed
-step, outside the events.  Multi-GPU runs (torchrun, one rank per GPU) give
-every rank its own full copy of the workload (weak scaling, no collective on
-the data path) and report the max over ranks.
+the launching stream around a CUDA-graph replay of the call; L2 is flushed
+before every timed step, outside the events.  The roofline object divides the
+algorithmic amount by the attention kernel's own event-timed duration, and
+takes the burst peak of MEASURED_PEAKS.json for a tensor-bound kernel (each
+launch is timed alone, after an idle L2 flush); power-cap throttling seen on
+the clocks is reported beside it.  Multi-GPU runs (torchrun, one rank per
+GPU) give every rank its own full copy of the workload (weak scaling, no
+collective on the data path) and report the max over ranks.
 
 --impl reference times the float64 CPU oracle (the correctness reference of
-the tests, not tuned for speed) on a bounded sample of the same workload, on
-rank 0 only.
+the tests, not tuned for speed) on a bounded sample of the headline
+workload, on rank 0 only.
 """
 from __future__ import annotations
 
@@ -38,14 +46,16 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from rotary_embedding_b200 import workloads as W  # noqa: E402
+import workloads as W  # noqa: E402
 
 METRIC = "prefill attention TFLOP/s and decode KV-cache GB/s on 1 B200, % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # Nominal B200 figures (HGX HBM3e bandwidth; dense bf16/fp16 tensor rate, no sparsity), reported beside
 # the measured peaks as a second ceiling.
 SPEC_PEAKS = {"hbm": (7700.0, "GB/s"), "tensor": (2250.0, "TFLOP/s")}
-DEFAULT_CONFIG = "gqa-decode"
+DEFAULT_CONFIG = "mla-prefill"
+# decode workloads reported beside the default headline
+DEFAULT_SUBS = ("mla-decode", "gqa-decode")
 
 
 def parse_args(argv=None):
@@ -54,6 +64,9 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(W.CONFIGS))
+    ap.add_argument("--sub", default=None,
+                    help="comma-separated workloads reported as 'decode' sub-records ('none' for none; "
+                         "default: mla-decode,gqa-decode beside the default headline, none otherwise)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU time budget of the oracle sample (cpu_baseline / reference arm)")
@@ -419,23 +432,25 @@ def time_kernel(fa, step, steps, flush_buf):
     return times
 
 
-def run_ours(args):
-    import torch.distributed as dist
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if not torch.cuda.is_available():
-        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
-        return 1
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
-    barrier = (lambda: dist.barrier()) if world > 1 else (lambda: None)
+def sub_names(args):
+    """Workloads reported as sub-records beside the headline."""
+    if args.sub is None:
+        return list(DEFAULT_SUBS) if args.config == DEFAULT_CONFIG else []
+    if args.sub.strip().lower() in ("", "none"):
+        return []
+    names = [n.strip() for n in args.sub.split(",") if n.strip()]
+    for n in names:
+        if n not in W.CONFIGS:
+            raise SystemExit(f"--sub: unknown workload {n!r}")
+    return names
 
-    import rotary_embedding_b200 as fa
-    w = W.CONFIGS[args.config]
+
+def measure(name, args, fa, device, world, barrier, peaks, peaks_src):
+    """Time one workload: the whole call (graph replay, L2 flushed per step),
+    the attention kernel alone (library events) and the end-to-end API leg.
+    Every rank runs the same steps and the same collectives in the same order.
+    Returns (record, clocks, w, inp, amount, unit)."""
+    w = W.CONFIGS[name]
     inp = W.make_inputs(w, seed=0)
     inp_dev = {k: v.to(device) for k, v in inp.items()}
     seqlens = (inp["cache_seqlens"].tolist() if w.mode == "kvcache"
@@ -456,7 +471,7 @@ def run_ours(args):
     with torch.cuda.graph(graph, capture_error_mode="relaxed"):
         step()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(device.index) as clk:
         # untimed soak so the clock sampler sees the GPU under this load
         t_end = time.perf_counter() + 1.5
         while time.perf_counter() < t_end:
@@ -468,6 +483,9 @@ def run_ours(args):
     ms = sum(times) / len(times)
     kernel_ms = sum(k_times) / len(k_times) if k_times else None
     ms_max, value = aggregate_over_ranks(ms, amount, world, device)
+    # every rank takes part in the reduction, with -1 where its kernel events could not be timed
+    kms_max = aggregate_over_ranks(kernel_ms if kernel_ms else -1.0, amount, world, device)[0]
+    kms_max = kms_max if kms_max > 0 else None
 
     e2e_value, h2d, d2h = None, 0, 0
     if not args.no_e2e:
@@ -477,40 +495,27 @@ def run_ours(args):
         _, e2e_value = aggregate_over_ranks(e_ms, amount, world, device)
         e2e_value = round(e2e_value, 3)
 
-    peaks, peaks_src = load_peaks()
     clocks = clk.summary()
-    if bound == "hbm":
-        peak_key = "hbm_gbs"
-    else:
-        # the cuBLAS figure taken under the same conditions as this kernel: the
-        # power-capped loop when the clocks sampled during the timed region show
-        # the power cap, the burst figure otherwise
-        capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
-        peak_key = "bf16_tflops_sustained" if capped and "bf16_tflops_sustained" in peaks else "bf16_tflops"
-    peak = float(peaks.get(peak_key, FALLBACK_PEAKS.get(peak_key, FALLBACK_PEAKS["bf16_tflops"])))
+    # A tensor-bound kernel takes the burst cuBLAS figure: each launch is
+    # timed alone, after an idle L2 flush, like the burst measurement.  The
+    # power cap, when the sampled clocks show it, is reported as a note.
+    peak_key = "hbm_gbs" if bound == "hbm" else "bf16_tflops"
+    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
     # algorithmic amount of one call / the attention kernel's own duration
     # (the whole call's duration if the kernel events could not be timed)
-    achieved = amount / ((kernel_ms if kernel_ms else ms) / 1e3)
+    achieved = amount / ((kms_max if kms_max else ms_max) / 1e3)
     kernel_tag = "rotary" if w.mode == "rotary" else ("decode" if plan["path"] == fa.FA_PATH_DECODE else "prefill")
     kernel_name = {fa.FA_PATH_DECODE: "decode_kernel", fa.FA_PATH_PREFILL: "prefill2_kernel / prefill_kernel",
                    fa.FA_PATH_DENSE: "prefill2_kernel / prefill_kernel"}.get(plan["path"], "rotary_kernel")
     if w.mode == "bwd":
         kernel_tag, kernel_name = "backward", "bwd_dkdv_kernel + bwd_dq_kernel"
-
-    traffic = traffic_record(args.config, kernel_tag)
-    result = {
-        "metric": METRIC,
+    capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
+    rec = {
+        "workload": w.name,
         "value": round(value, 3),
         "unit": unit,
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": max(args.warmup, 3),
         "ms_per_step": round(ms_max, 5),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
         "dtype": w.dtype,
-        "data": "synthetic (seeded, N(0,1)/U[0,1) as the workload states)",
         "config": {"workload": w.name, "batch": w.batch, "h_q": w.h_q, "h_kv": w.h_kv,
                    "d_qk": w.d_qk, "d_v": w.d_v, "s_q": w.s_q,
                    "cap_or_s_k": w.cap if w.mode == "kvcache" else w.s_k, "causal": w.causal,
@@ -520,22 +525,74 @@ def run_ours(args):
                    "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU",
                    "plan": plan},
         "roofline": {"bound": bound, "achieved": round(achieved, 3), "peak": peak,
-                     "unit": unit, "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_source": f"{peaks_src} ({peak_key})",
+                     "unit": unit, "frac": round(achieved / peak, 4),
+                     "traffic": traffic_record(name, kernel_tag),
+                     "peak_source": f"{peaks_src} ({peak_key})" + (
+                         "; sw_power_cap active on the sampled clocks" if capped and bound != "hbm" else ""),
                      "kernel": kernel_name,
-                     "kernel_ms": round(kernel_ms, 5) if kernel_ms else None,
+                     "kernel_ms": round(kms_max, 5) if kms_max else None,
                      "timing": ("CUDA events around the kernel's launch on its stream, graph replay, "
-                                "L2 flushed per step" if kernel_ms else "whole call (kernel events unavailable)"),
-                     "call_ms": round(ms, 5),
+                                "L2 flushed per step" if kms_max else "whole call (kernel events unavailable)"),
+                     "call_ms": round(ms_max, 5),
                      "spec_peak": SPEC_PEAKS[bound][0] if bound in SPEC_PEAKS else None,
                      "frac_of_spec": (round(achieved / SPEC_PEAKS[bound][0], 4) if bound in SPEC_PEAKS else None),
                      "amount_per_launch": amount},
-        "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(plan["launches"]) * args.steps,
     }
     if clocks:
+        rec["clocks"] = clocks
+    del graph
+    return rec, clocks, w, inp, amount, unit
+
+
+def run_ours(args):
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    barrier = (lambda: dist.barrier()) if world > 1 else (lambda: None)
+
+    import rotary_embedding_b200 as fa
+    peaks, peaks_src = load_peaks()
+    subs = sub_names(args)
+    head, clocks, w, inp, _, unit = measure(args.config, args, fa, device, world, barrier, peaks, peaks_src)
+    sub_recs = {}
+    for name in subs:
+        rec = measure(name, args, fa, device, world, barrier, peaks, peaks_src)[0]
+        sub_recs[name] = rec
+
+    result = {
+        "metric": METRIC,
+        "value": head["value"],
+        "unit": head["unit"],
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded, N(0,1)/U[0,1) as the workload states)",
+        "config": head["config"],
+        "roofline": head["roofline"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"] + sum(r["gpu_launches"] for r in sub_recs.values()),
+    }
+    if clocks:
         result["clocks"] = clocks
+    if sub_recs:
+        # each decode workload with its own value, roofline (HBM) and end-to-end leg
+        result["decode"] = sub_recs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         amt, secs, desc = cpu_sample(w, inp, args.cpu_seconds)
         result["cpu_baseline"] = {"value": round(amt / secs, 6), "unit": unit, "cores": 1,
