@@ -55,6 +55,14 @@
  *  - dtype is FA_DTYPE_F16 or FA_DTYPE_BF16 and is the same for q, k, v,
  *    caches, new rows, cos/sin and out.  Head dims are multiples of 8 in
  *    8..256.
+ *  - Which kernel runs: a kvcache call with s_q <= 8 and at most 32 query
+ *    rows per kv head (g * s_q) uses the split-KV decode kernel for head
+ *    dims (d_qk, d_v) 16/16, 32/32, 64/64, 128/128, 192/128 and 256/256;
+ *    other calls use the tcgen05 prefill kernels for 64/64, 128/128,
+ *    192/128, 128/64, 64/128 and 192/64.  Every other accepted pair (for
+ *    example 16/16, 32/32, 96/96 or 256/256 outside decode) runs on a
+ *    generic CUDA-core kernel without tensor cores: same results, far
+ *    lower throughput.  fa_kvcache_plan / fa_fwd_plan report the path.
  *  - Return value: FA_OK (0) or a negative FA_ERR_* code; fa_last_error()
  *    then gives a message (thread-local, valid until the next call on the
  *    same thread).  Arguments are fully validated on the host before any
@@ -118,6 +126,10 @@ typedef struct fa_tensor {
  *   scale          softmax scale; <= 0 means 1/sqrt(d_qk)
  *   out      [b, s_q, h_q, d_v]         written
  *   lse      fp32 device array [b, h_q, s_q] (contiguous) or NULL
+ *   (These fourteen arguments, in this order, are the call the attention-
+ *   with-KV-cache contract names; what follows is this library's addition.)
+ *   cache_seqlens_scalar  the offset of every batch entry when cache_seqlens
+ *                  is NULL; ignored otherwise
  *   workspace / workspace_bytes   device scratch of at least the size that
  *                  fa_kvcache_workspace_size() reports for the same shapes
  *                  (may be NULL when that size is 0); contents on entry are
@@ -129,9 +141,10 @@ typedef struct fa_tensor {
 int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
                    const fa_tensor *k_new, const fa_tensor *v_new,
                    const fa_tensor *cos, const fa_tensor *sin,
-                   const int32_t *cache_seqlens, int32_t cache_seqlens_scalar,
+                   const int32_t *cache_seqlens,
                    int32_t rotary_dim, int32_t interleaved, int32_t causal, float scale,
                    const fa_tensor *out, float *lse,
+                   int32_t cache_seqlens_scalar,
                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
@@ -152,8 +165,12 @@ int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor
  *    are rejected with FA_ERR_WORKSPACE (fa_last_error() says how much they
  *    need); nothing is enqueued.
  *  - The first call on a device looks up the scratch array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    (cudaGetSymbolAddress) with that device current.  Under CUDA's lazy
+ *    module loading (the default) that lookup is also what loads the
+ *    array's module on the device, reserving its 32 MiB there, and it may
+ *    synchronise.  So make one call on each device as a warm-up, before the
+ *    region that must not allocate and before any stream capture; later
+ *    calls allocate nothing and do not synchronise.
  *  - No cudaMalloc, cudaFree or other allocating routine is called.
  *  - Every call on a device shares the one scratch array: calls whose work
  *    overlaps on the GPU (different streams, or another thread) race on it
@@ -165,9 +182,10 @@ int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor
 int fa_kvcache_fwd_noalloc(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
                            const fa_tensor *k_new, const fa_tensor *v_new,
                            const fa_tensor *cos, const fa_tensor *sin,
-                           const int32_t *cache_seqlens, int32_t cache_seqlens_scalar,
+                           const int32_t *cache_seqlens,
                            int32_t rotary_dim, int32_t interleaved, int32_t causal, float scale,
-                           const fa_tensor *out, float *lse, void *stream);
+                           const fa_tensor *out, float *lse,
+                           int32_t cache_seqlens_scalar, void *stream);
 
 /* Workspace bytes fa_kvcache_fwd needs for these shapes (k_new may be NULL). */
 int fa_kvcache_workspace_size(const fa_tensor *q, const fa_tensor *k_cache,
@@ -198,10 +216,11 @@ int fa_fwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
 int fa_kvcache_fwd_window(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
                           const fa_tensor *k_new, const fa_tensor *v_new,
                           const fa_tensor *cos, const fa_tensor *sin,
-                          const int32_t *cache_seqlens, int32_t cache_seqlens_scalar,
+                          const int32_t *cache_seqlens,
                           int32_t rotary_dim, int32_t interleaved, int32_t causal,
                           int32_t window_left, int32_t window_right, float scale,
                           const fa_tensor *out, float *lse,
+                          int32_t cache_seqlens_scalar,
                           void *workspace, size_t workspace_bytes, void *stream);
 int fa_fwd_window(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
                   int32_t causal, int32_t window_left, int32_t window_right, float scale,

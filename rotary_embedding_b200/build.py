@@ -1,6 +1,8 @@
 """Build libfa.so in-tree from csrc/*.cu for sm_100a with nvcc.
 
-    python -m rotary_embedding_b200.build [--force] [--jobs N]
+    python rotary_embedding_b200/build.py [--force] [--jobs N]
+
+(run as a script: importing the package loads libfa.so, which this builds)
 
 Objects go to rotary_embedding_b200/_build/; the shared library is written
 next to this file so that it travels with the source tree.

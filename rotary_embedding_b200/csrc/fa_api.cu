@@ -23,6 +23,7 @@
 
 #include "fa.h"
 #include "fa_internal.h"
+#include "fa_testing.h"
 
 namespace fa {
 
@@ -32,6 +33,9 @@ __device__ int32_t g_status_word = 0;
 namespace {
 
 thread_local char g_last_error[512] = "";
+
+// Query tiles per CTA forced by fa_testing_set_prefill_tiles (0: the planner decides).
+int g_forced_tiles = 0;
 
 int fail(int code, const char *fmt, ...) {
     va_list ap;
@@ -221,12 +225,8 @@ int run_tc_attention(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
     const int64_t ctas2 = (int64_t)((p.n_q_tiles + 1) / 2) * (h_q / pack) * b;
     const int64_t sms = sm_count();
     p.tiles_per_cta = (ctas2 >= 2 * sms || (d_qk <= 64 && 2 * ctas2 >= sms)) ? 2 : 1;
-    // FA_PREFILL_TILES_PER_CTA=1|2 overrides the choice (tests use it to run
-    // both kernels on small shapes)
-    if (const char *env = getenv("FA_PREFILL_TILES_PER_CTA")) {
-        if (env[0] == '1') p.tiles_per_cta = 1;
-        if (env[0] == '2') p.tiles_per_cta = 2;
-    }
+    // a test may pin the kernel (fa_testing_set_prefill_tiles)
+    if (g_forced_tiles) p.tiles_per_cta = g_forced_tiles;
     // Under a causal mask the work of query tile t grows with t.  When the
     // two-tile grid is one wave, the slowest CTA sets the time, so pair tile
     // k with tile n-1-k (every CTA then sees about the same number of key
@@ -441,6 +441,12 @@ int fa_rotary(const fa_tensor *x, const fa_tensor *cos, const fa_tensor *sin,
     return FA_OK;
 }
 
+int fa_testing_set_prefill_tiles(int32_t tiles) {
+    if (tiles < 0 || tiles > 2) return fail(FA_ERR_INVALID_ARG, "prefill tiles per CTA must be 0, 1 or 2");
+    g_forced_tiles = tiles;
+    return FA_OK;
+}
+
 int fa_set_kernel_events(void *start, void *stop) {
     if ((start == nullptr) != (stop == nullptr))
         return fail(FA_ERR_INVALID_ARG, "fa_set_kernel_events: pass both events or neither");
@@ -520,21 +526,20 @@ int fa_fwd_plan(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, fa_p
 
 int fa_kvcache_fwd(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
                    const fa_tensor *k_new, const fa_tensor *v_new, const fa_tensor *cos,
-                   const fa_tensor *sin, const int32_t *cache_seqlens, int32_t cache_seqlens_scalar,
-                   int32_t rotary_dim, int32_t interleaved, int32_t causal, float scale,
-                   const fa_tensor *out, float *lse, void *workspace, size_t workspace_bytes,
-                   void *stream) {
-    return fa_kvcache_fwd_window(q, k_cache, v_cache, k_new, v_new, cos, sin, cache_seqlens,
-                                 cache_seqlens_scalar, rotary_dim, interleaved, causal, -1, -1, scale, out, lse,
-                                 workspace, workspace_bytes, stream);
+                   const fa_tensor *sin, const int32_t *cache_seqlens, int32_t rotary_dim,
+                   int32_t interleaved, int32_t causal, float scale, const fa_tensor *out, float *lse,
+                   int32_t cache_seqlens_scalar, void *workspace, size_t workspace_bytes, void *stream) {
+    return fa_kvcache_fwd_window(q, k_cache, v_cache, k_new, v_new, cos, sin, cache_seqlens, rotary_dim,
+                                 interleaved, causal, -1, -1, scale, out, lse, cache_seqlens_scalar, workspace,
+                                 workspace_bytes, stream);
 }
 
 int fa_kvcache_fwd_window(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
                           const fa_tensor *k_new, const fa_tensor *v_new, const fa_tensor *cos,
-                          const fa_tensor *sin, const int32_t *cache_seqlens, int32_t cache_seqlens_scalar,
-                          int32_t rotary_dim, int32_t interleaved, int32_t causal, int32_t window_left,
-                          int32_t window_right, float scale, const fa_tensor *out, float *lse, void *workspace,
-                          size_t workspace_bytes, void *stream) {
+                          const fa_tensor *sin, const int32_t *cache_seqlens, int32_t rotary_dim,
+                          int32_t interleaved, int32_t causal, int32_t window_left, int32_t window_right,
+                          float scale, const fa_tensor *out, float *lse, int32_t cache_seqlens_scalar,
+                          void *workspace, size_t workspace_bytes, void *stream) {
     g_last_error[0] = 0;
     if (window_left < -1 || window_right < -1)
         return fail(FA_ERR_INVALID_ARG, "window bounds must be >= -1 (-1 = unbounded)");

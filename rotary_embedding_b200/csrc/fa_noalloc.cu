@@ -53,9 +53,9 @@ void *scratch_address(int *status) {
 
 extern "C" int fa_kvcache_fwd_noalloc(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
                                       const fa_tensor *k_new, const fa_tensor *v_new, const fa_tensor *cos,
-                                      const fa_tensor *sin, const int32_t *cache_seqlens,
-                                      int32_t cache_seqlens_scalar, int32_t rotary_dim, int32_t interleaved,
-                                      int32_t causal, float scale, const fa_tensor *out, float *lse, void *stream) {
+                                      const fa_tensor *sin, const int32_t *cache_seqlens, int32_t rotary_dim,
+                                      int32_t interleaved, int32_t causal, float scale, const fa_tensor *out,
+                                      float *lse, int32_t cache_seqlens_scalar, void *stream) {
     size_t need = 0;
     int rc = fa_kvcache_workspace_size(q, k_cache, v_cache, k_new, cos ? rotary_dim : 0, &need);
     if (rc != FA_OK) return rc;
@@ -70,6 +70,6 @@ extern "C" int fa_kvcache_fwd_noalloc(const fa_tensor *q, const fa_tensor *k_cac
     if (!scratch) return st;
     // The scratch keeps whatever the previous call left in it; the kernels
     // write every scratch word before they read it, so nothing is cleared.
-    return fa_kvcache_fwd(q, k_cache, v_cache, k_new, v_new, cos, sin, cache_seqlens, cache_seqlens_scalar,
-                          rotary_dim, interleaved, causal, scale, out, lse, scratch, kScratchBytes, stream);
+    return fa_kvcache_fwd(q, k_cache, v_cache, k_new, v_new, cos, sin, cache_seqlens, rotary_dim, interleaved,
+                          causal, scale, out, lse, cache_seqlens_scalar, scratch, kScratchBytes, stream);
 }

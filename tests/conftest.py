@@ -21,3 +21,13 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(params=[1, 2], ids=["1tile", "2tiles"])
+def prefill_tiles(request):
+    """Run the test with the one-tile and with the two-tile tcgen05 prefill
+    kernel (pinned through the library's test hook, released afterwards)."""
+    import rotary_embedding_b200 as fa
+    fa.fa_testing_set_prefill_tiles(request.param)
+    yield request.param
+    fa.fa_testing_set_prefill_tiles(0)

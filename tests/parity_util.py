@@ -14,7 +14,7 @@ import torch
 
 import oracle
 import rotary_embedding_b200 as fa
-from rotary_embedding_b200 import workloads as W
+import workloads as W
 
 OUT_TOL = {"fp16": 2e-3, "bf16": 1.6e-2}
 LSE_TOL = 1e-3

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import rotary_embedding_b200 as fa
-from rotary_embedding_b200 import workloads as W
+import workloads as W
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -56,7 +56,7 @@ def _call(q, kc, vc, kn, vn, out, cos=None, sin=None, seq=0, rotary_dim=0, ws=No
     d = fa.describe
     r = lambda t: ctypes.byref(t) if t is not None else None  # noqa: E731
     return fa.lib.fa_kvcache_fwd(r(d(q)), r(d(kc)), r(d(vc)), r(d(kn)), r(d(vn)), r(d(cos)),
-                                 r(d(sin)), None, seq, rotary_dim, 0, 1, 0.0, r(d(out)), None,
+                                 r(d(sin)), None, rotary_dim, 0, 1, 0.0, r(d(out)), None, seq,
                                  ws, ws_bytes, None)
 
 
@@ -179,3 +179,26 @@ def test_kernel_events_hook_arguments():
     assert fa.lib.fa_set_kernel_events(ctypes.c_void_p(16), None) == fa.FA_ERR_INVALID_ARG
     assert fa.lib.fa_set_kernel_events(None, ctypes.c_void_p(16)) == fa.FA_ERR_INVALID_ARG
     assert fa.lib.fa_set_kernel_events(None, None) == fa.FA_OK
+
+
+def test_binding_rejects_host_tensors():
+    """The C ABI takes raw device addresses and cannot tell a host pointer from
+    a device one, so the binding refuses CPU tensors (and tensors on another
+    device than q) before anything is enqueued."""
+    q, kc, vc, kn, vn, out = _kv_tensors()
+    seq = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        fa.fa_kvcache_fwd(q, kc, vc, kn, vn, cache_seqlens=seq, causal=True)
+    with pytest.raises(ValueError, match="CUDA"):
+        fa.fa_kvcache_fwd_noalloc(q, kc, vc, kn, vn, cache_seqlens=3, causal=True)
+    with pytest.raises(ValueError, match="CUDA"):
+        fa.fa_fwd(q, kc, vc, causal=True)
+    cos = torch.zeros(16, 32, dtype=torch.float16)
+    with pytest.raises(ValueError, match="CUDA"):
+        fa.fa_rotary(q, cos, cos.clone(), 0)
+    cu = torch.tensor([0, 3], dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        fa.fa_fwd_varlen(q[0], kc[0], vc[0], cu, cu, 3)
+    lse = torch.zeros(2, 4, 3)
+    with pytest.raises(ValueError, match="CUDA"):
+        fa.fa_bwd(q, kc[:, :3], vc[:, :3], out, out, lse)

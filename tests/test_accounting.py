@@ -3,7 +3,7 @@ visible (query, key) pairs, FLOPs and bytes, checked on small shapes against
 brute-force enumeration of the mask's definition (CPU only)."""
 import pytest
 
-from rotary_embedding_b200 import workloads as W
+import workloads as W
 
 
 def _brute_pairs(s_q, N, causal, window):

@@ -20,7 +20,7 @@ import torch
 
 import oracle
 import rotary_embedding_b200 as fa
-from rotary_embedding_b200 import workloads as W
+import workloads as W
 
 DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
 TOL = {"bf16": 2e-2, "fp16": 3e-3}

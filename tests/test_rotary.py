@@ -10,7 +10,7 @@ import torch
 
 import oracle
 import rotary_embedding_b200 as fa
-from rotary_embedding_b200 import workloads as W
+import workloads as W
 from parity_util import ulp_distance
 
 DT = {"fp16": torch.float16, "bf16": torch.bfloat16}

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import rotary_embedding_b200 as fa
-from rotary_embedding_b200 import workloads as W
+import workloads as W
 from parity_util import LSE_TOL, OUT_TOL
 
 DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
@@ -49,11 +49,9 @@ def _check(out, lse, r_out, r_lse, dtype):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("tiles", ["1", "2"])
 @pytest.mark.parametrize("dims", [(64, 64), (128, 128), (192, 128)])
 @pytest.mark.parametrize("causal,window", [(True, (-1, -1)), (False, (-1, -1)), (True, (90, -1))])
-def test_varlen_parity(cuda_device, monkeypatch, tiles, dims, causal, window):
-    monkeypatch.setenv("FA_PREFILL_TILES_PER_CTA", tiles)
+def test_varlen_parity(cuda_device, prefill_tiles, dims, causal, window):
     lens_q = [130, 1, 0, 300, 64, 257]
     lens_k = [200, 77, 5, 300, 64, 257]      # s_k >= s_q (bottom-right), a key-only sequence
     q, k, v, cq, ck = _case(7, lens_q, lens_k, 8, 2, dims[0], dims[1], "bf16")

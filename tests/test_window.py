@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import rotary_embedding_b200 as fa
-from rotary_embedding_b200 import workloads as W
+import workloads as W
 from parity_util import LSE_TOL, OUT_TOL, ulp_distance
 
 DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
@@ -28,16 +28,14 @@ def _check(out, lse, r_out, r_lse, dtype):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("tiles", ["1", "2"])
 @pytest.mark.parametrize("dims", [(64, 64), (128, 128), (192, 128)])
 @pytest.mark.parametrize("causal,window", [(True, (100, -1)), (True, (0, -1)), (False, (40, 40)),
                                            (False, (0, 0)), (False, (-1, 60)), (True, (5000, -1)),
                                            (False, (300, -1))])
-def test_dense_window(cuda_device, monkeypatch, tiles, dims, causal, window):
-    monkeypatch.setenv("FA_PREFILL_TILES_PER_CTA", tiles)
+def test_dense_window(cuda_device, prefill_tiles, dims, causal, window):
     d_qk, d_v = dims
     dtype = "bf16"
-    g = torch.Generator().manual_seed(hash((tiles, dims, causal, window)) % 1000)
+    g = torch.Generator().manual_seed(hash((prefill_tiles, dims, causal, window)) % 1000)
     b, s_q, s_k, h_q, h_kv = 2, 300, 700, 4, 2
     q = _draw(g, (b, s_q, h_q, d_qk), dtype)
     k = _draw(g, (b, s_k, h_kv, d_qk), dtype)
