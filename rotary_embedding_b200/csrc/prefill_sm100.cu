@@ -35,12 +35,33 @@ namespace fa {
 
 // Pairs out of every 8 whose 2^x the two-tile softmax evaluates on the FMA
 // pipe (ex2_poly2) instead of the special function unit, in unmasked tiles.
+// At d_qk <= 64 a key tile's scores cost little tensor time next to their
+// exponentials and the special function unit bounds the softmax, so 3 of 8
+// pairs move; at larger d_qk that unit has room and the polynomial's extra
+// instructions only lengthen the softmax (measured: d_qk 192 3 % faster with
+// none, d_qk 64 equal or slower with fewer).
 #ifndef FA_EXP2_EMU_PAIRS
 #define FA_EXP2_EMU_PAIRS 3
 #endif
+template <int D_QK>
+constexpr int exp2_emu_pairs() { return D_QK <= 64 ? FA_EXP2_EMU_PAIRS : 0; }
 
 constexpr int kBM = 128;  // query rows per CTA
 constexpr int kBN = 128;  // key rows per tile
+
+// The grid is one-dimensional over (tile index, head group, batch entry) with
+// the tile index slowest and taken from the last: under a causal mask the
+// work of a query tile grows with its index, so every head's and batch
+// entry's heaviest tiles start first and the light ones fill the last wave.
+__device__ __forceinline__ void grid_order(const PrefillParams &p, int &tile, int &hgrp, int &b) {
+    const int nhg = p.h_q / p.pack;
+    const int per = nhg * p.b;                         // blocks per tile index
+    const int L = (int)blockIdx.x;
+    const int t = L / per, rem = L - t * per;
+    tile = (int)gridDim.x / per - 1 - t;
+    hgrp = rem % nhg;
+    b = rem / nhg;
+}
 
 template <int D_QK, int D_V>
 struct PrefillCfg {
@@ -84,15 +105,17 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pv_done + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = (int)gridDim.x - 1 - (int)blockIdx.x;   // heaviest causal tiles first
-    const int hgrp = blockIdx.y, b = blockIdx.z;
+    // heaviest causal tiles first across every head and batch entry: block L
+    // takes tile n - 1 - L / (head groups x batch)
+    int qt, hgrp, b;
+    grid_order(p, qt, hgrp, b);
     const int pack = p.pack;
     const int hq0 = hgrp * pack;                           // first query head of the tile
     const int hk = hq0 / p.g;
     const int i0 = qt * (kBM / pack);                      // first query position
 
     // keys N, query rows sq of this CTA's sequence, and the row offsets of a
-    // packed (varlen) sequence: blockIdx.z is then the sequence, whose rows
+    // packed (varlen) sequence: b is then the sequence, whose rows
     // qoff .. and koff .. sit in batch entry 0 of the packed tensors
     int N, sq = p.s_q, qoff = 0, koff = 0, tb = b;
     if (p.cu_q) {
@@ -104,13 +127,13 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
         // device-side preconditions: the sequence lies inside the packed rows
         if (qoff < 0 || sq < 0 || (int64_t)qoff + sq > p.total_q || koff < 0 || N < 0 ||
             (int64_t)koff + N > p.total_k) {
-            if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
+            if (threadIdx.x == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
             return;
         }
     } else if (p.kvcache) {
         const int L = seqlen_of(p.seqlens, p.seqlen_scalar, b);
         if (L < 0 || (int64_t)L + p.s_new > p.cap) {
-            if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
+            if (threadIdx.x == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
             return;
         }
         N = L + p.s_new;
@@ -386,30 +409,33 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
 // ============================================================================
 // Two query tiles per CTA (256 query rows), two softmax warpgroups.
 //
-// The tensor core alternates between the tiles: while warpgroup A turns S_A
-// into P_A, it runs PV_B(j-1) and QK_B(j), and the other way round:
-//   QK_A(0) QK_B(0) | PV_A(0) QK_A(1) | PV_B(0) QK_B(1) | PV_A(1) QK_A(2) | ...
-// Each tile has one TMEM S buffer; P is written over the first 64 columns of
-// it as 16-bit pairs and read from there as the A operand of PV.  The next
-// QK of the same tile is issued after that PV by the same thread, and the
-// tensor pipe executes one thread's MMAs in issue order, so the PV reads P
-// before the QK overwrites it.  When softmax X sees S_X(j) complete, every
-// earlier MMA of the CTA has completed too, so O_X is stable and can be
-// rescaled without a further wait.
-// Warps: 0 TMA, 1 MMA, 2-3 idle (warpgroup 0), 4-7 softmax of tile A
-// (warpgroup 1), 8-11 softmax of tile B (warpgroup 2); warp w reaches TMEM
+// Each tile x has its own S buffer, its own P buffer and its own O
+// accumulator in TMEM, so the tensor core never waits for a softmax to hand
+// back S: as soon as softmax warpgroup x has loaded S_x(j) into registers
+// (s_free), the MMA warp issues QK_x(j+1) into the same S buffer, and the
+// tensor core computes the next scores while the softmax turns the current
+// ones into P.  Per key tile j the MMA warp issues, in order,
+//   QK_0(j+1)  QK_1(j+1)  PV_0(j)  PV_1(j)
+// each after its operands are ready (K(j+1) loaded and S_x(j) consumed; V(j)
+// loaded and P_x(j) written).  PV_x(j) commits pv_done[x]; the softmax waits
+// for it before writing P_x(j+1) over P_x(j) or rescaling O_x, and before the
+// epilogue reads O_x.
+//
+// TMEM columns (512): S_x at x BN, P_x (16-bit pairs, BN/2 columns) after
+// both S buffers, O_x in the last 2 d_v columns.  That fits with BN = 128
+// key rows when d_v <= 64 and with BN = 80 otherwise (3 BN + 2 d_v <= 512).
+//
+// Warps: 0 TMA, 1 MMA, 2-3 idle (warpgroup 0), 4-7 softmax of tile 0
+// (warpgroup 1), 8-11 softmax of tile 1 (warpgroup 2); warp w reaches TMEM
 // lanes 32 (w % 4) .. 32 (w % 4) + 31.  The register file is split with
-// setmaxnreg: warpgroup 0 drops to 96 registers per thread (the MMA issue loop
-// must not spill), the two softmax warpgroups rise to 200 so that a whole
-// 128-column S row stays in registers (128 x 96 + 256 x 200 = 63488, within
-// the 384 x 168 the block is launched with).
+// setmaxnreg: warpgroup 0 drops to 64 registers per thread (enough for the
+// TMA and MMA issue loops), the two softmax warpgroups rise to 216 so that a
+// whole S row stays in registers (128 x 64 + 256 x 216 = 63488, within the
+// 384 x 168 the block is launched with).
 // ============================================================================
 template <int D_QK, int D_V>
 struct Prefill2Cfg {
-    // Key rows per tile: 128, or 96 for d_qk > 128 so that K and V both stay
-    // double-buffered next to the two Q tiles (a single V buffer would expose
-    // every V load in full).
-    static constexpr int BN = D_QK > 128 ? 96 : 128;
+    static constexpr int BN = D_V <= 64 ? 128 : 80;  // key rows per tile
     static constexpr int QBYTES = kBM * D_QK * 2;   // per tile
     static constexpr int KBYTES = BN * D_QK * 2;
     static constexpr int VBYTES = BN * D_V * 2;
@@ -422,9 +448,12 @@ struct Prefill2Cfg {
     static constexpr int KST = EVEN ? (KS_RAW > 3 ? 3 : KS_RAW) : 2;
     static constexpr int VST = EVEN ? KST : (AVAIL - 2 * KBYTES) / VBYTES;
     static constexpr int SMEM = 1024 + 2 * QBYTES + KST * KBYTES + VST * VBYTES + 256;
-    // TMEM columns: S of tile x at [128 x, 128 x + 128), O of tile x at [256 + 128 x, ...)
-    static __device__ __forceinline__ uint32_t t_s(int x) { return (uint32_t)(x * 128); }
-    static __device__ __forceinline__ uint32_t t_o(int x) { return (uint32_t)(256 + x * 128); }
+    static constexpr int PCOLS = ((BN / 2) + 15) / 16 * 16;   // P columns per tile, 16-aligned
+    static __device__ __forceinline__ uint32_t t_s(int x) { return (uint32_t)(x * BN); }
+    static __device__ __forceinline__ uint32_t t_p(int x) { return (uint32_t)(2 * BN + x * PCOLS); }
+    static __device__ __forceinline__ uint32_t t_o(int x) { return (uint32_t)(512 - 2 * D_V + x * D_V); }
+    static_assert(2 * BN + 2 * PCOLS <= 512 - 2 * D_V, "TMEM: S, P and O of both tiles");
+    static_assert(BN % 16 == 0 && KBOX % 1024 == 0, "key tile rows");
     static_assert(VST >= 1 && KST >= 2, "K/V ring");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
     static_assert(D_QK % 64 == 0 && D_V % 64 == 0 && D_V <= 128, "head dims");
@@ -448,21 +477,23 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
     uint64_t *k_empty = k_full + KST;       // KST
     uint64_t *v_full = k_empty + KST;       // VST
     uint64_t *v_empty = v_full + VST;       // VST
-    uint64_t *s_full = v_empty + VST;       // 2
-    uint64_t *p_full = s_full + 2;          // 2
-    uint64_t *o_full = p_full + 2;          // 2
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_full + 2);
+    uint64_t *s_full = v_empty + VST;       // 2: QK_x(j) complete
+    uint64_t *s_free = s_full + 2;          // 2: softmax x holds S_x(j) in registers
+    uint64_t *p_full = s_free + 2;          // 2: P_x(j) written
+    uint64_t *pv_done = p_full + 2;         // 2: PV_x(j) complete
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pv_done + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int blk = (int)gridDim.x - 1 - (int)blockIdx.x;   // heaviest causal blocks first
-    const int hgrp = blockIdx.y, b = blockIdx.z;
+    // heaviest causal blocks first across every head and batch entry
+    int blk, hgrp, b;
+    grid_order(p, blk, hgrp, b);
     const int pack = p.pack;
     const int hq0 = hgrp * pack;
     const int hk = hq0 / p.g;
     const int rows_per_tile = kBM / pack;                   // query positions per tile
 
     // keys N, query rows sq of this CTA's sequence, and the row offsets of a
-    // packed (varlen) sequence: blockIdx.z is then the sequence, whose rows
+    // packed (varlen) sequence: b is then the sequence, whose rows
     // qoff .. and koff .. sit in batch entry 0 of the packed tensors
     int N, sq = p.s_q, qoff = 0, koff = 0, tb = b;
     if (p.cu_q) {
@@ -474,13 +505,13 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         // device-side preconditions: the sequence lies inside the packed rows
         if (qoff < 0 || sq < 0 || (int64_t)qoff + sq > p.total_q || koff < 0 || N < 0 ||
             (int64_t)koff + N > p.total_k) {
-            if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
+            if (threadIdx.x == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
             return;
         }
     } else if (p.kvcache) {
         const int L = seqlen_of(p.seqlens, p.seqlen_scalar, b);
         if (L < 0 || (int64_t)L + p.s_new > p.cap) {
-            if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
+            if (threadIdx.x == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
             return;
         }
         N = L + p.s_new;
@@ -532,8 +563,9 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(&s_full[x], 1);
+            mbar_init(&s_free[x], 4);
             mbar_init(&p_full[x], 4);
-            mbar_init(&o_full[x], 1);
+            mbar_init(&pv_done[x], 1);
         }
         fence_barrier_init();
     }
@@ -547,7 +579,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
 
-    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
+    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0 && n_all > kb0) {
@@ -590,6 +622,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             const uint64_t dK0 = tc::smem_desc(smem_addr(sK), 16, 1024);
             const uint64_t dV0 = tc::smem_desc(smem_addr(sV), C::KBOX, 1024);
             bool ok = mbar_wait(q_full, 0, p.status);
+            auto in_range = [&](int x, int j) { return j >= kb[x] && j < n_kv[x]; };
             // key tile j sits in stage (j - kb0) % KST / VST
             auto issue_qk = [&](int x, int j) {
                 const uint64_t dq = dQ0 + (uint64_t)((x * C::QBYTES) >> 4);
@@ -608,12 +641,13 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             };
             auto issue_pv = [&](int x, int j) {
                 const uint64_t dv = dV0 + (uint64_t)((((j - kb0) % VST) * C::VBYTES) >> 4);
-                const uint32_t to = tmem + C::t_o(x), tp = tmem + C::t_s(x);
+                const uint32_t to = tmem + C::t_o(x), tp = tmem + C::t_p(x);
                 const uint32_t acc0 = j > kb[x] ? 1u : 0u;
                 if (leader) {
 #pragma unroll
                     for (int k = 0; k < BN / 16; ++k)
                         tc::mma_ts(to, tp + k * 8, dv + (uint64_t)(k * 16 * 128 / 16), idesc_pv, k > 0 ? 1u : acc0);
+                    tc::commit(&pv_done[x]);
                 }
                 __syncwarp();
             };
@@ -624,37 +658,44 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             // prologue: QK of the tiles whose range starts at the first loaded key tile
             if (ok && (ok = mbar_wait(&k_full[0], 0, p.status))) {
                 tc::fence_after_sync();
-                if (any0 && kb[0] == kb0) issue_qk(0, kb0);
-                if (any1 && kb[1] == kb0) issue_qk(1, kb0);
+                if (in_range(0, kb0)) issue_qk(0, kb0);
+                if (in_range(1, kb0)) issue_qk(1, kb0);
                 commit(&k_empty[0]);
             }
             for (int j = kb0; j < n_all && ok; ++j) {
                 const int u = j - kb0;
-                const int vs = u % VST;
                 const bool next = j + 1 < n_all;
-                const int ks1 = (u + 1) % KST;
+                // the next scores: QK_x(j+1) once K(j+1) is in and S_x(j) is consumed
+                if (next) {
+                    const int ks1 = (u + 1) % KST;
+                    if (!(ok = mbar_wait(&k_full[ks1], ((u + 1) / KST) & 1, p.status))) break;
+#pragma unroll
+                    for (int x = 0; x < 2; ++x) {
+                        if (!in_range(x, j + 1)) continue;
+                        if (in_range(x, j) && !(ok = mbar_wait(&s_free[x], (j - kb[x]) & 1, p.status))) break;
+                        tc::fence_after_sync();
+                        issue_qk(x, j + 1);
+                    }
+                    if (!ok) break;
+                    commit(&k_empty[ks1]);
+                }
+                // this tile's PV: P_x(j) V(j) once V(j) is in and P_x(j) is written
+                const int vs = u % VST;
                 if (!(ok = mbar_wait(&v_full[vs], (u / VST) & 1, p.status))) break;
-                if (next && !(ok = mbar_wait(&k_full[ks1], ((u + 1) / KST) & 1, p.status))) break;
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    if (j >= kb[x] && j < n_kv[x]) {
-                        if (!(ok = mbar_wait(&p_full[x], (j - kb[x]) & 1, p.status))) break;
-                        tc::fence_after_sync();
-                        issue_pv(x, j);
-                        if (j + 1 == n_kv[x]) commit(&o_full[x]);
-                        if (j + 1 < n_kv[x]) issue_qk(x, j + 1);
-                    } else if (j + 1 == kb[x] && kb[x] < n_kv[x]) {
-                        issue_qk(x, j + 1);   // this tile's range starts at the next key tile
-                    }
+                    if (!in_range(x, j)) continue;
+                    if (!(ok = mbar_wait(&p_full[x], (j - kb[x]) & 1, p.status))) break;
+                    tc::fence_after_sync();
+                    issue_pv(x, j);
                 }
                 if (!ok) break;
                 commit(&v_empty[vs]);
-                if (next) commit(&k_empty[ks1]);
             }
         }
     } else if (warp >= 4) {
         // ------------------------------------------------ softmax warpgroups
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 216;" ::: "memory");
         const int x = (warp - 4) >> 2;                 // tile of this warpgroup
         const int q4 = warp & 3;                       // TMEM lane quadrant this warp may access
         const int r = q4 * 32 + lane;                  // tile row = TMEM lane
@@ -670,20 +711,29 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         const float c = p.scale_log2;
         const uint64_t c2 = f2_pack(c, c);
         const uint32_t s_addr = tmem + lane_addr + C::t_s(x);
+        const uint32_t p_addr = tmem + lane_addr + C::t_p(x);
         const uint32_t o_addr = tmem + lane_addr + C::t_o(x);
-        const int nk = n_kv[x], jb = kb[x];
+        const int nk = n_kv[x], jb = kb[x], mfrom = mask_from[x], lmax = lo_max[x];
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = jb; j < nk && ok; ++j) {
             if (!(ok = mbar_wait(&s_full[x], (j - jb) & 1, p.status))) break;
             tc::fence_after_sync();
             const int j0 = j * BN;
-            constexpr int NCH = BN / 32;               // 32-column chunks of the S row
+            // the S row: NCH chunks of 32 columns and, when BN % 32 = 16, a
+            // 16-column tail (every index below is a compile-time constant)
+            constexpr int NCH = BN / 32, TAIL = BN % 32;
             uint32_t sr[NCH][32];
+            uint32_t st[TAIL > 0 ? TAIL : 2];
 #pragma unroll
             for (int h = 0; h < NCH; ++h) tc::ld32(s_addr + h * 32, sr[h]);
+            if constexpr (TAIL == 16) tc::ld16(s_addr + NCH * 32, st);
             tc::wait_ld();
-            const bool masked = j0 + BN > mask_from[x] || j0 < lo_max[x];
+            // S_x(j) is in registers: the MMA warp may compute S_x(j+1) over it
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[x]);
+            const bool masked = j0 + BN > mfrom || j0 < lmax;
             if (masked) {
                 // diagonal band, window edge or sequence end: -inf outside the
                 // visible keys (only these tiles pay for the comparisons)
@@ -691,22 +741,26 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                 for (int h = 0; h < NCH; ++h)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        const int key = j0 + h * 32 + e;
+                        const int key = j0 + 32 * h + e;
                         if (key > last_vis || key < first_vis) sr[h][e] = __float_as_uint(-INFINITY);
                     }
-            }
-            // row max: one independent three-input chain per chunk
-            float mx[NCH];
 #pragma unroll
-            for (int h = 0; h < NCH; ++h) {
-                mx[h] = -INFINITY;
+                for (int e = 0; e < TAIL; ++e) {
+                    const int key = j0 + 32 * NCH + e;
+                    if (key > last_vis || key < first_vis) st[e] = __float_as_uint(-INFINITY);
+                }
+            }
+            // row max: four independent three-input chains
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int h = 0; h < NCH; ++h)
 #pragma unroll
                 for (int e = 0; e < 32; e += 2)
-                    mx[h] = fmax3(mx[h], __uint_as_float(sr[h][e]), __uint_as_float(sr[h][e + 1]));
-            }
-            float mt = mx[0];
+                    mx[(e >> 1) & 3] = fmax3(mx[(e >> 1) & 3], __uint_as_float(sr[h][e]), __uint_as_float(sr[h][e + 1]));
 #pragma unroll
-            for (int h = 1; h < NCH; ++h) mt = fmaxf(mt, mx[h]);
+            for (int e = 0; e < TAIL; e += 2)
+                mx[(e >> 1) & 3] = fmax3(mx[(e >> 1) & 3], __uint_as_float(st[e]), __uint_as_float(st[e + 1]));
+            const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             float alpha = 1.f;
             bool rescale = false;
             if (mt > m_ref && (m_ref == -INFINITY || (mt - m_ref) * c > 8.f)) {
@@ -716,42 +770,11 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             }
             const float mc = m_ref == -INFINITY ? 0.f : m_ref * c;
             const uint64_t nmc2 = f2_pack(-mc, -mc);
-            // P = 2^(s c - m c), written as 16-bit pairs over the first BN/2
-            // columns of the S buffer (keys [32h, 32h+32) -> columns [16h, 16h+16),
-            // all of which were read above)
-            // In tiles without masked keys, 6 of every 16 pairs take 2^x on the
-            // FMA pipe (ex2_poly2) and the rest on the special function unit,
-            // which alone would bound the softmax; masked tiles need exact
-            // zeros and use the special function unit throughout.
-            // The fp32 P values overwrite S in registers; the row sum is taken
-            // after P has been handed to the MMA warp (off the critical path).
-            auto exp_row = [&](auto split) {
-#pragma unroll
-                for (int h = 0; h < NCH; ++h) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const uint64_t t =
-                            f2_fma(f2_pack(__uint_as_float(sr[h][e]), __uint_as_float(sr[h][e + 1])), c2, nmc2);
-                        float t0, t1, p0, p1;
-                        f2_unpack(t, t0, t1);
-                        if (decltype(split)::value && ((e >> 1) & 7) < FA_EXP2_EMU_PAIRS) {
-                            f2_unpack(ex2_poly2(t0, t1), p0, p1);
-                        } else {
-                            p0 = ex2(t0);
-                            p1 = ex2(t1);
-                        }
-                        sr[h][e] = __float_as_uint(p0);
-                        sr[h][e + 1] = __float_as_uint(p1);
-                        pk[e >> 1] = Elem<T>::pack2(p0, p1);
-                    }
-                    tc::st16(s_addr + h * 16, pk);
-                }
-            };
-            if (masked)
-                exp_row(std::integral_constant<bool, false>());
-            else
-                exp_row(std::integral_constant<bool, true>());
+            // P_x(j-1) has been read and O_x updated by PV_x(j-1)
+            if (j > jb) {
+                if (!(ok = mbar_wait(&pv_done[x], (j - 1 - jb) & 1, p.status))) break;
+                tc::fence_after_sync();
+            }
             if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
                 for (int h = 0; h < D_V / 32; ++h) {
@@ -763,6 +786,48 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                     tc::st32(o_addr + h * 32, orr);
                 }
             }
+            // P = 2^(s c - m c) as 16-bit pairs into the P buffer (keys
+            // [2k, 2k+2) -> column k).  In tiles without masked keys and at
+            // d_qk <= 64, 3 of every 8 pairs take 2^x on the FMA pipe
+            // (ex2_poly2) and the rest on the special function unit
+            // (exp2_emu_pairs); masked tiles need exact zeros and use the
+            // special function unit throughout.  The fp32 P values overwrite S
+            // in registers; the row sum is taken after P has been handed to
+            // the MMA warp (off the critical path).
+            // one pair of scores (a, b) -> P values in place, packed 16-bit pair returned
+            auto exp_pair = [&](auto split, uint32_t &a, uint32_t &b, int q) -> uint32_t {
+                const uint64_t t = f2_fma(f2_pack(__uint_as_float(a), __uint_as_float(b)), c2, nmc2);
+                float t0, t1, p0, p1;
+                f2_unpack(t, t0, t1);
+                if (decltype(split)::value && (q & 7) < exp2_emu_pairs<D_QK>()) {
+                    f2_unpack(ex2_poly2(t0, t1), p0, p1);
+                } else {
+                    p0 = ex2(t0);
+                    p1 = ex2(t1);
+                }
+                a = __float_as_uint(p0);
+                b = __float_as_uint(p1);
+                return Elem<T>::pack2(p0, p1);
+            };
+            auto exp_row = [&](auto split) {
+#pragma unroll
+                for (int h = 0; h < NCH; ++h) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) pk[q] = exp_pair(split, sr[h][2 * q], sr[h][2 * q + 1], q);
+                    tc::st16(p_addr + 16 * h, pk);
+                }
+                if constexpr (TAIL == 16) {
+                    uint32_t pk8[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) pk8[q] = exp_pair(split, st[2 * q], st[2 * q + 1], q);
+                    tc::st8(p_addr + 16 * NCH, pk8);
+                }
+            };
+            if (masked)
+                exp_row(std::integral_constant<bool, false>());
+            else
+                exp_row(std::integral_constant<bool, true>());
             tc::wait_st();
             if (p.kvcache && j == nk - 1 && j0 + BN > N) {
                 // cache rows past N_b may hold anything: zero them in the V tile
@@ -789,8 +854,10 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             for (int h = 0; h < NCH; ++h)
 #pragma unroll
                 for (int e = 0; e < 32; e += 2)
-                    rs2[(e >> 1) & 3] =
-                        f2_add(rs2[(e >> 1) & 3], f2_pack(__uint_as_float(sr[h][e]), __uint_as_float(sr[h][e + 1])));
+                    rs2[(e >> 1) & 3] = f2_add(rs2[(e >> 1) & 3], f2_pack(__uint_as_float(sr[h][e]), __uint_as_float(sr[h][e + 1])));
+#pragma unroll
+            for (int e = 0; e < TAIL; e += 2)
+                rs2[(e >> 1) & 3] = f2_add(rs2[(e >> 1) & 3], f2_pack(__uint_as_float(st[e]), __uint_as_float(st[e + 1])));
             float r0, r1, r2, r3, r4, r5, r6, r7;
             f2_unpack(rs2[0], r0, r1);
             f2_unpack(rs2[1], r2, r3);
@@ -799,7 +866,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             l = l * alpha + (((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7)));
         }
         // ------------------------------------------------ epilogue
-        if (ok && nk > jb && !mbar_wait(&o_full[x], 0, p.status)) ok = false;
+        if (ok && nk > jb && !mbar_wait(&pv_done[x], (nk - 1 - jb) & 1, p.status)) ok = false;
         tc::fence_after_sync();
         T *orow = static_cast<T *>(p.out) + tb * p.os.b + (int64_t)(qoff + i) * p.os.s + hq * p.os.h;
         const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -842,7 +909,19 @@ static cudaError_t run_prefill(const PrefillParams &p, const CUtensorMap &tmQ, c
         cudaError_t e = cudaFuncSetAttribute(prefill2_kernel<T, D_QK, D_V>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C2::SMEM);
         if (e != cudaSuccess) return e;
-        dim3 grid((p.n_q_tiles + 1) / 2, p.h_q / p.pack, p.b);
+        // the kernel's setmaxnreg split (128 x 64 + 256 x 216 registers) must
+        // fit in what the block is launched with, or the increase never returns
+        static int launch_regs = -1;
+        if (launch_regs < 0) {
+            cudaFuncAttributes fa_attr;
+            e = cudaFuncGetAttributes(&fa_attr, prefill2_kernel<T, D_QK, D_V>);
+            if (e != cudaSuccess) return e;
+            launch_regs = fa_attr.numRegs;
+        }
+        if (launch_regs * 384 < 128 * 64 + 256 * 216) return cudaErrorInvalidConfiguration;
+        const int64_t nblk = (int64_t)((p.n_q_tiles + 1) / 2) * (p.h_q / p.pack) * p.b;
+        if (nblk > 0x7fffffff) return cudaErrorInvalidConfiguration;
+        dim3 grid((unsigned)nblk);
         kernel_event(0, st);
         prefill2_kernel<T, D_QK, D_V><<<grid, 384, C2::SMEM, st>>>(tmQ, tmK, tmV, p);
         e = cudaGetLastError();
@@ -853,7 +932,9 @@ static cudaError_t run_prefill(const PrefillParams &p, const CUtensorMap &tmQ, c
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel<T, D_QK, D_V>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.n_q_tiles, p.h_q / p.pack, p.b);
+    const int64_t nblk = (int64_t)p.n_q_tiles * (p.h_q / p.pack) * p.b;
+    if (nblk > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    dim3 grid((unsigned)nblk);
     kernel_event(0, st);
     prefill_kernel<T, D_QK, D_V><<<grid, 256, C::SMEM, st>>>(tmQ, tmK, tmV, p);
     e = cudaGetLastError();
@@ -864,8 +945,8 @@ static cudaError_t run_prefill(const PrefillParams &p, const CUtensorMap &tmQ, c
 #define FA_PREFILL_DIMS(X) X(64, 64) X(128, 128) X(192, 128) X(128, 64) X(64, 128) X(192, 64)
 
 int prefill_block_n(int d_qk, int d_v, int tiles_per_cta) {
-    (void)d_v;
-    return (tiles_per_cta == 2 && d_qk > 128) ? 96 : kBN;
+    (void)d_qk;
+    return (tiles_per_cta == 2 && d_v > 64) ? 80 : kBN;
 }
 
 bool prefill_supported(int d_qk, int d_v) {
