@@ -14,158 +14,41 @@
 // Three kernels, no atomics, no waits between CTAs (the result does not
 // depend on scheduling):
 //  - bwd_dot_kernel: D_i, one warp per (batch, row, query head).
-//  - bwd_dkdv_kernel: one CTA per 64 keys of a (batch, kv head).  Its four
-//    warps own 16 keys each and walk the query tiles, of every query head of
-//    the group, that see any of those keys.  They form S^T = K Q^T and
-//    dP^T = V dO^T, so that P^T and dS^T leave the accumulators in the
-//    register layout the next products take as their A operand:
-//    dV += P^T dO and dK += dS^T Q.  dk and dv are written once, at the end.
-//  - bwd_dq_kernel: one CTA per 64 query rows of a (batch, query head); its
-//    warps own 16 rows each and walk the key tiles those rows see:
-//    S = Q K^T, dP = dO V^T, dQ += dS K.  (S and dP are formed twice, once
-//    per kernel: the price of writing dq without atomics.)
-// Products run on mma.sync m16n8k16 with fp32 accumulation; P and dS are
-// rounded to the element type as MMA operands.  Tiles are staged in shared
-// memory with cp.async (two buffers), in the swizzled layout of swz_offset so
-// that ldmatrix reads are free of bank conflicts; rows past the sequence are
-// zero-filled.
+//  - bwd_dkdv_kernel: one CTA per 128 keys of a (batch, kv head), walking the
+//    64-row query tiles, of every query head of the group, that see any of
+//    those keys.  On the tensor cores (tcgen05, operands staged by TMA,
+//    accumulators in TMEM): S^T = K Q^T and dP^T = V dO^T with the 128 keys
+//    as M; the elementwise warpgroup (thread t = key row t = TMEM lane t)
+//    turns them into P^T and dS^T, written back to TMEM as 16-bit pairs, the
+//    A operand of dV += P^T dO and dK += dS^T Q, which accumulate in TMEM for
+//    the whole walk.  S^T / dP^T of the next query tile are computed while
+//    the elementwise warpgroup works on the current one.
+//  - bwd_dq_kernel: one CTA per 128 query rows of a (batch, query head),
+//    walking 64-key tiles: S = Q K^T, dP = dO V^T, dQ += dS K, likewise.
+//    (S and dP are formed twice, once per kernel: the price of writing dq
+//    without atomics.)
+// P and dS are rounded to the element type as MMA operands; rows past a
+// sequence arrive as zeros from the TMA (out-of-bounds fill) and are masked.
+#include <type_traits>
+
 #include "fa_common.cuh"
 #include "fa_internal.h"
+#include "tcgen05.cuh"
 
 namespace fa {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kBwdThreads = 128;  // four warps
-constexpr int kKeysPerCta = 64;   // dk/dv kernel: 16 keys per warp
-constexpr int kRowsPerCta = 64;   // dq kernel: 16 query rows per warp
-constexpr int kDqBK = 32;         // dq kernel: keys per staged K/V tile
 
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)), "l"(gmem_src)
+// Four floats from shared memory, not moved across other memory operations
+// (keeps the elementwise loop from hoisting every tile value into registers).
+__device__ __forceinline__ float4 lds4(const float *p) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(smem_addr(p))
                  : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// Stage rows 0 .. ROWS-1 of a [rows][D] tile (row r at g + r * stride) into
-// the swizzled tile at `tile`; rows >= valid are zero-filled.
-template <typename T, int D, int ROWS>
-__device__ __forceinline__ void stage_rows(char *tile, const T *g, int64_t stride, int valid, int tid) {
-    constexpr int CPR = D / 8;  // 16-byte chunks per row
-    for (int idx = tid; idx < ROWS * CPR; idx += kBwdThreads) {
-        const int r = idx / CPR, c = idx % CPR;
-        char *dst = tile + swz_offset<D>(r, c * 8, ROWS);
-        if (r < valid)
-            cp_async16(dst, g + r * stride + c * 8);
-        else
-            *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
-    }
-}
-
-// acc[0 .. N8) += A (16 x K, rows of tile a at row a0) * B^T where B is the
-// tile b (rows b0 .. b0 + 8*N8 - 1, K columns): the product of two row-major
-// tiles over their shared column dimension (Q K^T, K Q^T, dO V^T, V dO^T).
-template <typename T, int K, int AROWS, int BROWS, int N8>
-__device__ __forceinline__ void mma_rows_rows(float (*acc)[4], uint32_t a_tile, int a0, uint32_t b_tile, int b0,
-                                              int lane) {
-#pragma unroll
-    for (int kk = 0; kk < K / 16; ++kk) {
-        uint32_t a[4];
-        ldmatrix_x4(a_tile + swz_offset<K>(a0 + (lane & 15), kk * 16 + ((lane >> 4) << 3), AROWS), a[0], a[1], a[2],
-                    a[3]);
-#pragma unroll
-        for (int n2 = 0; n2 < N8 / 2; ++n2) {
-            uint32_t b[4];
-            ldmatrix_x4(b_tile + swz_offset<K>(b0 + n2 * 16 + (lane & 7) + ((lane >> 4) << 3),
-                                               kk * 16 + (((lane >> 3) & 1) << 3), BROWS),
-                        b[0], b[1], b[2], b[3]);
-            Mma<T>::run(acc[2 * n2], a, b[0], b[1]);
-            Mma<T>::run(acc[2 * n2 + 1], a, b[2], b[3]);
-        }
-    }
-}
-
-// Two independent mma_rows_rows products (S and dP) interleaved in one
-// k-loop, so that twice as many accumulators are in flight per warp.
-template <typename T, int K1, int K2, int AROWS, int BROWS, int N8>
-__device__ __forceinline__ void mma_rows_rows2(float (*acc1)[4], uint32_t a1_tile, uint32_t b1_tile,
-                                               float (*acc2)[4], uint32_t a2_tile, uint32_t b2_tile, int a0,
-                                               int lane) {
-    constexpr int KS = (K1 > K2 ? K1 : K2) / 16;
-#pragma unroll
-    for (int kk = 0; kk < KS; ++kk) {
-        if (kk < K1 / 16) {
-            uint32_t a[4];
-            ldmatrix_x4(a1_tile + swz_offset<K1>(a0 + (lane & 15), kk * 16 + ((lane >> 4) << 3), AROWS), a[0], a[1],
-                        a[2], a[3]);
-#pragma unroll
-            for (int n2 = 0; n2 < N8 / 2; ++n2) {
-                uint32_t b[4];
-                ldmatrix_x4(b1_tile + swz_offset<K1>(n2 * 16 + (lane & 7) + ((lane >> 4) << 3),
-                                                     kk * 16 + (((lane >> 3) & 1) << 3), BROWS),
-                            b[0], b[1], b[2], b[3]);
-                Mma<T>::run(acc1[2 * n2], a, b[0], b[1]);
-                Mma<T>::run(acc1[2 * n2 + 1], a, b[2], b[3]);
-            }
-        }
-        if (kk < K2 / 16) {
-            uint32_t a[4];
-            ldmatrix_x4(a2_tile + swz_offset<K2>(a0 + (lane & 15), kk * 16 + ((lane >> 4) << 3), AROWS), a[0], a[1],
-                        a[2], a[3]);
-#pragma unroll
-            for (int n2 = 0; n2 < N8 / 2; ++n2) {
-                uint32_t b[4];
-                ldmatrix_x4(b2_tile + swz_offset<K2>(n2 * 16 + (lane & 7) + ((lane >> 4) << 3),
-                                                     kk * 16 + (((lane >> 3) & 1) << 3), BROWS),
-                            b[0], b[1], b[2], b[3]);
-                Mma<T>::run(acc2[2 * n2], a, b[0], b[1]);
-                Mma<T>::run(acc2[2 * n2 + 1], a, b[2], b[3]);
-            }
-        }
-    }
-}
-
-// acc[0 .. D/8) += X (16 x KR, given as accumulator fragments x[KR/8][4]) *
-// tile (rows 0 .. KR-1, D columns): X's columns contract with the tile's
-// rows (P^T dO, dS^T Q, dS K).
-template <typename T, int D, int KR, int ROWS>
-__device__ __forceinline__ void mma_frag_rows(float (*acc)[4], const float (*x)[4], uint32_t tile, int lane) {
-#pragma unroll
-    for (int kq = 0; kq < KR / 16; ++kq) {
-        uint32_t a[4];
-        a[0] = Elem<T>::pack2(x[2 * kq][0], x[2 * kq][1]);
-        a[1] = Elem<T>::pack2(x[2 * kq][2], x[2 * kq][3]);
-        a[2] = Elem<T>::pack2(x[2 * kq + 1][0], x[2 * kq + 1][1]);
-        a[3] = Elem<T>::pack2(x[2 * kq + 1][2], x[2 * kq + 1][3]);
-#pragma unroll
-        for (int nn = 0; nn < D / 16; ++nn) {
-            uint32_t b[4];
-            ldmatrix_x4_trans(tile + swz_offset<D>(kq * 16 + (lane & 7) + (((lane >> 3) & 1) << 3),
-                                                   nn * 16 + ((lane >> 4) << 3), ROWS),
-                              b[0], b[1], b[2], b[3]);
-            Mma<T>::run(acc[2 * nn], a, b[0], b[1]);
-            Mma<T>::run(acc[2 * nn + 1], a, b[2], b[3]);
-        }
-    }
-}
-
-// Store a warp's 16 x D accumulator block (rows row0 + 0..15, scaled by
-// `mul`) as element-type rows at g + row * stride; rows >= valid are skipped.
-template <typename T, int D>
-__device__ __forceinline__ void store_rows(T *g, int64_t stride, const float (*acc)[4], int row0, int valid,
-                                           float mul, int lane) {
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-        const int r = row0 + (lane >> 2) + hr * 8;
-        if (r >= valid) continue;
-        T *dst = g + r * stride + ((lane & 3) << 1);
-#pragma unroll
-        for (int n = 0; n < D / 8; ++n)
-            *reinterpret_cast<uint32_t *>(dst + n * 8) =
-                Elem<T>::pack2(acc[n][hr * 2] * mul, acc[n][hr * 2 + 1] * mul);
-    }
+    return v;
 }
 
 // ---------------------------------------------------------------- D_i
@@ -188,34 +71,69 @@ __global__ void __launch_bounds__(256) bwd_dot_kernel(const BwdParams p) {
     if (lane == 0) p.dsum[((int64_t)bi * p.h_q + h) * p.s_q + i] = acc;
 }
 
+
 // ---------------------------------------------------------------- dk, dv
-template <int D_QK, int D_V, int BQ>
-struct DkdvSmem {
-    static constexpr int K = kKeysPerCta * D_QK * 2;
-    static constexpr int V = kKeysPerCta * D_V * 2;
-    static constexpr int Q = BQ * D_QK * 2;
-    static constexpr int DO = BQ * D_V * 2;
-    static constexpr int OFF_V = K;
-    static constexpr int OFF_Q = OFF_V + V;             // two buffers
-    static constexpr int OFF_DO = OFF_Q + 2 * Q;        // two buffers
-    static constexpr int OFF_L = OFF_DO + 2 * DO;       // [2][BQ] lse * log2(e)
-    static constexpr int OFF_D = OFF_L + 2 * BQ * 4;    // [2][BQ] D
-    static constexpr int BYTES = OFF_D + 2 * BQ * 4;
+constexpr int kBK = 128;   // keys per dk/dv CTA (the MMA M)
+constexpr int kBQ = 64;    // query rows per tile of the dk/dv walk
+constexpr int kDqBM = 128; // query rows per dq CTA (the MMA M)
+constexpr int kDqBN = 64;  // keys per tile of the dq walk
+
+// Shared memory of the dk/dv kernel: the K and V tiles (loaded once), then a
+// ring of stages, each holding a Q tile, a dO tile and the tile's
+// lse * log2(e) and D values; every TMA destination is 1024-byte aligned
+// (128-byte swizzle).  TMEM: S^T, dP^T, P^T, dS^T (16-bit pairs), dV, dK.
+template <int D_QK, int D_V>
+struct DkdvCfg {
+    static constexpr int KBYTES = kBK * D_QK * 2;
+    static constexpr int VBYTES = kBK * D_V * 2;
+    static constexpr int KBOX = kBK * 128;     // bytes of one 64-column box of the K / V tile
+    static constexpr int QBYTES = kBQ * D_QK * 2;
+    static constexpr int DOBYTES = kBQ * D_V * 2;
+    static constexpr int QBOX = kBQ * 128;     // ... of a Q / dO tile
+    static constexpr int OFF_LD = QBYTES + DOBYTES;
+    static constexpr int STAGE = (OFF_LD + 2 * kBQ * 4 + 1023) / 1024 * 1024;
+    static constexpr int ST_RAW = (224 * 1024 - KBYTES - VBYTES) / STAGE;
+    static constexpr int ST = ST_RAW > 4 ? 4 : ST_RAW;
+    static constexpr int SMEM = 1024 + KBYTES + VBYTES + ST * STAGE + 256;
+    static constexpr uint32_t T_S = 0, T_DP = kBQ, T_P = 2 * kBQ, T_DS = 2 * kBQ + kBQ / 2, T_DV = 3 * kBQ,
+                              T_DK = 3 * kBQ + D_V;
+    static_assert(T_DK + D_QK <= 512, "TMEM columns");
+    static_assert(ST >= 2, "stage ring");
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
-template <typename T, int D_QK, int D_V, int BQ>
-__global__ void __launch_bounds__(kBwdThreads, 2) bwd_dkdv_kernel(const BwdParams p) {
-    using S = DkdvSmem<D_QK, D_V, BQ>;
-    extern __shared__ __align__(128) char smem[];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // blocks are dispatched roughly in linear-index order: key tile = the
-    // slowest index, so the low key tiles of every (batch, head), which the
-    // most query rows see under a causal mask, start first
-    const int slices = gridDim.y * gridDim.z;
-    const int lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
-    const int j0 = (lin / slices) * kKeysPerCta, hk = (lin % slices) % p.h_kv, bi = (lin % slices) / p.h_kv;
+template <typename T, int D_QK, int D_V>
+__global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                          const __grid_constant__ CUtensorMap tmV,
+                                                          const __grid_constant__ CUtensorMap tmQ,
+                                                          const __grid_constant__ CUtensorMap tmDO,
+                                                          const BwdParams p) {
+    using C = DkdvCfg<D_QK, D_V>;
+    constexpr int ST = C::ST;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sK = smem;
+    uint8_t *sV = sK + C::KBYTES;
+    uint8_t *sStage = sV + C::VBYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + ST * C::STAGE);
+    uint64_t *kv_full = bars;              // 1
+    uint64_t *full = kv_full + 1;          // ST: Q, dO (TMA) and lse / D (the producer warp's 32 lanes)
+    uint64_t *empty = full + ST;           // ST
+    uint64_t *s_full = empty + ST;         // S^T, dP^T of the tile complete
+    uint64_t *s_free = s_full + 1;         // ... read into registers
+    uint64_t *p_full = s_free + 1;         // P^T, dS^T written
+    uint64_t *pd_done = p_full + 1;        // dV, dK of the tile complete (P^T, dS^T free)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pd_done + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // key tile = the slowest index: the low key tiles of every (batch, kv
+    // head), which the most query rows see under a causal mask, start first
+    const int slices = p.h_kv * p.b;
+    const int kt = (int)blockIdx.x / slices, rem = (int)blockIdx.x - kt * slices;
+    const int hk = rem % p.h_kv, bi = rem / p.h_kv;
+    const int j0 = kt * kBK;
     const int N = p.s_k, s_q = p.s_q;
-    const int kvalid = min(kKeysPerCta, N - j0);
+    const int kvalid = min(kBK, N - j0);
     const int j_hi = j0 + kvalid - 1;
 
     // query rows that see any of keys j0 .. j_hi: the last visible key and
@@ -237,232 +155,494 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_dkdv_kernel(const BwdParam
         if (f > j_hi) hi = mid; else lo = mid + 1;
     }
     const int i_hi = lo - 1;
-    const int qt0 = i_lo / BQ;
-    const int n_qt = i_lo <= i_hi ? i_hi / BQ - qt0 + 1 : 0;
-    const int n_tiles = p.g * n_qt;
+    const int qt0 = i_lo / kBQ;
+    const int n_qt = i_lo <= i_hi ? i_hi / kBQ - qt0 + 1 : 0;
+    const int n_tiles = p.g * n_qt;   // tile u: query head hk g + u / n_qt, rows (qt0 + u % n_qt) kBQ ..
 
-    const T *kbase = static_cast<const T *>(p.k) + bi * p.ks.b + hk * p.ks.h;
-    const T *vbase = static_cast<const T *>(p.v) + bi * p.vs.b + hk * p.vs.h;
-    auto issue = [&](int u) {
-        const int hq = hk * p.g + u / n_qt;
-        const int i0 = (qt0 + u % n_qt) * BQ;
-        const int valid = min(BQ, s_q - i0);
-        const int buf = u & 1;
-        stage_rows<T, D_QK, BQ>(smem + S::OFF_Q + buf * S::Q,
-                                static_cast<const T *>(p.q) + bi * p.qs.b + (int64_t)i0 * p.qs.s + hq * p.qs.h,
-                                p.qs.s, valid, tid);
-        stage_rows<T, D_V, BQ>(smem + S::OFF_DO + buf * S::DO,
-                               static_cast<const T *>(p.dout) + bi * p.dos.b + (int64_t)i0 * p.dos.s + hq * p.dos.h,
-                               p.dos.s, valid, tid);
-        if (tid < BQ) {
-            const int64_t row = ((int64_t)bi * p.h_q + hq) * s_q + i0 + tid;
-            float *sl = reinterpret_cast<float *>(smem + S::OFF_L) + buf * BQ;
-            float *sd = reinterpret_cast<float *>(smem + S::OFF_D) + buf * BQ;
-            sl[tid] = tid < valid ? p.lse[row] * kLog2e : 0.f;
-            sd[tid] = tid < valid ? p.dsum[row] : 0.f;
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(&full[s], 1 + 32);
+            mbar_init(&empty[s], 1);
         }
-        cp_async_commit();
-    };
-
-    float dk[D_QK / 8][4], dv[D_V / 8][4];
-#pragma unroll
-    for (int n = 0; n < D_QK / 8; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dk[n][e] = 0.f;
-#pragma unroll
-    for (int n = 0; n < D_V / 8; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dv[n][e] = 0.f;
-
-    if (n_tiles > 0) {
-        stage_rows<T, D_QK, kKeysPerCta>(smem, kbase + (int64_t)j0 * p.ks.s, p.ks.s, kvalid, tid);
-        stage_rows<T, D_V, kKeysPerCta>(smem + S::OFF_V, vbase + (int64_t)j0 * p.vs.s, p.vs.s, kvalid, tid);
-        issue(0);
+        mbar_init(s_full, 1);
+        mbar_init(s_free, 4);
+        mbar_init(p_full, 4);
+        mbar_init(pd_done, 1);
+        fence_barrier_init();
     }
-    const uint32_t sK = smem_addr(smem), sV = smem_addr(smem + S::OFF_V);
-    const int key_r = warp * 16 + (lane >> 2);  // this thread's key rows: key_r, key_r + 8
-    for (int u = 0; u < n_tiles; ++u) {
-        if (u + 1 < n_tiles) {
-            issue(u + 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-        const int buf = u & 1;
-        const int i0 = (qt0 + u % n_qt) * BQ;
-        const uint32_t sQ = smem_addr(smem + S::OFF_Q + buf * S::Q);
-        const uint32_t sDO = smem_addr(smem + S::OFF_DO + buf * S::DO);
-        const float *sl = reinterpret_cast<const float *>(smem + S::OFF_L) + buf * BQ;
-        const float *sd = reinterpret_cast<const float *>(smem + S::OFF_D) + buf * BQ;
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
 
-        float s[BQ / 8][4], dp[BQ / 8][4];
+    if (warp == 0) {
+        // ------------------------------------------------ producer: TMA tiles; lse and D by all lanes
+        if (n_tiles > 0) {
+            if (lane == 0) {
+                tma_prefetch_desc(&tmK);
+                tma_prefetch_desc(&tmV);
+                tma_prefetch_desc(&tmQ);
+                tma_prefetch_desc(&tmDO);
+                mbar_arrive_expect_tx(kv_full, C::KBYTES + C::VBYTES);
 #pragma unroll
-        for (int n = 0; n < BQ / 8; ++n)
+                for (int c = 0; c < D_QK / 64; ++c) tma_load_4d(sK + c * C::KBOX, &tmK, kv_full, c * 64, hk, j0, bi);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.f;
-        // S^T = K Q^T and dP^T = V dO^T
-        mma_rows_rows2<T, D_QK, D_V, kKeysPerCta, BQ, BQ / 8>(s, sK, sQ, dp, sV, sDO, warp * 16, lane);
-
-        // the whole tile is visible when its rows all exist, its last row's
-        // first visible key is at most j0 and its first row's last visible
-        // key at least j0 + 63 (both bounds are nondecreasing in the row)
-        bool full = i0 + BQ <= s_q && kvalid == kKeysPerCta;
-        if (full) {
-            int64_t f, l;
-            visible_keys(i0, N, s_q, p.causal, p.win_left, p.win_right, f, l);
-            full = l >= j_hi;
-            visible_keys(i0 + BQ - 1, N, s_q, p.causal, p.win_left, p.win_right, f, l);
-            full = full && f <= j0;
+                for (int c = 0; c < D_V / 64; ++c) tma_load_4d(sV + c * C::KBOX, &tmV, kv_full, c * 64, hk, j0, bi);
+            }
+            for (int u = 0; u < n_tiles; ++u) {
+                const int st = u % ST;
+                if (u >= ST && !mbar_wait(&empty[st], ((u / ST) - 1) & 1, p.status)) break;
+                const int hq = hk * p.g + u / n_qt;
+                const int i0 = (qt0 + u % n_qt) * kBQ;
+                uint8_t *stage = sStage + st * C::STAGE;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[st], C::QBYTES + C::DOBYTES);
+#pragma unroll
+                    for (int c = 0; c < D_QK / 64; ++c)
+                        tma_load_4d(stage + c * C::QBOX, &tmQ, &full[st], c * 64, hq, i0, bi);
+#pragma unroll
+                    for (int c = 0; c < D_V / 64; ++c)
+                        tma_load_4d(stage + C::QBYTES + c * C::QBOX, &tmDO, &full[st], c * 64, hq, i0, bi);
+                }
+                // rows past s_q: lse = +inf makes P = 0 there
+                float *ld = reinterpret_cast<float *>(stage + C::OFF_LD);
+                for (int t = lane; t < kBQ; t += 32) {
+                    const int i = i0 + t;
+                    const int64_t row = ((int64_t)bi * p.h_q + hq) * s_q + i;
+                    ld[t] = i < s_q ? p.lse[row] * kLog2e : INFINITY;
+                    ld[kBQ + t] = i < s_q ? p.dsum[row] : 0.f;
+                }
+                mbar_arrive(&full[st]);
+            }
         }
-        // P^T and dS^T in place: element (key j, query i)
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (whole warp loops, one lane issues)
+        if (n_tiles > 0) {
+            const bool leader = tc::elect_one();
+            const uint32_t idesc_s = tc::idesc_f16(bf16, kBK, kBQ, false);
+            const uint32_t idesc_dv = tc::idesc_f16(bf16, kBK, D_V, true);
+            const uint32_t idesc_dk = tc::idesc_f16(bf16, kBK, D_QK, true);
+            const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aS = smem_addr(sStage);
+            bool ok = mbar_wait(kv_full, 0, p.status);
+            // S^T = K Q^T and dP^T = V dO^T (K-major operands)
+            auto issue_sdp = [&](int u) {
+                const uint32_t q = aS + (u % ST) * C::STAGE, o = q + C::QBYTES;
+                if (leader) {
 #pragma unroll
-        for (int n = 0; n < BQ / 8; ++n)
+                    for (int k = 0; k < D_QK / 16; ++k)
+                        tc::mma_ss(tmem + C::T_S, tc::smem_desc(aK + (k >> 2) * C::KBOX + (k & 3) * 32, 16, 1024),
+                                   tc::smem_desc(q + (k >> 2) * C::QBOX + (k & 3) * 32, 16, 1024), idesc_s, k > 0);
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const int qc = n * 8 + ((lane & 3) << 1) + c;
-                const int i = i0 + qc;
-                int64_t f = 0, l = N;
-                if (!full) visible_keys(i, N, s_q, p.causal, p.win_left, p.win_right, f, l);
-                const float L = sl[qc], Dd = sd[qc];
+                    for (int k = 0; k < D_V / 16; ++k)
+                        tc::mma_ss(tmem + C::T_DP, tc::smem_desc(aV + (k >> 2) * C::KBOX + (k & 3) * 32, 16, 1024),
+                                   tc::smem_desc(o + (k >> 2) * C::QBOX + (k & 3) * 32, 16, 1024), idesc_s, k > 0);
+                    tc::commit(s_full);
+                }
+                __syncwarp();
+            };
+            // dV += P^T dO and dK += dS^T Q (P^T, dS^T from TMEM; dO, Q as MN-major B)
+            auto issue_acc = [&](int u) {
+                const uint32_t q = aS + (u % ST) * C::STAGE, o = q + C::QBYTES;
+                if (leader) {
 #pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                    const int j = j0 + key_r + hr * 8;
-                    const bool vis = full || (i < s_q && j < N && j >= f && j <= l);
-                    const float pv = vis ? ex2(s[n][hr * 2 + c] * p.scale_log2 - L) : 0.f;
-                    s[n][hr * 2 + c] = pv;
-                    dp[n][hr * 2 + c] = pv * (dp[n][hr * 2 + c] - Dd);
+                    for (int k = 0; k < kBQ / 16; ++k)
+                        tc::mma_ts(tmem + C::T_DV, tmem + C::T_P + k * 8, tc::smem_desc(o + k * 16 * 128, C::QBOX, 1024),
+                                   idesc_dv, (u > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int k = 0; k < kBQ / 16; ++k)
+                        tc::mma_ts(tmem + C::T_DK, tmem + C::T_DS + k * 8, tc::smem_desc(q + k * 16 * 128, C::QBOX, 1024),
+                                   idesc_dk, (u > 0 || k > 0) ? 1u : 0u);
+                    tc::commit(&empty[u % ST]);
+                    tc::commit(pd_done);
+                }
+                __syncwarp();
+            };
+            if (ok && (ok = mbar_wait(&full[0], 0, p.status))) {
+                tc::fence_after_sync();
+                issue_sdp(0);
+            }
+            for (int u = 0; u < n_tiles && ok; ++u) {
+                if (u + 1 < n_tiles) {
+                    if (!(ok = mbar_wait(&full[(u + 1) % ST], ((u + 1) / ST) & 1, p.status))) break;
+                    if (!(ok = mbar_wait(s_free, u & 1, p.status))) break;
+                    tc::fence_after_sync();
+                    issue_sdp(u + 1);
+                }
+                if (!(ok = mbar_wait(p_full, u & 1, p.status))) break;
+                tc::fence_after_sync();
+                issue_acc(u);
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------ elementwise warpgroup: key row j = TMEM lane
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+        const int j = j0 + r;
+        const bool key_valid = r < kvalid;
+        // queries that see key j: i_min .. i_max (bottom-right alignment a_i = i + N - s_q)
+        const int64_t off = (int64_t)N - s_q;
+        int64_t i_min = 0, i_max = (int64_t)s_q - 1;
+        if (p.causal) i_min = max(i_min, (int64_t)j - off);
+        if (p.win_right >= 0) i_min = max(i_min, (int64_t)j - p.win_right - off);
+        if (p.win_left >= 0) i_max = min(i_max, (int64_t)j + p.win_left - off);
+        if (!key_valid) i_max = -1;
+        const float c = p.scale_log2;
+        bool ok = true;
+        for (int u = 0; u < n_tiles && ok; ++u) {
+            if (!(ok = mbar_wait(s_full, u & 1, p.status))) break;
+            tc::fence_after_sync();
+            uint32_t sr[2][32], dr[2][32];
+            tc::ld32(tmem + lane_addr + C::T_S, sr[0]);
+            tc::ld32(tmem + lane_addr + C::T_S + 32, sr[1]);
+            tc::ld32(tmem + lane_addr + C::T_DP, dr[0]);
+            tc::ld32(tmem + lane_addr + C::T_DP + 32, dr[1]);
+            tc::wait_ld();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_free);
+            const int st = u % ST;
+            if (!(ok = mbar_wait(&full[st], (u / ST) & 1, p.status))) break;
+            // P^T and dS^T of the previous tile have been read by its dV / dK
+            if (u > 0) {
+                if (!(ok = mbar_wait(pd_done, (u - 1) & 1, p.status))) break;
+                tc::fence_after_sync();
+            }
+            const float *ld = reinterpret_cast<const float *>(sStage + st * C::STAGE + C::OFF_LD);
+            const int64_t i0 = (int64_t)(qt0 + u % n_qt) * kBQ;
+            const bool all_vis = i0 >= i_min && i0 + kBQ - 1 <= i_max;
+            // 16 query columns at a time: P^T and dS^T as 16-bit pairs
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                const int h = qq >> 1, e0 = (qq & 1) * 16;
+                float Lq[16], Dq[16];
+#pragma unroll
+                for (int e = 0; e < 16; e += 4) {
+                    const float4 l4 = lds4(ld + 16 * qq + e), d4 = lds4(ld + kBQ + 16 * qq + e);
+                    Lq[e] = l4.x; Lq[e + 1] = l4.y; Lq[e + 2] = l4.z; Lq[e + 3] = l4.w;
+                    Dq[e] = d4.x; Dq[e + 1] = d4.y; Dq[e + 2] = d4.z; Dq[e + 3] = d4.w;
+                }
+                uint32_t pp[8], pd[8];
+#pragma unroll
+                for (int e = 0; e < 16; e += 2) {
+                    const int qc = 16 * qq + e;
+                    float p0 = ex2(fmaf(__uint_as_float(sr[h][e0 + e]), c, -Lq[e]));
+                    float p1 = ex2(fmaf(__uint_as_float(sr[h][e0 + e + 1]), c, -Lq[e + 1]));
+                    if (!all_vis) {
+                        if (i0 + qc < i_min || i0 + qc > i_max) p0 = 0.f;
+                        if (i0 + qc + 1 < i_min || i0 + qc + 1 > i_max) p1 = 0.f;
+                    }
+                    pp[e >> 1] = Elem<T>::pack2(p0, p1);
+                    pd[e >> 1] = Elem<T>::pack2(p0 * (__uint_as_float(dr[h][e0 + e]) - Dq[e]),
+                                                p1 * (__uint_as_float(dr[h][e0 + e + 1]) - Dq[e + 1]));
+                }
+                tc::st8(tmem + lane_addr + C::T_P + 8 * qq, pp);
+                tc::st8(tmem + lane_addr + C::T_DS + 8 * qq, pd);
+            }
+            tc::wait_st();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        // ------------------------------------------------ epilogue: dv = dV, dk = scale dK
+        const bool have = n_tiles > 0;
+        if (have && ok) ok = mbar_wait(pd_done, (n_tiles - 1) & 1, p.status);
+        tc::fence_after_sync();
+        T *dvrow = static_cast<T *>(p.dv) + bi * p.dvs.b + (int64_t)j * p.dvs.s + hk * p.dvs.h;
+        T *dkrow = static_cast<T *>(p.dk) + bi * p.dks.b + (int64_t)j * p.dks.s + hk * p.dks.h;
+#pragma unroll
+        for (int h = 0; h < (D_V + D_QK) / 32; ++h) {
+            const bool is_v = h < D_V / 32;
+            const int col = is_v ? h * 32 : (h - D_V / 32) * 32;
+            uint32_t orr[32];
+            if (have) {
+                tc::ld32(tmem + lane_addr + (is_v ? C::T_DV : C::T_DK) + col, orr);
+                tc::wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) orr[e] = 0u;
+            }
+            if (key_valid) {
+                const float mul = is_v ? 1.f : p.scale;
+                T *dst = (is_v ? dvrow : dkrow) + col;
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                    float f[8];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) f[t] = __uint_as_float(orr[e + t]) * mul;
+                    reinterpret_cast<uint4 *>(dst + e)[0] = pack8<T>(f);
                 }
             }
-        mma_frag_rows<T, D_V, BQ, BQ>(dv, s, sDO, lane);    // dV += P^T dO
-        mma_frag_rows<T, D_QK, BQ, BQ>(dk, dp, sQ, lane);   // dK += dS^T Q
-        __syncthreads();
+        }
     }
-
-    store_rows<T, D_QK>(static_cast<T *>(p.dk) + bi * p.dks.b + (int64_t)j0 * p.dks.s + hk * p.dks.h, p.dks.s, dk,
-                        warp * 16, kvalid, p.scale, lane);
-    store_rows<T, D_V>(static_cast<T *>(p.dv) + bi * p.dvs.b + (int64_t)j0 * p.dvs.s + hk * p.dvs.h, p.dvs.s, dv,
-                       warp * 16, kvalid, 1.f, lane);
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
 }
 
 // ---------------------------------------------------------------- dq
+// Shared memory: the Q and dO tiles (loaded once) and a ring of K / V
+// stages.  TMEM: S, dP, dS (16-bit pairs), dQ.
 template <int D_QK, int D_V>
-struct DqSmem {
-    static constexpr int Q = kRowsPerCta * D_QK * 2;
-    static constexpr int DO = kRowsPerCta * D_V * 2;
-    static constexpr int K = kDqBK * D_QK * 2;
-    static constexpr int V = kDqBK * D_V * 2;
-    static constexpr int OFF_DO = Q;
-    static constexpr int OFF_K = OFF_DO + DO;   // two buffers
-    static constexpr int OFF_V = OFF_K + 2 * K;  // two buffers
-    static constexpr int BYTES = OFF_V + 2 * V;
+struct DqCfg {
+    static constexpr int QBYTES = kDqBM * D_QK * 2;
+    static constexpr int DOBYTES = kDqBM * D_V * 2;
+    static constexpr int QBOX = kDqBM * 128;
+    static constexpr int KBYTES = kDqBN * D_QK * 2;
+    static constexpr int VBYTES = kDqBN * D_V * 2;
+    static constexpr int KBOX = kDqBN * 128;
+    static constexpr int STAGE = KBYTES + VBYTES;
+    static constexpr int ST_RAW = (224 * 1024 - QBYTES - DOBYTES) / STAGE;
+    static constexpr int ST = ST_RAW > 4 ? 4 : ST_RAW;
+    static constexpr int SMEM = 1024 + QBYTES + DOBYTES + ST * STAGE + 256;
+    static constexpr uint32_t T_S = 0, T_DP = kDqBN, T_DS = 2 * kDqBN, T_DQ = 2 * kDqBN + kDqBN / 2;
+    static_assert(T_DQ + D_QK <= 512, "TMEM columns");
+    static_assert(STAGE % 1024 == 0 && ST >= 2, "stage ring");
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
 template <typename T, int D_QK, int D_V>
-__global__ void __launch_bounds__(kBwdThreads, 2) bwd_dq_kernel(const BwdParams p) {
-    using S = DqSmem<D_QK, D_V>;
-    extern __shared__ __align__(128) char smem[];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // the last query tiles of every (batch, head), which see the most keys
-    // under a causal mask, start first (see bwd_dkdv_kernel)
-    const int slices = gridDim.y * gridDim.z;
-    const int lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
-    const int i0 = (gridDim.x - 1 - lin / slices) * kRowsPerCta, hq = (lin % slices) % p.h_q,
-              bi = (lin % slices) / p.h_q;
-    const int hk = hq / p.g;
-    const int N = p.s_k, s_q = p.s_q;
-    const int qvalid = min(kRowsPerCta, s_q - i0);
+__global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                        const __grid_constant__ CUtensorMap tmDO,
+                                                        const __grid_constant__ CUtensorMap tmK,
+                                                        const __grid_constant__ CUtensorMap tmV,
+                                                        const BwdParams p) {
+    using C = DqCfg<D_QK, D_V>;
+    constexpr int ST = C::ST;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem;
+    uint8_t *sDO = sQ + C::QBYTES;
+    uint8_t *sStage = sDO + C::DOBYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + ST * C::STAGE);
+    uint64_t *q_full = bars;               // 1
+    uint64_t *full = q_full + 1;           // ST
+    uint64_t *empty = full + ST;           // ST
+    uint64_t *s_full = empty + ST;
+    uint64_t *s_free = s_full + 1;
+    uint64_t *p_full = s_free + 1;
+    uint64_t *ds_done = p_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ds_done + 1);
 
-    // keys seen by rows i0 .. i0 + qvalid - 1
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the last query tiles of every (batch, head), which see the most keys
+    // under a causal mask, start first
+    const int slices = p.h_q * p.b;
+    const int n_qtiles = (int)gridDim.x / slices;
+    const int t = (int)blockIdx.x / slices, rem = (int)blockIdx.x - t * slices;
+    const int hq = rem % p.h_q, bi = rem / p.h_q;
+    const int hk = hq / p.g;
+    const int i0 = (n_qtiles - 1 - t) * kDqBM;
+    const int N = p.s_k, s_q = p.s_q;
+    const int qvalid = min(kDqBM, s_q - i0);
     int64_t f0, l0, f1, l1;
     visible_keys(i0, N, s_q, p.causal, p.win_left, p.win_right, f0, l0);
     visible_keys(i0 + qvalid - 1, N, s_q, p.causal, p.win_left, p.win_right, f1, l1);
     const int kv_end = (int)max((int64_t)0, min((int64_t)N, l1 + 1));
-    const int kt0 = (int)min(f0, (int64_t)kv_end) / kDqBK;
-    const int n_kt = kv_end > 0 ? (kv_end + kDqBK - 1) / kDqBK - kt0 : 0;
+    const int kt0 = (int)min(f0, (int64_t)kv_end) / kDqBN;
+    const int n_kt = kv_end > 0 ? (kv_end + kDqBN - 1) / kDqBN - kt0 : 0;
 
-    const T *kbase = static_cast<const T *>(p.k) + bi * p.ks.b + hk * p.ks.h;
-    const T *vbase = static_cast<const T *>(p.v) + bi * p.vs.b + hk * p.vs.h;
-    auto issue = [&](int u) {
-        const int j0 = (kt0 + u) * kDqBK;
-        const int valid = min(kDqBK, N - j0);
-        const int buf = u & 1;
-        stage_rows<T, D_QK, kDqBK>(smem + S::OFF_K + buf * S::K, kbase + (int64_t)j0 * p.ks.s, p.ks.s, valid, tid);
-        stage_rows<T, D_V, kDqBK>(smem + S::OFF_V + buf * S::V, vbase + (int64_t)j0 * p.vs.s, p.vs.s, valid, tid);
-        cp_async_commit();
-    };
-
-    // this thread's rows: r0 = i0 + warp*16 + lane/4 and r0 + 8
-    const int rbase = i0 + warp * 16 + (lane >> 2);
-    float L[2], Dd[2];
-    int64_t fv[2], lv[2];
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-        const int i = rbase + hr * 8;
-        visible_keys(i, N, s_q, p.causal, p.win_left, p.win_right, fv[hr], lv[hr]);
-        if (i >= s_q) lv[hr] = -1;  // past the rows: nothing visible
-        const int64_t row = ((int64_t)bi * p.h_q + hq) * s_q + min(i, s_q - 1);
-        L[hr] = i < s_q ? p.lse[row] * kLog2e : 0.f;
-        Dd[hr] = i < s_q ? p.dsum[row] : 0.f;
-    }
-
-    float dq[D_QK / 8][4];
-#pragma unroll
-    for (int n = 0; n < D_QK / 8; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dq[n][e] = 0.f;
-
-    if (n_kt > 0) {
-        stage_rows<T, D_QK, kRowsPerCta>(smem, static_cast<const T *>(p.q) + bi * p.qs.b + (int64_t)i0 * p.qs.s +
-                                                   hq * p.qs.h,
-                                         p.qs.s, qvalid, tid);
-        stage_rows<T, D_V, kRowsPerCta>(smem + S::OFF_DO, static_cast<const T *>(p.dout) + bi * p.dos.b +
-                                                              (int64_t)i0 * p.dos.s + hq * p.dos.h,
-                                        p.dos.s, qvalid, tid);
-        issue(0);
-    }
-    const uint32_t sQ = smem_addr(smem), sDO = smem_addr(smem + S::OFF_DO);
-    for (int u = 0; u < n_kt; ++u) {
-        if (u + 1 < n_kt) {
-            issue(u + 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
         }
-        __syncthreads();
-        const int buf = u & 1;
-        const int j0 = (kt0 + u) * kDqBK;
-        const uint32_t sK = smem_addr(smem + S::OFF_K + buf * S::K);
-        const uint32_t sV = smem_addr(smem + S::OFF_V + buf * S::V);
-
-        float s[kDqBK / 8][4], dp[kDqBK / 8][4];
-#pragma unroll
-        for (int n = 0; n < kDqBK / 8; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.f;
-        // S = Q K^T and dP = dO V^T
-        mma_rows_rows2<T, D_QK, D_V, kRowsPerCta, kDqBK, kDqBK / 8>(s, sQ, sK, dp, sDO, sV, warp * 16, lane);
-
-#pragma unroll
-        for (int n = 0; n < kDqBK / 8; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int hr = e >> 1;
-                const int j = j0 + n * 8 + ((lane & 3) << 1) + (e & 1);
-                const bool vis = j < N && j >= fv[hr] && j <= lv[hr];
-                const float pv = vis ? ex2(s[n][e] * p.scale_log2 - L[hr]) : 0.f;
-                dp[n][e] = pv * (dp[n][e] - Dd[hr]);
-            }
-        mma_frag_rows<T, D_QK, kDqBK, kDqBK>(dq, dp, sK, lane);  // dQ += dS K
-        __syncthreads();
+        mbar_init(s_full, 1);
+        mbar_init(s_free, 4);
+        mbar_init(p_full, 4);
+        mbar_init(ds_done, 1);
+        fence_barrier_init();
     }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
 
-    store_rows<T, D_QK>(static_cast<T *>(p.dq) + bi * p.dqs.b + (int64_t)i0 * p.dqs.s + hq * p.dqs.h, p.dqs.s, dq,
-                        warp * 16, qvalid, p.scale, lane);
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0 && n_kt > 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmDO);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            mbar_arrive_expect_tx(q_full, C::QBYTES + C::DOBYTES);
+#pragma unroll
+            for (int c = 0; c < D_QK / 64; ++c) tma_load_4d(sQ + c * C::QBOX, &tmQ, q_full, c * 64, hq, i0, bi);
+#pragma unroll
+            for (int c = 0; c < D_V / 64; ++c) tma_load_4d(sDO + c * C::QBOX, &tmDO, q_full, c * 64, hq, i0, bi);
+            for (int u = 0; u < n_kt; ++u) {
+                const int st = u % ST;
+                if (u >= ST && !mbar_wait(&empty[st], ((u / ST) - 1) & 1, p.status)) break;
+                const int jt = (kt0 + u) * kDqBN;
+                uint8_t *stage = sStage + st * C::STAGE;
+                mbar_arrive_expect_tx(&full[st], C::STAGE);
+#pragma unroll
+                for (int c = 0; c < D_QK / 64; ++c) tma_load_4d(stage + c * C::KBOX, &tmK, &full[st], c * 64, hk, jt, bi);
+#pragma unroll
+                for (int c = 0; c < D_V / 64; ++c)
+                    tma_load_4d(stage + C::KBYTES + c * C::KBOX, &tmV, &full[st], c * 64, hk, jt, bi);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (n_kt > 0) {
+            const bool leader = tc::elect_one();
+            const uint32_t idesc_s = tc::idesc_f16(bf16, kDqBM, kDqBN, false);
+            const uint32_t idesc_dq = tc::idesc_f16(bf16, kDqBM, D_QK, true);
+            const uint32_t aQ = smem_addr(sQ), aDO = smem_addr(sDO), aS = smem_addr(sStage);
+            bool ok = mbar_wait(q_full, 0, p.status);
+            // S = Q K^T and dP = dO V^T
+            auto issue_sdp = [&](int u) {
+                const uint32_t kk = aS + (u % ST) * C::STAGE, vv = kk + C::KBYTES;
+                if (leader) {
+#pragma unroll
+                    for (int k = 0; k < D_QK / 16; ++k)
+                        tc::mma_ss(tmem + C::T_S, tc::smem_desc(aQ + (k >> 2) * C::QBOX + (k & 3) * 32, 16, 1024),
+                                   tc::smem_desc(kk + (k >> 2) * C::KBOX + (k & 3) * 32, 16, 1024), idesc_s, k > 0);
+#pragma unroll
+                    for (int k = 0; k < D_V / 16; ++k)
+                        tc::mma_ss(tmem + C::T_DP, tc::smem_desc(aDO + (k >> 2) * C::QBOX + (k & 3) * 32, 16, 1024),
+                                   tc::smem_desc(vv + (k >> 2) * C::KBOX + (k & 3) * 32, 16, 1024), idesc_s, k > 0);
+                    tc::commit(s_full);
+                }
+                __syncwarp();
+            };
+            // dQ += dS K (dS from TMEM, K as MN-major B)
+            auto issue_dq = [&](int u) {
+                const uint32_t kk = aS + (u % ST) * C::STAGE;
+                if (leader) {
+#pragma unroll
+                    for (int k = 0; k < kDqBN / 16; ++k)
+                        tc::mma_ts(tmem + C::T_DQ, tmem + C::T_DS + k * 8, tc::smem_desc(kk + k * 16 * 128, C::KBOX, 1024),
+                                   idesc_dq, (u > 0 || k > 0) ? 1u : 0u);
+                    tc::commit(&empty[u % ST]);
+                    tc::commit(ds_done);
+                }
+                __syncwarp();
+            };
+            if (ok && (ok = mbar_wait(&full[0], 0, p.status))) {
+                tc::fence_after_sync();
+                issue_sdp(0);
+            }
+            for (int u = 0; u < n_kt && ok; ++u) {
+                if (u + 1 < n_kt) {
+                    if (!(ok = mbar_wait(&full[(u + 1) % ST], ((u + 1) / ST) & 1, p.status))) break;
+                    if (!(ok = mbar_wait(s_free, u & 1, p.status))) break;
+                    tc::fence_after_sync();
+                    issue_sdp(u + 1);
+                }
+                if (!(ok = mbar_wait(p_full, u & 1, p.status))) break;
+                tc::fence_after_sync();
+                issue_dq(u);
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------ elementwise warpgroup: query row i = TMEM lane
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+        const int i = i0 + r;
+        const bool row_valid = r < qvalid;
+        int64_t fv, lv;
+        visible_keys(i, N, s_q, p.causal, p.win_left, p.win_right, fv, lv);
+        if (!row_valid) lv = -1;
+        const int64_t row = ((int64_t)bi * p.h_q + hq) * s_q + (row_valid ? i : 0);
+        const float L = row_valid ? p.lse[row] * kLog2e : INFINITY;
+        const float Dd = row_valid ? p.dsum[row] : 0.f;
+        const float c = p.scale_log2;
+        bool ok = true;
+        for (int u = 0; u < n_kt && ok; ++u) {
+            if (!(ok = mbar_wait(s_full, u & 1, p.status))) break;
+            tc::fence_after_sync();
+            uint32_t sr[2][32], dr[2][32];
+            tc::ld32(tmem + lane_addr + C::T_S, sr[0]);
+            tc::ld32(tmem + lane_addr + C::T_S + 32, sr[1]);
+            tc::ld32(tmem + lane_addr + C::T_DP, dr[0]);
+            tc::ld32(tmem + lane_addr + C::T_DP + 32, dr[1]);
+            tc::wait_ld();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_free);
+            // dS of the previous key tile has been read by its dQ product
+            if (u > 0) {
+                if (!(ok = mbar_wait(ds_done, (u - 1) & 1, p.status))) break;
+                tc::fence_after_sync();
+            }
+            const int64_t jt = (int64_t)(kt0 + u) * kDqBN;
+            const bool all_vis = jt >= fv && jt + kDqBN - 1 <= lv;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pd[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const int64_t jj = jt + 32 * h + e;
+                    float p0 = ex2(fmaf(__uint_as_float(sr[h][e]), c, -L));
+                    float p1 = ex2(fmaf(__uint_as_float(sr[h][e + 1]), c, -L));
+                    if (!all_vis) {
+                        if (jj < fv || jj > lv) p0 = 0.f;
+                        if (jj + 1 < fv || jj + 1 > lv) p1 = 0.f;
+                    }
+                    pd[e >> 1] = Elem<T>::pack2(p0 * (__uint_as_float(dr[h][e]) - Dd),
+                                                p1 * (__uint_as_float(dr[h][e + 1]) - Dd));
+                }
+                tc::st16(tmem + lane_addr + C::T_DS + 16 * h, pd);
+            }
+            tc::wait_st();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        // ------------------------------------------------ epilogue: dq = scale dQ
+        const bool have = n_kt > 0;
+        if (have && ok) ok = mbar_wait(ds_done, (n_kt - 1) & 1, p.status);
+        tc::fence_after_sync();
+        T *dqrow = static_cast<T *>(p.dq) + bi * p.dqs.b + (int64_t)i * p.dqs.s + hq * p.dqs.h;
+#pragma unroll
+        for (int h = 0; h < D_QK / 32; ++h) {
+            uint32_t orr[32];
+            if (have) {
+                tc::ld32(tmem + lane_addr + C::T_DQ + h * 32, orr);
+                tc::wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) orr[e] = 0u;
+            }
+            if (row_valid) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                    float f[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) f[q] = __uint_as_float(orr[e + q]) * p.scale;
+                    reinterpret_cast<uint4 *>(dqrow + h * 32 + e)[0] = pack8<T>(f);
+                }
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
 }
 
-template <typename T, int D_QK, int D_V, int BQ>
-cudaError_t run_bwd(const BwdParams &p, cudaStream_t st) {
+template <typename T, int D_QK, int D_V>
+cudaError_t run_bwd(const BwdParams &p, const BwdMaps &m, cudaStream_t st) {
     const int64_t rows = (int64_t)p.b * p.s_q * p.h_q;
     if (rows > 0) {
         bwd_dot_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);
@@ -471,21 +651,23 @@ cudaError_t run_bwd(const BwdParams &p, cudaStream_t st) {
     }
     kernel_event(0, st);
     if (p.s_k > 0) {
-        using SK = DkdvSmem<D_QK, D_V, BQ>;
-        cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<T, D_QK, D_V, BQ>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SK::BYTES);
+        using CK = DkdvCfg<D_QK, D_V>;
+        cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<T, D_QK, D_V>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, CK::SMEM);
         if (e != cudaSuccess) return e;
-        dim3 grid((p.s_k + kKeysPerCta - 1) / kKeysPerCta, p.h_kv, p.b);
-        bwd_dkdv_kernel<T, D_QK, D_V, BQ><<<grid, kBwdThreads, SK::BYTES, st>>>(p);
+        const int64_t grid = (int64_t)((p.s_k + kBK - 1) / kBK) * p.h_kv * p.b;
+        if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+        bwd_dkdv_kernel<T, D_QK, D_V><<<(unsigned)grid, 256, CK::SMEM, st>>>(m.k128, m.v128, m.q64, m.do64, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (p.s_q > 0) {
-        using SQ = DqSmem<D_QK, D_V>;
+        using CQ = DqCfg<D_QK, D_V>;
         cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<T, D_QK, D_V>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SQ::BYTES);
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, CQ::SMEM);
         if (e != cudaSuccess) return e;
-        dim3 grid((p.s_q + kRowsPerCta - 1) / kRowsPerCta, p.h_q, p.b);
-        bwd_dq_kernel<T, D_QK, D_V><<<grid, kBwdThreads, SQ::BYTES, st>>>(p);
+        const int64_t grid = (int64_t)((p.s_q + kDqBM - 1) / kDqBM) * p.h_q * p.b;
+        if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+        bwd_dq_kernel<T, D_QK, D_V><<<(unsigned)grid, 256, CQ::SMEM, st>>>(m.q128, m.do128, m.k64, m.v64, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     kernel_event(1, st);
@@ -493,10 +675,10 @@ cudaError_t run_bwd(const BwdParams &p, cudaStream_t st) {
 }
 
 template <typename T>
-cudaError_t dispatch_bwd(const BwdParams &p, cudaStream_t st) {
-    if (p.d_qk == 64 && p.d_v == 64) return run_bwd<T, 64, 64, 64>(p, st);
-    if (p.d_qk == 128 && p.d_v == 128) return run_bwd<T, 128, 128, 32>(p, st);
-    if (p.d_qk == 192 && p.d_v == 128) return run_bwd<T, 192, 128, 32>(p, st);
+cudaError_t dispatch_bwd(const BwdParams &p, const BwdMaps &m, cudaStream_t st) {
+    if (p.d_qk == 64 && p.d_v == 64) return run_bwd<T, 64, 64>(p, m, st);
+    if (p.d_qk == 128 && p.d_v == 128) return run_bwd<T, 128, 128>(p, m, st);
+    if (p.d_qk == 192 && p.d_v == 128) return run_bwd<T, 192, 128>(p, m, st);
     return cudaErrorInvalidValue;
 }
 
@@ -506,8 +688,8 @@ bool bwd_supported(int d_qk, int d_v) {
     return (d_qk == 64 && d_v == 64) || (d_qk == 128 && d_v == 128) || (d_qk == 192 && d_v == 128);
 }
 
-cudaError_t launch_bwd(const BwdParams &p, int dtype, cudaStream_t st) {
-    return dtype == FA_DTYPE_BF16 ? dispatch_bwd<__nv_bfloat16>(p, st) : dispatch_bwd<__half>(p, st);
+cudaError_t launch_bwd(const BwdParams &p, const BwdMaps &m, int dtype, cudaStream_t st) {
+    return dtype == FA_DTYPE_BF16 ? dispatch_bwd<__nv_bfloat16>(p, m, st) : dispatch_bwd<__half>(p, m, st);
 }
 
 }  // namespace fa

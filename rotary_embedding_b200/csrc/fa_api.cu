@@ -889,7 +889,10 @@ int fa_bwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, const fa_
         return fail(FA_ERR_WORKSPACE, "workspace of %zu bytes needed", need);
     if (reinterpret_cast<uintptr_t>(workspace) & 15) return fail(FA_ERR_LAYOUT, "workspace not 16-byte aligned");
     const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)d_qk);
+    int32_t *status = status_word();
+    if (!status) return fail(FA_ERR_CUDA, "no CUDA device");
     BwdParams p{};
+    p.status = status;
     p.q = q->data;
     p.qs = s3(qd);
     p.k = k->data;
@@ -921,7 +924,23 @@ int fa_bwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, const fa_
     p.win_right = window_right;
     p.scale = sc;
     p.scale_log2 = sc * 1.4426950408889634f;
-    cudaError_t e = launch_bwd(p, q->dtype, static_cast<cudaStream_t>(stream));
+    // TMA maps of the tiles the kernels load; a side with no rows (s_q or s_k
+    // = 0) is never loaded (the kernels then only write zeros), and a map
+    // cannot be encoded over it
+    BwdMaps m;
+    std::memset(&m, 0, sizeof(m));
+    auto map = [&](CUtensorMap *tm, const fa_tensor *t, int rows, const char *name) {
+        return t->shape[1] == 0 ? (int)FA_OK : make_rows_map(tm, t, rows, name);
+    };
+    if ((rc = map(&m.k128, k, 128, "k"))) return rc;
+    if ((rc = map(&m.v128, v, 128, "v"))) return rc;
+    if ((rc = map(&m.q64, q, 64, "q"))) return rc;
+    if ((rc = map(&m.do64, dout, 64, "dout"))) return rc;
+    if ((rc = map(&m.q128, q, 128, "q"))) return rc;
+    if ((rc = map(&m.do128, dout, 128, "dout"))) return rc;
+    if ((rc = map(&m.k64, k, 64, "k"))) return rc;
+    if ((rc = map(&m.v64, v, 64, "v"))) return rc;
+    cudaError_t e = launch_bwd(p, m, q->dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return FA_OK;
 }

@@ -155,6 +155,7 @@ void kernel_event(int which, cudaStream_t st);
 
 // Attention backward (dq, dk, dv) over dense [b, s, h, d] tensors.
 struct BwdParams {
+    int32_t *status;   // device status word (bounded waits record timeouts here)
     const void *q;
     Strides3 qs;
     const void *k;
@@ -190,7 +191,14 @@ cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmQ, const C
                           const CUtensorMap &tmV, int dtype, int d_qk, int d_v, int mt, cudaStream_t st);
 bool decode_supported(int d_qk, int d_v, int mt);
 cudaError_t launch_simt_attn(const SimtAttnParams &p, int dtype, cudaStream_t st);
+// TMA maps of the backward kernels over the caller's [b, s, h, d] tensors,
+// named by the rows of their box: the dk/dv kernel reads 128-row K and V
+// tiles and 64-row Q and dO tiles, the dq kernel 128-row Q and dO tiles and
+// 64-row K and V tiles.
+struct BwdMaps {
+    CUtensorMap k128, v128, q64, do64, q128, do128, k64, v64;
+};
 bool bwd_supported(int d_qk, int d_v);
-cudaError_t launch_bwd(const BwdParams &p, int dtype, cudaStream_t st);
+cudaError_t launch_bwd(const BwdParams &p, const BwdMaps &m, int dtype, cudaStream_t st);
 
 }  // namespace fa
