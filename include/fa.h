@@ -271,8 +271,9 @@ int fa_fwd_varlen(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
  *  - Head dims (d_qk, d_v): 64/64, 128/128, 192/128, else
  *    FA_ERR_UNSUPPORTED.  scale <= 0 means 1/sqrt(d_qk).
  *  - workspace: caller-owned device memory of fa_bwd_workspace_size bytes,
- *    16-byte aligned (FA_ERR_WORKSPACE if smaller); it holds D_i =
- *    dout_i . out_i as fp32 [b, h_q, s_q] and is dead after the call.
+ *    16-byte aligned (FA_ERR_WORKSPACE if smaller); it holds lse_i log2(e)
+ *    and D_i = dout_i . out_i as two fp32 arrays [b, h_q, s_q rounded up to
+ *    64] and is dead after the call.
  *  - Enqueued on `stream`; returns without synchronising.  The result does
  *    not depend on scheduling (no atomics).  Errors: FA_ERR_INVALID_ARG
  *    (shapes, types, window bounds below -1, lse missing), FA_ERR_LAYOUT,

@@ -40,37 +40,58 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Four floats from shared memory, not moved across other memory operations
-// (keeps the elementwise loop from hoisting every tile value into registers).
-__device__ __forceinline__ float4 lds4(const float *p) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(smem_addr(p))
+// Untiled bulk copy global -> shared (16-byte aligned, size a multiple of
+// 16), completing on `bar` like a TMA tile load.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
                  : "memory");
-    return v;
 }
+
+// Register split of the backward kernels (384 threads launched at 168 per
+// thread): warpgroup 0 (TMA, MMA, two idle warps) down to 64, the two
+// elementwise warpgroups up to 200: 128 x 64 + 256 x 200 = 59392 <= 64512.
+constexpr int kBwdRegsLow = 64, kBwdRegsHigh = 200;
 
 // ---------------------------------------------------------------- D_i
+// Per query row i of every (batch, query head), into the workspace: lse_i
+// log2(e) and D_i = dout_i . out_i; the padding rows s_q .. s_q_pad - 1 get
+// +inf and 0 (P = 0 there).  One 16-byte chunk (8 elements) of the row per
+// lane (d_v / 8 lanes per row, 32 * 8 / d_v rows per warp, 8 warps per
+// block), the chunks' partial sums reduced with shuffles inside the row's
+// lanes.  Rows are taken in (batch, row, head) order, so a warp's loads of
+// the heads of one row are contiguous.
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_dot_kernel(const BwdParams p) {
-    const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lanes_per_row = p.d_v / 8;                   // 8, 16 or 32 (d_v 64, 128, 256)
+    const int rows_per_warp = 32 / lanes_per_row;
     const int lane = threadIdx.x & 31;
-    const int64_t rows = (int64_t)p.b * p.s_q * p.h_q;
-    if (w >= rows) return;
-    const int h = (int)(w % p.h_q);
-    const int64_t bi_i = w / p.h_q;
-    const int i = (int)(bi_i % p.s_q), bi = (int)(bi_i / p.s_q);
-    const T *o = static_cast<const T *>(p.out) + bi * p.os.b + (int64_t)i * p.os.s + h * p.os.h;
-    const T *d = static_cast<const T *>(p.dout) + bi * p.dos.b + (int64_t)i * p.dos.s + h * p.dos.h;
+    const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int64_t rowg = w * rows_per_warp + lane / lanes_per_row;
+    const int chunk = lane % lanes_per_row;
+    const int64_t rows = (int64_t)p.b * p.s_q_pad * p.h_q;
+    const int h = (int)(rowg % p.h_q);
+    const int64_t bi_i = rowg / p.h_q;
+    const int i = (int)(bi_i % p.s_q_pad), bi = (int)(bi_i / p.s_q_pad);
+    const bool real = rowg < rows && i < p.s_q;
     float acc = 0.f;
-    for (int t = lane * 2; t < p.d_v; t += 64)
-        acc += Elem<T>::to_f(o[t]) * Elem<T>::to_f(d[t]) + Elem<T>::to_f(o[t + 1]) * Elem<T>::to_f(d[t + 1]);
+    if (real) {
+        const T *o = static_cast<const T *>(p.out) + bi * p.os.b + (int64_t)i * p.os.s + h * p.os.h;
+        const T *d = static_cast<const T *>(p.dout) + bi * p.dos.b + (int64_t)i * p.dos.s + h * p.dos.h;
+        float fo[8], fd[8];
+        unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(o) + chunk), fo);
+        unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(d) + chunk), fd);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) p.dsum[((int64_t)bi * p.h_q + h) * p.s_q + i] = acc;
+        for (int t = 0; t < 8; ++t) acc = fmaf(fo[t], fd[t], acc);
+    }
+    for (int off = lanes_per_row / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (rowg < rows && chunk == 0) {
+        const int64_t at = ((int64_t)bi * p.h_q + h) * p.s_q_pad + i;
+        p.lsum[at] = real ? p.lse[((int64_t)bi * p.h_q + h) * p.s_q + i] * kLog2e : INFINITY;
+        p.dsum[at] = acc;
+    }
 }
-
 
 // ---------------------------------------------------------------- dk, dv
 constexpr int kBK = 128;   // keys per dk/dv CTA (the MMA M)
@@ -103,7 +124,7 @@ struct DkdvCfg {
 };
 
 template <typename T, int D_QK, int D_V>
-__global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(384, 1) bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK,
                                                           const __grid_constant__ CUtensorMap tmV,
                                                           const __grid_constant__ CUtensorMap tmQ,
                                                           const __grid_constant__ CUtensorMap tmDO,
@@ -117,7 +138,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
     uint8_t *sStage = sV + C::VBYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sStage + ST * C::STAGE);
     uint64_t *kv_full = bars;              // 1
-    uint64_t *full = kv_full + 1;          // ST: Q, dO (TMA) and lse / D (the producer warp's 32 lanes)
+    uint64_t *full = kv_full + 1;          // ST: Q, dO (TMA) and lse / D (bulk copies)
     uint64_t *empty = full + ST;           // ST
     uint64_t *s_full = empty + ST;         // S^T, dP^T of the tile complete
     uint64_t *s_free = s_full + 1;         // ... read into registers
@@ -162,12 +183,12 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
         for (int s = 0; s < ST; ++s) {
-            mbar_init(&full[s], 1 + 32);
+            mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(s_free, 4);
-        mbar_init(p_full, 4);
+        mbar_init(s_free, 8);
+        mbar_init(p_full, 8);
         mbar_init(pd_done, 1);
         fence_barrier_init();
     }
@@ -181,44 +202,36 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
 
+    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kBwdRegsLow) : "memory");
     if (warp == 0) {
-        // ------------------------------------------------ producer: TMA tiles; lse and D by all lanes
-        if (n_tiles > 0) {
-            if (lane == 0) {
-                tma_prefetch_desc(&tmK);
-                tma_prefetch_desc(&tmV);
-                tma_prefetch_desc(&tmQ);
-                tma_prefetch_desc(&tmDO);
-                mbar_arrive_expect_tx(kv_full, C::KBYTES + C::VBYTES);
+        // ------------------------------------------------ producer: TMA tiles and the lse / D runs
+        if (lane == 0 && n_tiles > 0) {
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmDO);
+            mbar_arrive_expect_tx(kv_full, C::KBYTES + C::VBYTES);
 #pragma unroll
-                for (int c = 0; c < D_QK / 64; ++c) tma_load_4d(sK + c * C::KBOX, &tmK, kv_full, c * 64, hk, j0, bi);
+            for (int c = 0; c < D_QK / 64; ++c) tma_load_4d(sK + c * C::KBOX, &tmK, kv_full, c * 64, hk, j0, bi);
 #pragma unroll
-                for (int c = 0; c < D_V / 64; ++c) tma_load_4d(sV + c * C::KBOX, &tmV, kv_full, c * 64, hk, j0, bi);
-            }
+            for (int c = 0; c < D_V / 64; ++c) tma_load_4d(sV + c * C::KBOX, &tmV, kv_full, c * 64, hk, j0, bi);
             for (int u = 0; u < n_tiles; ++u) {
                 const int st = u % ST;
                 if (u >= ST && !mbar_wait(&empty[st], ((u / ST) - 1) & 1, p.status)) break;
                 const int hq = hk * p.g + u / n_qt;
                 const int i0 = (qt0 + u % n_qt) * kBQ;
                 uint8_t *stage = sStage + st * C::STAGE;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[st], C::QBYTES + C::DOBYTES);
+                mbar_arrive_expect_tx(&full[st], C::QBYTES + C::DOBYTES + 2 * kBQ * 4);
 #pragma unroll
-                    for (int c = 0; c < D_QK / 64; ++c)
-                        tma_load_4d(stage + c * C::QBOX, &tmQ, &full[st], c * 64, hq, i0, bi);
+                for (int c = 0; c < D_QK / 64; ++c)
+                    tma_load_4d(stage + c * C::QBOX, &tmQ, &full[st], c * 64, hq, i0, bi);
 #pragma unroll
-                    for (int c = 0; c < D_V / 64; ++c)
-                        tma_load_4d(stage + C::QBYTES + c * C::QBOX, &tmDO, &full[st], c * 64, hq, i0, bi);
-                }
-                // rows past s_q: lse = +inf makes P = 0 there
-                float *ld = reinterpret_cast<float *>(stage + C::OFF_LD);
-                for (int t = lane; t < kBQ; t += 32) {
-                    const int i = i0 + t;
-                    const int64_t row = ((int64_t)bi * p.h_q + hq) * s_q + i;
-                    ld[t] = i < s_q ? p.lse[row] * kLog2e : INFINITY;
-                    ld[kBQ + t] = i < s_q ? p.dsum[row] : 0.f;
-                }
-                mbar_arrive(&full[st]);
+                for (int c = 0; c < D_V / 64; ++c)
+                    tma_load_4d(stage + C::QBYTES + c * C::QBOX, &tmDO, &full[st], c * 64, hq, i0, bi);
+                // the tile's 64 rows are one aligned run of each workspace array
+                const int64_t run = ((int64_t)bi * p.h_q + hq) * p.s_q_pad + i0;
+                bulk_load(stage + C::OFF_LD, p.lsum + run, kBQ * 4, &full[st]);
+                bulk_load(stage + C::OFF_LD + kBQ * 4, p.dsum + run, kBQ * 4, &full[st]);
             }
         }
     } else if (warp == 1) {
@@ -228,36 +241,41 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
             const uint32_t idesc_s = tc::idesc_f16(bf16, kBK, kBQ, false);
             const uint32_t idesc_dv = tc::idesc_f16(bf16, kBK, D_V, true);
             const uint32_t idesc_dk = tc::idesc_f16(bf16, kBK, D_QK, true);
-            const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aS = smem_addr(sStage);
+            // descriptors of the first k-step of each operand; a k-step (and a
+            // stage) only moves the start address field (16-byte units)
+            const uint64_t dK0 = tc::smem_desc(smem_addr(sK), 16, 1024);
+            const uint64_t dV0 = tc::smem_desc(smem_addr(sV), 16, 1024);
+            const uint64_t dS0 = tc::smem_desc(smem_addr(sStage), 16, 1024);            // Q / dO, K-major
+            const uint64_t dM0 = tc::smem_desc(smem_addr(sStage), C::QBOX, 1024);        // Q / dO, MN-major
             bool ok = mbar_wait(kv_full, 0, p.status);
             // S^T = K Q^T and dP^T = V dO^T (K-major operands)
             auto issue_sdp = [&](int u) {
-                const uint32_t q = aS + (u % ST) * C::STAGE, o = q + C::QBYTES;
+                const uint64_t q = dS0 + (uint64_t)(((u % ST) * C::STAGE) >> 4), o = q + (uint64_t)(C::QBYTES >> 4);
                 if (leader) {
 #pragma unroll
                     for (int k = 0; k < D_QK / 16; ++k)
-                        tc::mma_ss(tmem + C::T_S, tc::smem_desc(aK + (k >> 2) * C::KBOX + (k & 3) * 32, 16, 1024),
-                                   tc::smem_desc(q + (k >> 2) * C::QBOX + (k & 3) * 32, 16, 1024), idesc_s, k > 0);
+                        tc::mma_ss(tmem + C::T_S, dK0 + (uint64_t)(((k >> 2) * C::KBOX + (k & 3) * 32) >> 4),
+                                   q + (uint64_t)(((k >> 2) * C::QBOX + (k & 3) * 32) >> 4), idesc_s, k > 0);
 #pragma unroll
                     for (int k = 0; k < D_V / 16; ++k)
-                        tc::mma_ss(tmem + C::T_DP, tc::smem_desc(aV + (k >> 2) * C::KBOX + (k & 3) * 32, 16, 1024),
-                                   tc::smem_desc(o + (k >> 2) * C::QBOX + (k & 3) * 32, 16, 1024), idesc_s, k > 0);
+                        tc::mma_ss(tmem + C::T_DP, dV0 + (uint64_t)(((k >> 2) * C::KBOX + (k & 3) * 32) >> 4),
+                                   o + (uint64_t)(((k >> 2) * C::QBOX + (k & 3) * 32) >> 4), idesc_s, k > 0);
                     tc::commit(s_full);
                 }
                 __syncwarp();
             };
             // dV += P^T dO and dK += dS^T Q (P^T, dS^T from TMEM; dO, Q as MN-major B)
             auto issue_acc = [&](int u) {
-                const uint32_t q = aS + (u % ST) * C::STAGE, o = q + C::QBYTES;
+                const uint64_t q = dM0 + (uint64_t)(((u % ST) * C::STAGE) >> 4), o = q + (uint64_t)(C::QBYTES >> 4);
                 if (leader) {
 #pragma unroll
                     for (int k = 0; k < kBQ / 16; ++k)
-                        tc::mma_ts(tmem + C::T_DV, tmem + C::T_P + k * 8, tc::smem_desc(o + k * 16 * 128, C::QBOX, 1024),
-                                   idesc_dv, (u > 0 || k > 0) ? 1u : 0u);
+                        tc::mma_ts(tmem + C::T_DV, tmem + C::T_P + k * 8, o + (uint64_t)(k * 16 * 128 / 16), idesc_dv,
+                                   (u > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
                     for (int k = 0; k < kBQ / 16; ++k)
-                        tc::mma_ts(tmem + C::T_DK, tmem + C::T_DS + k * 8, tc::smem_desc(q + k * 16 * 128, C::QBOX, 1024),
-                                   idesc_dk, (u > 0 || k > 0) ? 1u : 0u);
+                        tc::mma_ts(tmem + C::T_DK, tmem + C::T_DS + k * 8, q + (uint64_t)(k * 16 * 128 / 16), idesc_dk,
+                                   (u > 0 || k > 0) ? 1u : 0u);
                     tc::commit(&empty[u % ST]);
                     tc::commit(pd_done);
                 }
@@ -280,7 +298,10 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
             }
         }
     } else if (warp >= 4) {
-        // ------------------------------------------------ elementwise warpgroup: key row j = TMEM lane
+        // ------------------------------------------------ elementwise warpgroups: key row j = TMEM lane,
+        // warpgroup hf takes query columns [32 hf, 32 hf + 32) of every tile
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kBwdRegsHigh) : "memory");
+        const int hf = (warp - 4) >> 2;
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
@@ -293,16 +314,16 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
         if (p.win_right >= 0) i_min = max(i_min, (int64_t)j - p.win_right - off);
         if (p.win_left >= 0) i_max = min(i_max, (int64_t)j + p.win_left - off);
         if (!key_valid) i_max = -1;
+        // as 32-bit bounds (clamped to the query rows, which fit 32 bits)
+        const int i_min32 = (int)min(i_min, (int64_t)s_q), i_max32 = (int)max(i_max, (int64_t)-1);
         const float c = p.scale_log2;
         bool ok = true;
         for (int u = 0; u < n_tiles && ok; ++u) {
             if (!(ok = mbar_wait(s_full, u & 1, p.status))) break;
             tc::fence_after_sync();
-            uint32_t sr[2][32], dr[2][32];
-            tc::ld32(tmem + lane_addr + C::T_S, sr[0]);
-            tc::ld32(tmem + lane_addr + C::T_S + 32, sr[1]);
-            tc::ld32(tmem + lane_addr + C::T_DP, dr[0]);
-            tc::ld32(tmem + lane_addr + C::T_DP + 32, dr[1]);
+            uint32_t sr[32], dr[32];
+            tc::ld32(tmem + lane_addr + C::T_S + 32 * hf, sr);
+            tc::ld32(tmem + lane_addr + C::T_DP + 32 * hf, dr);
             tc::wait_ld();
             tc::fence_before_sync();
             __syncwarp();
@@ -314,43 +335,45 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
                 if (!(ok = mbar_wait(pd_done, (u - 1) & 1, p.status))) break;
                 tc::fence_after_sync();
             }
-            const float *ld = reinterpret_cast<const float *>(sStage + st * C::STAGE + C::OFF_LD);
-            const int64_t i0 = (int64_t)(qt0 + u % n_qt) * kBQ;
-            const bool all_vis = i0 >= i_min && i0 + kBQ - 1 <= i_max;
-            // 16 query columns at a time: P^T and dS^T as 16-bit pairs
+            const float *ld = reinterpret_cast<const float *>(sStage + st * C::STAGE + C::OFF_LD) + 32 * hf;
+            const int i0 = (qt0 + u % n_qt) * kBQ + 32 * hf;   // this warpgroup's first query
+            uint32_t pp[16], pd[16];
+            // P^T = 2^(s c - L), dS^T = P^T (dP^T - D); tiles on a mask edge
+            // (masked = true) zero the pairs no mask admits
+            auto math = [&](auto masked) {
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                const int h = qq >> 1, e0 = (qq & 1) * 16;
-                float Lq[16], Dq[16];
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 L = *reinterpret_cast<const float4 *>(ld + e);
+                    const float4 D = *reinterpret_cast<const float4 *>(ld + kBQ + e);
+                    const float lv[4] = {L.x, L.y, L.z, L.w}, dv4[4] = {D.x, D.y, D.z, D.w};
 #pragma unroll
-                for (int e = 0; e < 16; e += 4) {
-                    const float4 l4 = lds4(ld + 16 * qq + e), d4 = lds4(ld + kBQ + 16 * qq + e);
-                    Lq[e] = l4.x; Lq[e + 1] = l4.y; Lq[e + 2] = l4.z; Lq[e + 3] = l4.w;
-                    Dq[e] = d4.x; Dq[e + 1] = d4.y; Dq[e + 2] = d4.z; Dq[e + 3] = d4.w;
-                }
-                uint32_t pp[8], pd[8];
-#pragma unroll
-                for (int e = 0; e < 16; e += 2) {
-                    const int qc = 16 * qq + e;
-                    float p0 = ex2(fmaf(__uint_as_float(sr[h][e0 + e]), c, -Lq[e]));
-                    float p1 = ex2(fmaf(__uint_as_float(sr[h][e0 + e + 1]), c, -Lq[e + 1]));
-                    if (!all_vis) {
-                        if (i0 + qc < i_min || i0 + qc > i_max) p0 = 0.f;
-                        if (i0 + qc + 1 < i_min || i0 + qc + 1 > i_max) p1 = 0.f;
+                    for (int t = 0; t < 4; t += 2) {
+                        float p0 = ex2(fmaf(__uint_as_float(sr[e + t]), c, -lv[t]));
+                        float p1 = ex2(fmaf(__uint_as_float(sr[e + t + 1]), c, -lv[t + 1]));
+                        if (decltype(masked)::value) {
+                            const int q = i0 + e + t;
+                            if (q < i_min32 || q > i_max32) p0 = 0.f;
+                            if (q + 1 < i_min32 || q + 1 > i_max32) p1 = 0.f;
+                        }
+                        pp[(e + t) >> 1] = Elem<T>::pack2(p0, p1);
+                        pd[(e + t) >> 1] = Elem<T>::pack2(p0 * (__uint_as_float(dr[e + t]) - dv4[t]),
+                                                          p1 * (__uint_as_float(dr[e + t + 1]) - dv4[t + 1]));
                     }
-                    pp[e >> 1] = Elem<T>::pack2(p0, p1);
-                    pd[e >> 1] = Elem<T>::pack2(p0 * (__uint_as_float(dr[h][e0 + e]) - Dq[e]),
-                                                p1 * (__uint_as_float(dr[h][e0 + e + 1]) - Dq[e + 1]));
                 }
-                tc::st8(tmem + lane_addr + C::T_P + 8 * qq, pp);
-                tc::st8(tmem + lane_addr + C::T_DS + 8 * qq, pd);
-            }
+            };
+            if (i0 >= i_min32 && i0 + 31 <= i_max32)
+                math(std::integral_constant<bool, false>());
+            else
+                math(std::integral_constant<bool, true>());
+            tc::st16(tmem + lane_addr + C::T_P + 16 * hf, pp);
+            tc::st16(tmem + lane_addr + C::T_DS + 16 * hf, pd);
             tc::wait_st();
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
         }
-        // ------------------------------------------------ epilogue: dv = dV, dk = scale dK
+        // ------------------------------------------------ epilogue: dv = dV, dk = scale dK (32-column
+        // chunks alternate between the two warpgroups)
         const bool have = n_tiles > 0;
         if (have && ok) ok = mbar_wait(pd_done, (n_tiles - 1) & 1, p.status);
         tc::fence_after_sync();
@@ -358,6 +381,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dkdv_kernel(const __grid_constant_
         T *dkrow = static_cast<T *>(p.dk) + bi * p.dks.b + (int64_t)j * p.dks.s + hk * p.dks.h;
 #pragma unroll
         for (int h = 0; h < (D_V + D_QK) / 32; ++h) {
+            if ((h & 1) != hf) continue;
             const bool is_v = h < D_V / 32;
             const int col = is_v ? h * 32 : (h - D_V / 32) * 32;
             uint32_t orr[32];
@@ -411,7 +435,7 @@ struct DqCfg {
 };
 
 template <typename T, int D_QK, int D_V>
-__global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ,
+__global__ void __launch_bounds__(384, 1) bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                         const __grid_constant__ CUtensorMap tmDO,
                                                         const __grid_constant__ CUtensorMap tmK,
                                                         const __grid_constant__ CUtensorMap tmV,
@@ -458,8 +482,8 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
             mbar_init(&empty[s], 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(s_free, 4);
-        mbar_init(p_full, 4);
+        mbar_init(s_free, 8);
+        mbar_init(p_full, 8);
         mbar_init(ds_done, 1);
         fence_barrier_init();
     }
@@ -473,6 +497,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
     const uint32_t tmem = *tmem_slot;
     constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
 
+    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kBwdRegsLow) : "memory");
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0 && n_kt > 0) {
@@ -504,32 +529,35 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
             const bool leader = tc::elect_one();
             const uint32_t idesc_s = tc::idesc_f16(bf16, kDqBM, kDqBN, false);
             const uint32_t idesc_dq = tc::idesc_f16(bf16, kDqBM, D_QK, true);
-            const uint32_t aQ = smem_addr(sQ), aDO = smem_addr(sDO), aS = smem_addr(sStage);
+            const uint64_t dQ0 = tc::smem_desc(smem_addr(sQ), 16, 1024);
+            const uint64_t dO0 = tc::smem_desc(smem_addr(sDO), 16, 1024);
+            const uint64_t dS0 = tc::smem_desc(smem_addr(sStage), 16, 1024);            // K / V, K-major
+            const uint64_t dM0 = tc::smem_desc(smem_addr(sStage), C::KBOX, 1024);        // K, MN-major
             bool ok = mbar_wait(q_full, 0, p.status);
             // S = Q K^T and dP = dO V^T
             auto issue_sdp = [&](int u) {
-                const uint32_t kk = aS + (u % ST) * C::STAGE, vv = kk + C::KBYTES;
+                const uint64_t kk = dS0 + (uint64_t)(((u % ST) * C::STAGE) >> 4), vv = kk + (uint64_t)(C::KBYTES >> 4);
                 if (leader) {
 #pragma unroll
                     for (int k = 0; k < D_QK / 16; ++k)
-                        tc::mma_ss(tmem + C::T_S, tc::smem_desc(aQ + (k >> 2) * C::QBOX + (k & 3) * 32, 16, 1024),
-                                   tc::smem_desc(kk + (k >> 2) * C::KBOX + (k & 3) * 32, 16, 1024), idesc_s, k > 0);
+                        tc::mma_ss(tmem + C::T_S, dQ0 + (uint64_t)(((k >> 2) * C::QBOX + (k & 3) * 32) >> 4),
+                                   kk + (uint64_t)(((k >> 2) * C::KBOX + (k & 3) * 32) >> 4), idesc_s, k > 0);
 #pragma unroll
                     for (int k = 0; k < D_V / 16; ++k)
-                        tc::mma_ss(tmem + C::T_DP, tc::smem_desc(aDO + (k >> 2) * C::QBOX + (k & 3) * 32, 16, 1024),
-                                   tc::smem_desc(vv + (k >> 2) * C::KBOX + (k & 3) * 32, 16, 1024), idesc_s, k > 0);
+                        tc::mma_ss(tmem + C::T_DP, dO0 + (uint64_t)(((k >> 2) * C::QBOX + (k & 3) * 32) >> 4),
+                                   vv + (uint64_t)(((k >> 2) * C::KBOX + (k & 3) * 32) >> 4), idesc_s, k > 0);
                     tc::commit(s_full);
                 }
                 __syncwarp();
             };
             // dQ += dS K (dS from TMEM, K as MN-major B)
             auto issue_dq = [&](int u) {
-                const uint32_t kk = aS + (u % ST) * C::STAGE;
+                const uint64_t kk = dM0 + (uint64_t)(((u % ST) * C::STAGE) >> 4);
                 if (leader) {
 #pragma unroll
                     for (int k = 0; k < kDqBN / 16; ++k)
-                        tc::mma_ts(tmem + C::T_DQ, tmem + C::T_DS + k * 8, tc::smem_desc(kk + k * 16 * 128, C::KBOX, 1024),
-                                   idesc_dq, (u > 0 || k > 0) ? 1u : 0u);
+                        tc::mma_ts(tmem + C::T_DQ, tmem + C::T_DS + k * 8, kk + (uint64_t)(k * 16 * 128 / 16), idesc_dq,
+                                   (u > 0 || k > 0) ? 1u : 0u);
                     tc::commit(&empty[u % ST]);
                     tc::commit(ds_done);
                 }
@@ -552,7 +580,10 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
             }
         }
     } else if (warp >= 4) {
-        // ------------------------------------------------ elementwise warpgroup: query row i = TMEM lane
+        // ------------------------------------------------ elementwise warpgroups: query row i = TMEM lane,
+        // warpgroup hf takes key columns [32 hf, 32 hf + 32) of every tile
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kBwdRegsHigh) : "memory");
+        const int hf = (warp - 4) >> 2;
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
@@ -561,19 +592,19 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
         int64_t fv, lv;
         visible_keys(i, N, s_q, p.causal, p.win_left, p.win_right, fv, lv);
         if (!row_valid) lv = -1;
-        const int64_t row = ((int64_t)bi * p.h_q + hq) * s_q + (row_valid ? i : 0);
-        const float L = row_valid ? p.lse[row] * kLog2e : INFINITY;
-        const float Dd = row_valid ? p.dsum[row] : 0.f;
+        // as 32-bit bounds (keys fit 32 bits)
+        const int fv32 = (int)min(fv, (int64_t)N), lv32 = (int)max(lv, (int64_t)-1);
+        const int64_t at = ((int64_t)bi * p.h_q + hq) * p.s_q_pad + (row_valid ? i : 0);
+        const float L = row_valid ? p.lsum[at] : INFINITY;
+        const float Dd = row_valid ? p.dsum[at] : 0.f;
         const float c = p.scale_log2;
         bool ok = true;
         for (int u = 0; u < n_kt && ok; ++u) {
             if (!(ok = mbar_wait(s_full, u & 1, p.status))) break;
             tc::fence_after_sync();
-            uint32_t sr[2][32], dr[2][32];
-            tc::ld32(tmem + lane_addr + C::T_S, sr[0]);
-            tc::ld32(tmem + lane_addr + C::T_S + 32, sr[1]);
-            tc::ld32(tmem + lane_addr + C::T_DP, dr[0]);
-            tc::ld32(tmem + lane_addr + C::T_DP + 32, dr[1]);
+            uint32_t sr[32], dr[32];
+            tc::ld32(tmem + lane_addr + C::T_S + 32 * hf, sr);
+            tc::ld32(tmem + lane_addr + C::T_DP + 32 * hf, dr);
             tc::wait_ld();
             tc::fence_before_sync();
             __syncwarp();
@@ -583,37 +614,41 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
                 if (!(ok = mbar_wait(ds_done, (u - 1) & 1, p.status))) break;
                 tc::fence_after_sync();
             }
-            const int64_t jt = (int64_t)(kt0 + u) * kDqBN;
-            const bool all_vis = jt >= fv && jt + kDqBN - 1 <= lv;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t pd[16];
+            const int jt = (kt0 + u) * kDqBN + 32 * hf;   // this warpgroup's first key
+            uint32_t pd[16];
+            // dS = 2^(s c - L) (dP - D); tiles on a mask edge (masked = true)
+            // zero the pairs no mask admits
+            auto math = [&](auto masked) {
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const int64_t jj = jt + 32 * h + e;
-                    float p0 = ex2(fmaf(__uint_as_float(sr[h][e]), c, -L));
-                    float p1 = ex2(fmaf(__uint_as_float(sr[h][e + 1]), c, -L));
-                    if (!all_vis) {
-                        if (jj < fv || jj > lv) p0 = 0.f;
-                        if (jj + 1 < fv || jj + 1 > lv) p1 = 0.f;
+                    float p0 = ex2(fmaf(__uint_as_float(sr[e]), c, -L));
+                    float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), c, -L));
+                    if (decltype(masked)::value) {
+                        if (jt + e < fv32 || jt + e > lv32) p0 = 0.f;
+                        if (jt + e + 1 < fv32 || jt + e + 1 > lv32) p1 = 0.f;
                     }
-                    pd[e >> 1] = Elem<T>::pack2(p0 * (__uint_as_float(dr[h][e]) - Dd),
-                                                p1 * (__uint_as_float(dr[h][e + 1]) - Dd));
+                    pd[e >> 1] = Elem<T>::pack2(p0 * (__uint_as_float(dr[e]) - Dd), p1 * (__uint_as_float(dr[e + 1]) - Dd));
                 }
-                tc::st16(tmem + lane_addr + C::T_DS + 16 * h, pd);
-            }
+            };
+            if (jt >= fv32 && jt + 31 <= lv32)
+                math(std::integral_constant<bool, false>());
+            else
+                math(std::integral_constant<bool, true>());
+            tc::st16(tmem + lane_addr + C::T_DS + 16 * hf, pd);
             tc::wait_st();
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
         }
-        // ------------------------------------------------ epilogue: dq = scale dQ
+        // ------------------------------------------------ epilogue: dq = scale dQ (32-column chunks
+        // alternate between the two warpgroups)
         const bool have = n_kt > 0;
         if (have && ok) ok = mbar_wait(ds_done, (n_kt - 1) & 1, p.status);
         tc::fence_after_sync();
         T *dqrow = static_cast<T *>(p.dq) + bi * p.dqs.b + (int64_t)i * p.dqs.s + hq * p.dqs.h;
 #pragma unroll
         for (int h = 0; h < D_QK / 32; ++h) {
+            if ((h & 1) != hf) continue;
             uint32_t orr[32];
             if (have) {
                 tc::ld32(tmem + lane_addr + C::T_DQ + h * 32, orr);
@@ -641,11 +676,21 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(const __grid_constant__ 
     }
 }
 
+// The register split must fit in what the block is launched with (384
+// threads x the kernel's count), or setmaxnreg.inc would never return.
+template <typename K>
+bool regs_fit(K kernel) {
+    cudaFuncAttributes a;
+    if (cudaFuncGetAttributes(&a, kernel) != cudaSuccess) return false;
+    return a.numRegs * 384 >= 128 * kBwdRegsLow + 256 * kBwdRegsHigh;
+}
+
 template <typename T, int D_QK, int D_V>
 cudaError_t run_bwd(const BwdParams &p, const BwdMaps &m, cudaStream_t st) {
-    const int64_t rows = (int64_t)p.b * p.s_q * p.h_q;
+    const int64_t rows = (int64_t)p.b * p.s_q_pad * p.h_q;
     if (rows > 0) {
-        bwd_dot_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);
+        const int64_t rows_per_block = 8 * (32 / (D_V / 8));
+        bwd_dot_kernel<T><<<(unsigned)((rows + rows_per_block - 1) / rows_per_block), 256, 0, st>>>(p);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -657,7 +702,8 @@ cudaError_t run_bwd(const BwdParams &p, const BwdMaps &m, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         const int64_t grid = (int64_t)((p.s_k + kBK - 1) / kBK) * p.h_kv * p.b;
         if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
-        bwd_dkdv_kernel<T, D_QK, D_V><<<(unsigned)grid, 256, CK::SMEM, st>>>(m.k128, m.v128, m.q64, m.do64, p);
+        if (!regs_fit(bwd_dkdv_kernel<T, D_QK, D_V>)) return cudaErrorInvalidConfiguration;
+        bwd_dkdv_kernel<T, D_QK, D_V><<<(unsigned)grid, 384, CK::SMEM, st>>>(m.k128, m.v128, m.q64, m.do64, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (p.s_q > 0) {
@@ -667,7 +713,8 @@ cudaError_t run_bwd(const BwdParams &p, const BwdMaps &m, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         const int64_t grid = (int64_t)((p.s_q + kDqBM - 1) / kDqBM) * p.h_q * p.b;
         if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
-        bwd_dq_kernel<T, D_QK, D_V><<<(unsigned)grid, 256, CQ::SMEM, st>>>(m.q128, m.do128, m.k64, m.v64, p);
+        if (!regs_fit(bwd_dq_kernel<T, D_QK, D_V>)) return cudaErrorInvalidConfiguration;
+        bwd_dq_kernel<T, D_QK, D_V><<<(unsigned)grid, 384, CQ::SMEM, st>>>(m.q128, m.do128, m.k64, m.v64, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     kernel_event(1, st);

@@ -841,7 +841,9 @@ int fa_bwd_workspace_size(const fa_tensor *q, size_t *bytes) {
     Dims4 qd;
     int rc;
     if ((rc = check_tensor(q, "q", 4, 0, &qd))) return rc;
-    *bytes = align_up((size_t)(qd.n[0] * qd.n[1] * qd.n[2]) * sizeof(float), 256);
+    // lse * log2(e) and D_i, each [b, h_q, s_q rounded up to 64]
+    const size_t rows = (size_t)qd.n[0] * qd.n[2] * (size_t)((qd.n[1] + 63) / 64 * 64);
+    *bytes = 2 * align_up(rows * sizeof(float), 256);
     return FA_OK;
 }
 
@@ -904,7 +906,9 @@ int fa_bwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, const fa_
     p.dout = dout->data;
     p.dos = s3(dod);
     p.lse = lse;
-    p.dsum = static_cast<float *>(workspace);
+    p.s_q_pad = (int)((s_q + 63) / 64 * 64);
+    p.lsum = static_cast<float *>(workspace);
+    p.dsum = reinterpret_cast<float *>(static_cast<char *>(workspace) + need / 2);
     p.dq = dq->data;
     p.dqs = s3(dqd);
     p.dk = dk->data;

@@ -167,7 +167,11 @@ struct BwdParams {
     const void *dout;
     Strides3 dos;
     const float *lse;  // [b, h_q, s_q], natural log, from the forward
-    float *dsum;       // [b, h_q, s_q] workspace: D_i = dout_i . out_i
+    // workspace, [b, h_q, s_q_pad] each (s_q rounded up to 64 rows, so that
+    // every 64-row tile of a (batch, head) is one aligned 256-byte run):
+    float *lsum;       //   lse_i * log2(e) (+inf on the padding rows)
+    float *dsum;       //   D_i = dout_i . out_i (0 on the padding rows)
+    int s_q_pad;
     void *dq;
     Strides3 dqs;
     void *dk;

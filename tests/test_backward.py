@@ -46,7 +46,8 @@ def test_bwd_host_validation():
     assert call(wl=-2) == fa.FA_ERR_INVALID_ARG                                              # window bound
     assert call(wsb=16) == fa.FA_ERR_WORKSPACE                                               # workspace
     assert call(kk=q.to(torch.bfloat16)) == fa.FA_ERR_INVALID_ARG                            # dtype mix
-    assert fa.fa_bwd_workspace_size(q) == 256
+    # lse * log2(e) and D_i, each fp32 [b, h_q, s_q rounded up to 64 rows], 256-byte aligned
+    assert fa.fa_bwd_workspace_size(q) == 2 * 1 * 2 * 64 * 4
 
 
 def _case(seed, b, s_q, s_k, h_q, h_kv, d_qk, d_v, dtype):
