@@ -2,18 +2,21 @@
 // ROCm/flash-attention PR #99: COS/SIN (seqlen, rotary_dim/2), SEQLEN_OFFSET
 // as an int or one value per batch entry, INTERLEAVED, CONJUGATE, IS_VARLEN).
 //
-// A block takes RT consecutive rows and HG heads (RT * HG * d / 8 <= 2048
-// 16-byte chunks; HG < h only when one row's heads exceed that).  Its 256
-// threads copy the chunks into shared memory with cp.async (no registers held
-// while they are in flight) while the first RT threads find the rows'
-// positions; after a barrier the block stages the cos/sin rows of those
-// positions in shared memory as fp32 (one parallel round trip to L2, where
-// the tables stay); after a second barrier every thread rotates its chunks
-// from shared memory and stores them.  Every load precedes the barriers that
-// precede every store, so out may be x itself.  CONJUGATE rotates by the negated angle (sin replaced by -sin).
-// Positions: batched row i of entry b at offsets[b] + i; packed rows of
-// sequence k (rows cu[k] .. cu[k+1]-1) at offsets[k] + R - cu[k].  Rows of a
-// packed tensor outside every sequence are copied unchanged.
+// A pure stream: every thread takes one unit of one (row, head) -- with
+// half-split pairs a 16-byte chunk of the first half and its partner chunk
+// rotary_dim/2 further on, with interleaved pairs one chunk holding four
+// pairs -- loads it with 16-byte loads straight into registers, reads the
+// row's cos/sin values (a few hundred bytes per row, served from L1/L2),
+// rotates in fp32 with the shared RoPE pair formula, rounds, and stores.
+// There is no staging and no block-wide barrier, so every SM keeps as many
+// loads in flight as its resident threads allow.  Dims past rotary_dim are
+// copied (out of place) or left untouched (in place, out = x).  CONJUGATE
+// rotates by the negated angle (sin replaced by -sin).  Positions: batched
+// row i of entry b at offsets[b] + i; packed rows of sequence k (rows
+// cu[k] .. cu[k+1]-1) at offsets[k] + R - cu[k] (the sequence found by
+// binary search); rows of a packed tensor outside every sequence are copied
+// unchanged; a row whose position falls outside the table is left as it is
+// and the device status records it.
 #include <algorithm>
 
 #include "fa_common.cuh"
@@ -22,14 +25,6 @@
 namespace fa {
 
 constexpr int kRotThreads = 256;
-constexpr int kRotChunks = 2048;                       // 16-byte chunks per block (32 KB)
-constexpr int kRotPer = kRotChunks / kRotThreads;       // chunks per thread
-constexpr int kRotMaxRows = 16;                        // rows per block
-
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)), "l"(gmem_src)
-                 : "memory");
-}
 
 // n / d for 0 <= n < 2^31 by a multiply-high and a shift (the round-up
 // reciprocal method of Granlund and Montgomery, "Division by invariant
@@ -50,172 +45,184 @@ __device__ __forceinline__ int fdiv(int n, const FastDiv &f) {
     return (int)((__umulhi((uint32_t)n, f.m) + (uint32_t)n) >> f.s);
 }
 
+// Units of a (row, head): MODE 0 interleaved (chunk c, four pairs; then the
+// chunks past rotary_dim), MODE 1 half-split with rotary_dim/2 a multiple of
+// 8 (chunk c < r/16 and its partner; then the chunks past rotary_dim), MODE 2
+// half-split otherwise (pair j < r/2, i.e. elements j and j + r/2, one by
+// one; then the elements past rotary_dim).  Every unit owns what it writes,
+// so out may be x.
 struct RotaryGrid {
-    int RT, HG, per_row, total;
-    FastDiv div_row, div_ck, div_s;
+    int units;            // units per (row, head)
+    int rot_units;        // units that rotate (the rest copy)
+    int copy_from;        // MODE 1: first chunk of the copied dims
+    int in_place;         // out == x: copy units are skipped
+    int cs_vec;           // cos/sin rows 16-byte aligned: vector loads
+    FastDiv div_units, div_h, div_s;
 };
 
-// Pairing: 0 interleaved; 1 half-split with rotary_dim/2 a multiple of 8 (the
-// partner of a chunk is a chunk); 2 half-split otherwise (element partners).
-template <typename T, int PAIR>
-__global__ void __launch_bounds__(kRotThreads, 4) rotary_kernel(RotaryParams p, RotaryGrid g) {
-    extern __shared__ uint4 sbuf[];                    // [kRotChunks]
-    __shared__ int64_t pos_s[kRotMaxRows];
-    __shared__ __align__(16) float cs_s[kRotMaxRows][128];
-    __shared__ __align__(16) float sn_s[kRotMaxRows][128];
-    const int tid = threadIdx.x;
-    const int R0 = blockIdx.x * g.RT;
-    const int h0 = blockIdx.y * g.HG;
-    const int ck = p.d >> 3;
-    const int half = p.r >> 1;
-    constexpr bool inter = PAIR == 0;
+// Table row of packed / batched row R (kOutside: a packed row outside every
+// sequence).
+constexpr int64_t kOutside = INT64_MIN;
+__device__ __forceinline__ int64_t row_position(const RotaryParams &p, const RotaryGrid &g, int R) {
+    if (!p.cu_seqlens) {
+        const int rb = fdiv(R, g.div_s), ri = R - rb * p.s;
+        return (int64_t)(p.offsets ? __ldg(p.offsets + rb) : p.offset_scalar) + ri;
+    }
+    if (R < __ldg(p.cu_seqlens) || R >= __ldg(p.cu_seqlens + p.n_seqs)) return kOutside;
+    int lo = 0, hi = p.n_seqs;   // cu[lo] <= R < cu[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(p.cu_seqlens + mid) <= R) lo = mid; else hi = mid;
+    }
+    return (int64_t)(p.offsets ? __ldg(p.offsets + lo) : p.offset_scalar) + R - __ldg(p.cu_seqlens + lo);
+}
 
-    // the block's chunks into shared memory: chunk idx = (row r, head hl, chunk c)
-    for (int idx = tid; idx < g.total; idx += kRotThreads) {
-        const int r = fdiv(idx, g.div_row), rem = idx - r * g.per_row;
-        const int hl = fdiv(rem, g.div_ck), c = rem - hl * ck;
-        const int R = R0 + r, h = h0 + hl;
-        if (R >= p.rows || h >= p.h) continue;
+// NV consecutive table values from column j0 of a row, as fp32 times
+// `sign` (-1 for the conjugate); columns at or past `ncols` read as 0.
+template <typename T, int NV>
+__device__ __forceinline__ void table_vals(const T *row, int j0, int ncols, bool vec, float sign, float *v) {
+    if (NV == 8 && vec && j0 + 8 <= ncols) {
+        float f[8];
+        unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(row + j0)), f);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = sign * f[k];
+    } else {
+#pragma unroll
+        for (int k = 0; k < NV; ++k) v[k] = j0 + k < ncols ? sign * Elem<T>::to_f(row[j0 + k]) : 0.f;
+    }
+}
+
+template <typename T, int MODE>
+__global__ void __launch_bounds__(kRotThreads) rotary_kernel(RotaryParams p, RotaryGrid g) {
+    const int64_t total = (int64_t)p.rows * p.h * g.units;
+    for (int64_t item = (int64_t)blockIdx.x * kRotThreads + threadIdx.x; item < total;
+         item += (int64_t)gridDim.x * kRotThreads) {
+        const int it = (int)item;   // total < 2^31 (checked at launch)
+        const int rh = fdiv(it, g.div_units), u = it - rh * g.units;
+        const int R = fdiv(rh, g.div_h), h = rh - R * p.h;
+        const bool rot = u < g.rot_units && p.r > 0;
+        if (!rot && g.in_place) continue;   // dims past rotary_dim stay as they are
         const int rb = fdiv(R, g.div_s), ri = R - rb * p.s;
         const T *xrow = static_cast<const T *>(p.x) + rb * p.xs.b + ri * p.xs.s + (int64_t)h * p.xs.h;
-        cp_async16(&sbuf[idx], reinterpret_cast<const uint4 *>(xrow) + c);
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-
-    // positions of the block's rows: -1 = outside every packed sequence (copy),
-    // -2 = outside the table (left as it is)
-    if (tid < g.RT) {
-        const int R = R0 + tid;
-        int64_t pos = -1;
-        if (R < p.rows) {
-            if (!p.cu_seqlens) {
-                const int rb = fdiv(R, g.div_s), ri = R - rb * p.s;
-                pos = (int64_t)(p.offsets ? __ldg(p.offsets + rb) : p.offset_scalar) + ri;
-            } else if (R >= __ldg(p.cu_seqlens) && R < __ldg(p.cu_seqlens + p.n_seqs)) {
-                int lo = 0, hi = p.n_seqs;   // cu[lo] <= R < cu[hi]
-                while (hi - lo > 1) {
-                    const int mid = (lo + hi) >> 1;
-                    if (__ldg(p.cu_seqlens + mid) <= R) lo = mid; else hi = mid;
-                }
-                pos = (int64_t)(p.offsets ? __ldg(p.offsets + lo) : p.offset_scalar) + R - __ldg(p.cu_seqlens + lo);
-            }
-            if (p.r > 0 && pos != -1 && (pos < 0 || pos >= p.cs_rows)) {
-                if (blockIdx.y == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
-                pos = -2;
-            }
-        }
-        pos_s[tid] = pos;
-    }
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    __syncthreads();
-    if (p.r > 0) {
-        const float sgn = p.conjugate ? -1.f : 1.f;
-        for (int idx = tid; idx < g.RT * half; idx += kRotThreads) {
-            const int r = idx / half, j = idx - r * half;
-            const int64_t pos = pos_s[r];
-            if (pos < 0) continue;
-            cs_s[r][j] = Elem<T>::to_f(static_cast<const T *>(p.cos)[pos * p.cs_row + j]);
-            sn_s[r][j] = sgn * Elem<T>::to_f(static_cast<const T *>(p.sin)[pos * p.cs_row + j]);
-        }
-    }
-    __syncthreads();
-
-    for (int idx = tid; idx < g.total; idx += kRotThreads) {
-        const int r = fdiv(idx, g.div_row), rem = idx - r * g.per_row;
-        const int hl = fdiv(rem, g.div_ck), c = rem - hl * ck;
-        const int R = R0 + r, h = h0 + hl;
-        if (R >= p.rows || h >= p.h) continue;
-        const int64_t pos = pos_s[r];
-        if (pos == -2) continue;
-        const int rb = fdiv(R, g.div_s), ri = R - rb * p.s;
         T *orow = static_cast<T *>(p.out) + rb * p.os.b + ri * p.os.s + (int64_t)h * p.os.h;
-        const uint4 raw = sbuf[idx];
-        const int t0 = 8 * c;
-        if (p.r == 0 || pos < 0 || t0 >= p.r) {
-            reinterpret_cast<uint4 *>(orow)[c] = raw;   // unrotated dims: bit copy
+        int64_t pos = 0;
+        if (p.r > 0) {
+            pos = row_position(p, g, R);
+            if (pos != kOutside && (pos < 0 || pos >= p.cs_rows)) {
+                if (h == 0 && u == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
+                continue;                      // the whole row is left as it is
+            }
+        }
+        if (!rot || pos == kOutside) {
+            // a copied chunk: past rotary_dim, or a packed row outside every sequence
+            if (MODE == 1) {
+                if (!rot) {
+                    const int c = g.copy_from + (u - g.rot_units);
+                    reinterpret_cast<uint4 *>(orow)[c] = __ldg(reinterpret_cast<const uint4 *>(xrow) + c);
+                } else if (!g.in_place) {
+                    const int c0 = u, c1 = u + (p.r >> 4);
+                    reinterpret_cast<uint4 *>(orow)[c0] = __ldg(reinterpret_cast<const uint4 *>(xrow) + c0);
+                    reinterpret_cast<uint4 *>(orow)[c1] = __ldg(reinterpret_cast<const uint4 *>(xrow) + c1);
+                }
+            } else if (MODE == 2) {
+                if (!rot) {
+                    const int t = p.r + (u - g.rot_units);
+                    orow[t] = xrow[t];
+                } else if (!g.in_place) {
+                    orow[u] = xrow[u];
+                    orow[u + (p.r >> 1)] = xrow[u + (p.r >> 1)];
+                }
+            } else if (!g.in_place) {
+                const int c = rot ? u : g.copy_from + (u - g.rot_units);
+                reinterpret_cast<uint4 *>(orow)[c] = __ldg(reinterpret_cast<const uint4 *>(xrow) + c);
+            }
             continue;
         }
-        float f[8], q[8], cv[8], sv[8];
-        unpack8<T>(raw, f);
-        if (PAIR == 0) {
-            // pairs (2j, 2j+1), j = t0/2 .. t0/2 + 3
-            const float4 c4 = *reinterpret_cast<const float4 *>(&cs_s[r][t0 >> 1]);
-            const float4 s4 = *reinterpret_cast<const float4 *>(&sn_s[r][t0 >> 1]);
-            const float ca[4] = {c4.x, c4.y, c4.z, c4.w}, sa[4] = {s4.x, s4.y, s4.z, s4.w};
+        const T *crow = static_cast<const T *>(p.cos) + pos * p.cs_row;
+        const T *srow = static_cast<const T *>(p.sin) + pos * p.cs_row;
+        const float sgn = p.conjugate ? -1.f : 1.f;
+        if (MODE == 1) {
+            // pairs (j, j + r/2): chunk u of the first half and its partner
+            const int half = p.r >> 1;
+            const int c0 = u, c1 = u + (half >> 3);
+            float a[8], b[8], cs[8], sn[8];
+            unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(xrow) + c0), a);
+            unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(xrow) + c1), b);
+            table_vals<T, 8>(crow, 8 * u, half, g.cs_vec, 1.f, cs);
+            table_vals<T, 8>(srow, 8 * u, half, g.cs_vec, sgn, sn);
+            float ya[8], yb[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                q[k] = f[k ^ 1];
-                cv[k] = ca[k >> 1];
-                sv[k] = sa[k >> 1];
+                ya[k] = rope_elem(a[k], b[k], cs[k], sn[k], true);
+                yb[k] = rope_elem(b[k], a[k], cs[k], sn[k], false);
             }
-        } else if (PAIR == 1) {
-            // pairs (j, j + r/2): the chunk's angles are j0 .. j0 + 7
-            const int pc = (t0 < half) ? c + (half >> 3) : c - (half >> 3);
-            unpack8<T>(sbuf[idx - c + pc], q);
-            const int j0 = t0 < half ? t0 : t0 - half;
-            const float4 c0 = *reinterpret_cast<const float4 *>(&cs_s[r][j0]);
-            const float4 c1 = *reinterpret_cast<const float4 *>(&cs_s[r][j0 + 4]);
-            const float4 s0 = *reinterpret_cast<const float4 *>(&sn_s[r][j0]);
-            const float4 s1 = *reinterpret_cast<const float4 *>(&sn_s[r][j0 + 4]);
-            cv[0] = c0.x; cv[1] = c0.y; cv[2] = c0.z; cv[3] = c0.w;
-            cv[4] = c1.x; cv[5] = c1.y; cv[6] = c1.z; cv[7] = c1.w;
-            sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
-            sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+            reinterpret_cast<uint4 *>(orow)[c0] = pack8<T>(ya);
+            reinterpret_cast<uint4 *>(orow)[c1] = pack8<T>(yb);
+        } else if (MODE == 0) {
+            // pairs (2j, 2j+1) inside chunk u: angles 4u .. 4u+3
+            float f[8], cs[4], sn[4], y[8];
+            unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(xrow) + u), f);
+            table_vals<T, 4>(crow, 4 * u, p.r >> 1, false, 1.f, cs);
+            table_vals<T, 4>(srow, 4 * u, p.r >> 1, false, sgn, sn);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int t = 8 * u + k;
+                y[k] = t < p.r ? rope_elem(f[k], f[k ^ 1], cs[k >> 1], sn[k >> 1], (k & 1) == 0) : f[k];
+            }
+            reinterpret_cast<uint4 *>(orow)[u] = pack8<T>(y);
         } else {
-            const T *hrow = reinterpret_cast<const T *>(&sbuf[idx - c]);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int t = t0 + k;
-                const int tt = t < p.r ? t : 0;
-                const int partner = tt < half ? tt + half : tt - half;
-                const int j = tt < half ? tt : tt - half;
-                q[k] = Elem<T>::to_f(hrow[partner]);
-                cv[k] = cs_s[r][j];
-                sv[k] = sn_s[r][j];
-            }
+            // half-split with rotary_dim/2 not a multiple of 8: pair u, elements u and u + r/2
+            const int half = p.r >> 1;
+            const float a = Elem<T>::to_f(xrow[u]), b = Elem<T>::to_f(xrow[u + half]);
+            const float cs = Elem<T>::to_f(crow[u]), sn = sgn * Elem<T>::to_f(srow[u]);
+            orow[u] = Elem<T>::from_f(rope_elem(a, b, cs, sn, true));
+            orow[u + half] = Elem<T>::from_f(rope_elem(b, a, cs, sn, false));
         }
-        const bool first_half = t0 < half;   // half-split: every element of the chunk on one side
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int t = t0 + k;
-            if (t < p.r) {
-                const bool first = PAIR == 0 ? (k & 1) == 0 : (PAIR == 1 ? first_half : t < half);
-                f[k] = rope_elem(f[k], q[k], cv[k], sv[k], first);
-            }
-        }
-        reinterpret_cast<uint4 *>(orow)[c] = pack8<T>(f);
     }
 }
 
 cudaError_t launch_rotary(const RotaryParams &p, int dtype, cudaStream_t st) {
     if (p.rows == 0 || p.h == 0) return cudaSuccess;
     const int ck = p.d / 8;
+    const int half = p.r / 2;
+    // rotary_dim 0 (a plain copy) takes the chunk units of MODE 0
+    const int mode = (p.interleaved || p.r == 0) ? 0 : (half % 8 == 0 ? 1 : 2);
     RotaryGrid g;
-    g.HG = std::min(p.h, std::max(1, kRotChunks / ck));   // heads per block
-    g.RT = std::max(1, std::min(kRotMaxRows, kRotChunks / (g.HG * ck)));
-    g.per_row = g.HG * ck;
-    g.total = g.RT * g.per_row;
-    g.div_row = make_fastdiv((uint32_t)g.per_row);
-    g.div_ck = make_fastdiv((uint32_t)ck);
-    g.div_s = make_fastdiv((uint32_t)std::max(p.s, 1));
-    const int64_t gx = (p.rows + g.RT - 1) / g.RT;
-    const int64_t gy = (p.h + g.HG - 1) / g.HG;
-    // rows are indexed with 32-bit arithmetic in the kernel (fdiv needs < 2^31)
-    if (p.rows > 0x7fffffff - kRotMaxRows || gx > 0x7fffffff || gy > 65535) return cudaErrorInvalidConfiguration;
-    dim3 grid((unsigned)gx, (unsigned)gy);
-    const size_t smem = (size_t)kRotChunks * 16;
-    const int pair = p.interleaved ? 0 : ((p.r / 2) % 8 == 0 ? 1 : 2);
-    kernel_event(0, st);
-#define FA_ROT_LAUNCH(T, P)                                                                              \
-    do {                                                                                                 \
-        cudaFuncSetAttribute(rotary_kernel<T, P>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-        rotary_kernel<T, P><<<grid, kRotThreads, smem, st>>>(p, g);                                      \
-    } while (0)
-    if (dtype == FA_DTYPE_F16) {
-        if (pair == 0) FA_ROT_LAUNCH(__half, 0); else if (pair == 1) FA_ROT_LAUNCH(__half, 1); else FA_ROT_LAUNCH(__half, 2);
+    g.in_place = p.out == p.x;
+    if (mode == 1) {
+        g.rot_units = half / 8;
+        g.copy_from = p.r / 8;
+        g.units = g.rot_units + (ck - g.copy_from);
+    } else if (mode == 0) {
+        g.rot_units = p.r > 0 ? (p.r + 7) / 8 : 0;
+        g.copy_from = g.rot_units;
+        g.units = ck;
     } else {
-        if (pair == 0) FA_ROT_LAUNCH(__nv_bfloat16, 0);
-        else if (pair == 1) FA_ROT_LAUNCH(__nv_bfloat16, 1);
+        g.rot_units = half;           // pairs
+        g.copy_from = p.r;            // elements past rotary_dim
+        g.units = half + (p.d - p.r);
+    }
+    const int elem = 2;
+    g.cs_vec = p.cos && (reinterpret_cast<uintptr_t>(p.cos) % 16 == 0) &&
+               (reinterpret_cast<uintptr_t>(p.sin) % 16 == 0) && ((p.cs_row * elem) % 16 == 0);
+    g.div_units = make_fastdiv((uint32_t)std::max(g.units, 1));
+    g.div_h = make_fastdiv((uint32_t)p.h);
+    g.div_s = make_fastdiv((uint32_t)std::max(p.s, 1));
+    const int64_t total = (int64_t)p.rows * p.h * g.units;
+    if (total == 0) return cudaSuccess;
+    // item indices are 32-bit in the kernel (fdiv needs < 2^31)
+    if (total > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    // enough blocks to fill every SM several times; the grid-stride loop covers the rest
+    const int64_t want = (total + kRotThreads - 1) / kRotThreads;
+    const int64_t cap = (int64_t)sm_count() * 64;
+    dim3 grid((unsigned)std::min(want, cap));
+    kernel_event(0, st);
+#define FA_ROT_LAUNCH(T, M) rotary_kernel<T, M><<<grid, kRotThreads, 0, st>>>(p, g)
+    if (dtype == FA_DTYPE_F16) {
+        if (mode == 0) FA_ROT_LAUNCH(__half, 0); else if (mode == 1) FA_ROT_LAUNCH(__half, 1); else FA_ROT_LAUNCH(__half, 2);
+    } else {
+        if (mode == 0) FA_ROT_LAUNCH(__nv_bfloat16, 0);
+        else if (mode == 1) FA_ROT_LAUNCH(__nv_bfloat16, 1);
         else FA_ROT_LAUNCH(__nv_bfloat16, 2);
     }
 #undef FA_ROT_LAUNCH
