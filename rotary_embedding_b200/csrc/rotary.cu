@@ -2,14 +2,15 @@
 // ROCm/flash-attention PR #99: COS/SIN (seqlen, rotary_dim/2), SEQLEN_OFFSET
 // as an int or one value per batch entry, INTERLEAVED, CONJUGATE, IS_VARLEN).
 //
-// A pure stream: every thread takes one unit of one (row, head) -- with
-// half-split pairs a 16-byte chunk of the first half and its partner chunk
-// rotary_dim/2 further on, with interleaved pairs one chunk holding four
-// pairs -- loads it with 16-byte loads straight into registers, reads the
-// row's cos/sin values (a few hundred bytes per row, served from L1/L2),
-// rotates in fp32 with the shared RoPE pair formula, rounds, and stores.
-// There is no staging and no block-wide barrier, so every SM keeps as many
-// loads in flight as its resident threads allow.  Dims past rotary_dim are
+// A pure stream: every thread takes one unit of up to four heads of one row
+// -- with half-split pairs a 16-byte chunk of the first half and its partner
+// chunk rotary_dim/2 further on, with interleaved pairs one chunk holding
+// four pairs -- issues the 16-byte loads of all those heads at once, reads
+// the row's cos/sin values once for them (a few hundred bytes per row,
+// served from L1/L2), rotates in fp32 with the shared RoPE pair formula,
+// rounds, and stores.  There is no staging and no block-wide barrier; one
+// wave of resident blocks walks the items with a grid-stride loop, each
+// thread keeping up to 128 bytes of loads in flight.  Dims past rotary_dim are
 // copied (out of place) or left untouched (in place, out = x).  CONJUGATE
 // rotates by the negated angle (sin replaced by -sin).  Positions: batched
 // row i of entry b at offsets[b] + i; packed rows of sequence k (rows
@@ -92,49 +93,59 @@ __device__ __forceinline__ void table_vals(const T *row, int j0, int ncols, bool
     }
 }
 
-template <typename T, int MODE>
+// One item = unit u of heads hg HU .. hg HU + HU - 1 of row R: the heads
+// share the row's position and cos/sin values, and the thread issues the
+// 16-byte loads of all its heads before it waits on any of them (HU x 32
+// bytes in flight per thread in MODE 1).
+template <typename T, int MODE, int HU>
 __global__ void __launch_bounds__(kRotThreads) rotary_kernel(RotaryParams p, RotaryGrid g) {
-    const int64_t total = (int64_t)p.rows * p.h * g.units;
+    const int n_hg = p.h / HU;
+    const int64_t total = (int64_t)p.rows * n_hg * g.units;
     for (int64_t item = (int64_t)blockIdx.x * kRotThreads + threadIdx.x; item < total;
          item += (int64_t)gridDim.x * kRotThreads) {
         const int it = (int)item;   // total < 2^31 (checked at launch)
         const int rh = fdiv(it, g.div_units), u = it - rh * g.units;
-        const int R = fdiv(rh, g.div_h), h = rh - R * p.h;
+        const int R = fdiv(rh, g.div_h), h0 = (rh - R * n_hg) * HU;
         const bool rot = u < g.rot_units && p.r > 0;
         if (!rot && g.in_place) continue;   // dims past rotary_dim stay as they are
         const int rb = fdiv(R, g.div_s), ri = R - rb * p.s;
-        const T *xrow = static_cast<const T *>(p.x) + rb * p.xs.b + ri * p.xs.s + (int64_t)h * p.xs.h;
-        T *orow = static_cast<T *>(p.out) + rb * p.os.b + ri * p.os.s + (int64_t)h * p.os.h;
+        const T *xrow0 = static_cast<const T *>(p.x) + rb * p.xs.b + ri * p.xs.s + (int64_t)h0 * p.xs.h;
+        T *orow0 = static_cast<T *>(p.out) + rb * p.os.b + ri * p.os.s + (int64_t)h0 * p.os.h;
         int64_t pos = 0;
         if (p.r > 0) {
             pos = row_position(p, g, R);
             if (pos != kOutside && (pos < 0 || pos >= p.cs_rows)) {
-                if (h == 0 && u == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
+                if (h0 == 0 && u == 0) record_status(p.status, FA_ERR_DEVICE_PRECONDITION);
                 continue;                      // the whole row is left as it is
             }
         }
         if (!rot || pos == kOutside) {
-            // a copied chunk: past rotary_dim, or a packed row outside every sequence
-            if (MODE == 1) {
-                if (!rot) {
-                    const int c = g.copy_from + (u - g.rot_units);
+            // copied chunks: past rotary_dim, or a packed row outside every sequence
+#pragma unroll
+            for (int k = 0; k < HU; ++k) {
+                const T *xrow = xrow0 + (int64_t)k * p.xs.h;
+                T *orow = orow0 + (int64_t)k * p.os.h;
+                if (MODE == 1) {
+                    if (!rot) {
+                        const int c = g.copy_from + (u - g.rot_units);
+                        reinterpret_cast<uint4 *>(orow)[c] = __ldg(reinterpret_cast<const uint4 *>(xrow) + c);
+                    } else if (!g.in_place) {
+                        const int c0 = u, c1 = u + (p.r >> 4);
+                        reinterpret_cast<uint4 *>(orow)[c0] = __ldg(reinterpret_cast<const uint4 *>(xrow) + c0);
+                        reinterpret_cast<uint4 *>(orow)[c1] = __ldg(reinterpret_cast<const uint4 *>(xrow) + c1);
+                    }
+                } else if (MODE == 2) {
+                    if (!rot) {
+                        const int t = p.r + (u - g.rot_units);
+                        orow[t] = xrow[t];
+                    } else if (!g.in_place) {
+                        orow[u] = xrow[u];
+                        orow[u + (p.r >> 1)] = xrow[u + (p.r >> 1)];
+                    }
+                } else if (!g.in_place) {
+                    const int c = rot ? u : g.copy_from + (u - g.rot_units);
                     reinterpret_cast<uint4 *>(orow)[c] = __ldg(reinterpret_cast<const uint4 *>(xrow) + c);
-                } else if (!g.in_place) {
-                    const int c0 = u, c1 = u + (p.r >> 4);
-                    reinterpret_cast<uint4 *>(orow)[c0] = __ldg(reinterpret_cast<const uint4 *>(xrow) + c0);
-                    reinterpret_cast<uint4 *>(orow)[c1] = __ldg(reinterpret_cast<const uint4 *>(xrow) + c1);
                 }
-            } else if (MODE == 2) {
-                if (!rot) {
-                    const int t = p.r + (u - g.rot_units);
-                    orow[t] = xrow[t];
-                } else if (!g.in_place) {
-                    orow[u] = xrow[u];
-                    orow[u + (p.r >> 1)] = xrow[u + (p.r >> 1)];
-                }
-            } else if (!g.in_place) {
-                const int c = rot ? u : g.copy_from + (u - g.rot_units);
-                reinterpret_cast<uint4 *>(orow)[c] = __ldg(reinterpret_cast<const uint4 *>(xrow) + c);
             }
             continue;
         }
@@ -145,40 +156,95 @@ __global__ void __launch_bounds__(kRotThreads) rotary_kernel(RotaryParams p, Rot
             // pairs (j, j + r/2): chunk u of the first half and its partner
             const int half = p.r >> 1;
             const int c0 = u, c1 = u + (half >> 3);
-            float a[8], b[8], cs[8], sn[8];
-            unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(xrow) + c0), a);
-            unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(xrow) + c1), b);
+            uint4 ra[HU], rb2[HU];
+#pragma unroll
+            for (int k = 0; k < HU; ++k) {
+                const uint4 *xr = reinterpret_cast<const uint4 *>(xrow0 + (int64_t)k * p.xs.h);
+                ra[k] = __ldg(xr + c0);
+                rb2[k] = __ldg(xr + c1);
+            }
+            float cs[8], sn[8];
             table_vals<T, 8>(crow, 8 * u, half, g.cs_vec, 1.f, cs);
             table_vals<T, 8>(srow, 8 * u, half, g.cs_vec, sgn, sn);
-            float ya[8], yb[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                ya[k] = rope_elem(a[k], b[k], cs[k], sn[k], true);
-                yb[k] = rope_elem(b[k], a[k], cs[k], sn[k], false);
+            for (int k = 0; k < HU; ++k) {
+                float a[8], b[8], ya[8], yb[8];
+                unpack8<T>(ra[k], a);
+                unpack8<T>(rb2[k], b);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    ya[e] = rope_elem(a[e], b[e], cs[e], sn[e], true);
+                    yb[e] = rope_elem(b[e], a[e], cs[e], sn[e], false);
+                }
+                uint4 *orow = reinterpret_cast<uint4 *>(orow0 + (int64_t)k * p.os.h);
+                orow[c0] = pack8<T>(ya);
+                orow[c1] = pack8<T>(yb);
             }
-            reinterpret_cast<uint4 *>(orow)[c0] = pack8<T>(ya);
-            reinterpret_cast<uint4 *>(orow)[c1] = pack8<T>(yb);
         } else if (MODE == 0) {
             // pairs (2j, 2j+1) inside chunk u: angles 4u .. 4u+3
-            float f[8], cs[4], sn[4], y[8];
-            unpack8<T>(__ldg(reinterpret_cast<const uint4 *>(xrow) + u), f);
+            uint4 rx[HU];
+#pragma unroll
+            for (int k = 0; k < HU; ++k) rx[k] = __ldg(reinterpret_cast<const uint4 *>(xrow0 + (int64_t)k * p.xs.h) + u);
+            float cs[4], sn[4];
             table_vals<T, 4>(crow, 4 * u, p.r >> 1, false, 1.f, cs);
             table_vals<T, 4>(srow, 4 * u, p.r >> 1, false, sgn, sn);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int t = 8 * u + k;
-                y[k] = t < p.r ? rope_elem(f[k], f[k ^ 1], cs[k >> 1], sn[k >> 1], (k & 1) == 0) : f[k];
+            for (int k = 0; k < HU; ++k) {
+                float f[8], y[8];
+                unpack8<T>(rx[k], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int t = 8 * u + e;
+                    y[e] = t < p.r ? rope_elem(f[e], f[e ^ 1], cs[e >> 1], sn[e >> 1], (e & 1) == 0) : f[e];
+                }
+                reinterpret_cast<uint4 *>(orow0 + (int64_t)k * p.os.h)[u] = pack8<T>(y);
             }
-            reinterpret_cast<uint4 *>(orow)[u] = pack8<T>(y);
         } else {
             // half-split with rotary_dim/2 not a multiple of 8: pair u, elements u and u + r/2
             const int half = p.r >> 1;
-            const float a = Elem<T>::to_f(xrow[u]), b = Elem<T>::to_f(xrow[u + half]);
             const float cs = Elem<T>::to_f(crow[u]), sn = sgn * Elem<T>::to_f(srow[u]);
-            orow[u] = Elem<T>::from_f(rope_elem(a, b, cs, sn, true));
-            orow[u + half] = Elem<T>::from_f(rope_elem(b, a, cs, sn, false));
+#pragma unroll
+            for (int k = 0; k < HU; ++k) {
+                const T *xrow = xrow0 + (int64_t)k * p.xs.h;
+                T *orow = orow0 + (int64_t)k * p.os.h;
+                const float a = Elem<T>::to_f(xrow[u]), b = Elem<T>::to_f(xrow[u + half]);
+                orow[u] = Elem<T>::from_f(rope_elem(a, b, cs, sn, true));
+                orow[u + half] = Elem<T>::from_f(rope_elem(b, a, cs, sn, false));
+            }
         }
     }
+}
+
+template <typename T, int MODE, int HU>
+static cudaError_t run_rotary(const RotaryParams &p, const RotaryGrid &g, int64_t total, cudaStream_t st) {
+    // one wave of resident blocks; the grid-stride loop covers the rest
+    static int per_sm = 0;
+    if (per_sm == 0) {
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotary_kernel<T, MODE, HU>,
+                                                                      kRotThreads, 0);
+        if (e != cudaSuccess || per_sm < 1) per_sm = 1;
+    }
+    const int64_t want = (total + kRotThreads - 1) / kRotThreads;
+    const int64_t wave = (int64_t)sm_count() * per_sm;
+    dim3 grid((unsigned)std::min(want, wave));
+    kernel_event(0, st);
+    rotary_kernel<T, MODE, HU><<<grid, kRotThreads, 0, st>>>(p, g);
+    const cudaError_t e = cudaGetLastError();
+    kernel_event(1, st);
+    return e;
+}
+
+template <typename T, int MODE>
+static cudaError_t run_rotary_hu(const RotaryParams &p, RotaryGrid &g, cudaStream_t st) {
+    const int hu = p.h % 4 == 0 ? 4 : (p.h % 2 == 0 ? 2 : 1);
+    g.div_h = make_fastdiv((uint32_t)(p.h / hu));
+    const int64_t total = (int64_t)p.rows * (p.h / hu) * g.units;
+    if (total == 0) return cudaSuccess;
+    // item indices are 32-bit in the kernel (fdiv needs < 2^31)
+    if (total > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    if (hu == 4) return run_rotary<T, MODE, 4>(p, g, total, st);
+    if (hu == 2) return run_rotary<T, MODE, 2>(p, g, total, st);
+    return run_rotary<T, MODE, 1>(p, g, total, st);
 }
 
 cudaError_t launch_rotary(const RotaryParams &p, int dtype, cudaStream_t st) {
@@ -206,29 +272,15 @@ cudaError_t launch_rotary(const RotaryParams &p, int dtype, cudaStream_t st) {
     g.cs_vec = p.cos && (reinterpret_cast<uintptr_t>(p.cos) % 16 == 0) &&
                (reinterpret_cast<uintptr_t>(p.sin) % 16 == 0) && ((p.cs_row * elem) % 16 == 0);
     g.div_units = make_fastdiv((uint32_t)std::max(g.units, 1));
-    g.div_h = make_fastdiv((uint32_t)p.h);
     g.div_s = make_fastdiv((uint32_t)std::max(p.s, 1));
-    const int64_t total = (int64_t)p.rows * p.h * g.units;
-    if (total == 0) return cudaSuccess;
-    // item indices are 32-bit in the kernel (fdiv needs < 2^31)
-    if (total > 0x7fffffff) return cudaErrorInvalidConfiguration;
-    // enough blocks to fill every SM several times; the grid-stride loop covers the rest
-    const int64_t want = (total + kRotThreads - 1) / kRotThreads;
-    const int64_t cap = (int64_t)sm_count() * 64;
-    dim3 grid((unsigned)std::min(want, cap));
-    kernel_event(0, st);
-#define FA_ROT_LAUNCH(T, M) rotary_kernel<T, M><<<grid, kRotThreads, 0, st>>>(p, g)
     if (dtype == FA_DTYPE_F16) {
-        if (mode == 0) FA_ROT_LAUNCH(__half, 0); else if (mode == 1) FA_ROT_LAUNCH(__half, 1); else FA_ROT_LAUNCH(__half, 2);
-    } else {
-        if (mode == 0) FA_ROT_LAUNCH(__nv_bfloat16, 0);
-        else if (mode == 1) FA_ROT_LAUNCH(__nv_bfloat16, 1);
-        else FA_ROT_LAUNCH(__nv_bfloat16, 2);
+        if (mode == 0) return run_rotary_hu<__half, 0>(p, g, st);
+        if (mode == 1) return run_rotary_hu<__half, 1>(p, g, st);
+        return run_rotary_hu<__half, 2>(p, g, st);
     }
-#undef FA_ROT_LAUNCH
-    const cudaError_t e = cudaGetLastError();
-    kernel_event(1, st);
-    return e;
+    if (mode == 0) return run_rotary_hu<__nv_bfloat16, 0>(p, g, st);
+    if (mode == 1) return run_rotary_hu<__nv_bfloat16, 1>(p, g, st);
+    return run_rotary_hu<__nv_bfloat16, 2>(p, g, st);
 }
 
 }  // namespace fa

@@ -77,6 +77,26 @@ def test_rotary_batched(cuda_device, dtype, d, r, inter, conj):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("h", [2, 6, 12])
+@pytest.mark.parametrize("inter", [False, True])
+@pytest.mark.parametrize("in_place", [False, True])
+def test_rotary_head_groups(cuda_device, h, inter, in_place):
+    # heads are taken in groups of 4, 2 or 1 per thread; partial rotary_dim
+    # exercises the copied chunks of every group
+    b, s, d, r = 2, 23, 128, 64
+    x, cos, sin = _inputs((b, s, h, d), "bf16", r, 80, seed=100 + h)
+    offs = torch.tensor([3, 40], dtype=torch.int32)
+    xd = x.to(cuda_device)
+    out = fa.fa_rotary(xd, cos.to(cuda_device), sin.to(cuda_device), offs.to(cuda_device), r, inter, False,
+                       out=xd if in_place else None)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == 0
+    ref = _expect(x, cos, sin, offs.numpy(), r, inter, False, "bf16")
+    assert ulp_distance(out.cpu(), ref).max() <= 1
+    assert torch.equal(out.cpu()[..., r:], x[..., r:])
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 def test_rotary_scalar_offset_in_place_and_transposed(cuda_device, dtype):
     b, s, h, d, r = 2, 19, 4, 128, 96
