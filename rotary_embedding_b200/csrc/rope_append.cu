@@ -33,7 +33,7 @@ template <typename T>
 __global__ void __launch_bounds__(kRopeThreads, 8) rope_append_kernel(RopeAppendParams p) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (p.zero_word && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.zero_word = 0;
-    __shared__ float cs_s[128], sn_s[128];
+    __shared__ __align__(16) float cs_s[128], sn_s[128];
     const int rows = max(1, max(p.q_rot ? p.s_q : 0, p.s_new));
     const int b = blockIdx.x / rows, i = blockIdx.x % rows;
     const int ck = p.d_qk >> 3, cv = p.d_v >> 3;
@@ -119,6 +119,45 @@ __global__ void __launch_bounds__(kRopeThreads, 8) rope_append_kernel(RopeAppend
         }
         float f[8], pf[8];
         unpack8<T>(raw[u], f);
+        if (t0 + 8 <= p.r && (inter || chunk_partner)) {
+            // a whole chunk of pairs (the common case): straight-line code,
+            // the chunk's cos/sin values read as float4 from shared memory
+            float c8[8], s8[8];
+            if (inter) {
+                // pairs (2j, 2j+1), j = t0/2 .. t0/2 + 3
+                const float4 cv = *reinterpret_cast<const float4 *>(cs_s + (t0 >> 1));
+                const float4 sv = *reinterpret_cast<const float4 *>(sn_s + (t0 >> 1));
+                c8[0] = c8[1] = cv.x; c8[2] = c8[3] = cv.y; c8[4] = c8[5] = cv.z; c8[6] = c8[7] = cv.w;
+                s8[0] = s8[1] = sv.x; s8[2] = s8[3] = sv.y; s8[4] = s8[5] = sv.z; s8[6] = s8[7] = sv.w;
+#pragma unroll
+                for (int k = 0; k < 8; k += 2) {
+                    const float a = f[k], b = f[k + 1];
+                    f[k] = rope_elem(a, b, c8[k], s8[k], true);
+                    f[k + 1] = rope_elem(b, a, c8[k], s8[k], false);
+                }
+            } else {
+                // pairs (j, j + r/2): the chunk lies wholly in one half
+                unpack8<T>(praw[u], pf);
+                const bool first = t0 < half;
+                const int j0 = first ? t0 : t0 - half;
+                const float4 *cq = reinterpret_cast<const float4 *>(cs_s + j0);
+                const float4 *sq = reinterpret_cast<const float4 *>(sn_s + j0);
+                const float4 c0 = cq[0], c1 = cq[1], s0 = sq[0], s1 = sq[1];
+                c8[0] = c0.x; c8[1] = c0.y; c8[2] = c0.z; c8[3] = c0.w;
+                c8[4] = c1.x; c8[5] = c1.y; c8[6] = c1.z; c8[7] = c1.w;
+                s8[0] = s0.x; s8[1] = s0.y; s8[2] = s0.z; s8[3] = s0.w;
+                s8[4] = s1.x; s8[5] = s1.y; s8[6] = s1.z; s8[7] = s1.w;
+                if (first) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) f[k] = rope_elem(f[k], pf[k], c8[k], s8[k], true);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) f[k] = rope_elem(f[k], pf[k], c8[k], s8[k], false);
+                }
+            }
+            reinterpret_cast<uint4 *>(dst)[c] = pack8<T>(f);
+            continue;
+        }
         if (inter) {
 #pragma unroll
             for (int k = 0; k < 8; ++k) pf[k] = f[k ^ 1];
