@@ -14,11 +14,14 @@ extern "C" {
 #endif
 
 /*
- * fa_testing_set_prefill_tiles -- query tiles per CTA of the tcgen05
- * prefill / dense attention kernels for every following fa_fwd*,
- * fa_fwd_varlen and prefill-path fa_kvcache_fwd* call.
+ * fa_testing_set_prefill_tiles -- which tcgen05 prefill / dense attention
+ * kernel runs every following fa_fwd*, fa_fwd_varlen and prefill-path
+ * fa_kvcache_fwd* call.
  *   tiles  0 = the planner's choice (the default), 1 = the one-tile kernel,
- *          2 = the two-tile kernel; anything else is FA_ERR_INVALID_ARG.
+ *          2 = the two-tile kernel on pairs of query tiles, 3 = the two-tile
+ *          kernel on one query tile with its key range split between the two
+ *          softmax warpgroups (packed sequences run as 2); anything else is
+ *          FA_ERR_INVALID_ARG.
  * Process-wide and not synchronised: set it while no other thread is
  * calling the library, and set it back to 0 when done.
  */

@@ -405,8 +405,9 @@ lib.fa_testing_set_prefill_tiles.restype = ctypes.c_int
 
 def fa_testing_set_prefill_tiles(tiles: int) -> None:
     """Test hook (include/fa_testing.h): pin the prefill kernel of later calls
-    to one (1) or two (2) query tiles per CTA, or give the choice back to the
-    planner (0)."""
+    to one (1) or two (2) query tiles per CTA, to one tile with its key range
+    split between the two softmax warpgroups (3), or give the choice back to
+    the planner (0)."""
     _check(lib.fa_testing_set_prefill_tiles(int(tiles)))
 
 

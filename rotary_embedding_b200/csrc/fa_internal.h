@@ -122,6 +122,10 @@ struct PrefillParams {
     // two-tile kernel: 0 = CTA k takes query tiles 2k and 2k+1; 1 = tiles k
     // and n_q_tiles-1-k (equal causal work per CTA, for single-wave grids)
     int pair_ends;
+    // two-tile kernel: 1 = both tiles of a CTA are the same query tile, with
+    // the key range cut in two halves merged at the end (grid: one CTA per
+    // query tile)
+    int key_split;
     int win_left, win_right;  // sliding window; -1 = unbounded
     // packed sequences (varlen): grid z = sequence s with query rows
     // cu_q[s] .. cu_q[s+1]-1 and key rows cu_k[s] .. of batch entry 0;

@@ -427,7 +427,20 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
 //
 // Warps: 0 TMA, 1 MMA, 2-3 idle (warpgroup 0), 4-7 softmax of tile 0
 // (warpgroup 1), 8-11 softmax of tile 1 (warpgroup 2); warp w reaches TMEM
-// lanes 32 (w % 4) .. 32 (w % 4) + 31.  The register file is split with
+// lanes 32 (w % 4) .. 32 (w % 4) + 31.
+//
+// KSPLIT: on grids too small for two tiles per CTA, the two "tiles" of a CTA
+// are the same 128 query rows with the key range cut in two: softmax
+// warpgroup 0 takes the first half of the visible key tiles, warpgroup 1
+// the second, each with its own S, P, O, running max and sum, over one Q
+// tile.  Per step u the K tiles of both halves are loaded, then their V
+// tiles, and the MMA warp keeps the order QK_0(u+1) QK_1(u+1) PV_0(u) PV_1(u).
+// At the end the two warpgroups exchange (max, sum) per row through shared
+// memory (the unused second Q buffer) and each merges half of the output
+// columns from both O accumulators:
+//   out = (2^(m0 - m) O_0 + 2^(m1 - m) O_1) / (2^(m0 - m) l0 + 2^(m1 - m) l1).
+// The CTA count doubles against pairs of tiles, and both warpgroups stay
+// busy on every step, which pairs of causal tiles of unequal length do not.  The register file is split with
 // setmaxnreg: warpgroup 0 drops to 64 registers per thread (enough for the
 // TMA and MMA issue loops), the two softmax warpgroups rise to 216 so that a
 // whole S row stays in registers (128 x 64 + 256 x 216 = 63488, within the
@@ -459,13 +472,15 @@ struct Prefill2Cfg {
     static_assert(D_QK % 64 == 0 && D_V % 64 == 0 && D_V <= 128, "head dims");
 };
 
-template <typename T, int D_QK, int D_V>
+template <typename T, int D_QK, int D_V, bool KSPLIT>
 __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                           const __grid_constant__ CUtensorMap tmK,
                                                           const __grid_constant__ CUtensorMap tmV,
                                                           const PrefillParams p) {
     using C = Prefill2Cfg<D_QK, D_V>;
     constexpr int KST = C::KST, VST = C::VST, BN = C::BN;
+    // the split order loads two K tiles ahead of the V tiles they pair with
+    static_assert(!KSPLIT || (KST >= 2 && VST >= 2), "key-split rings");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem;                              // 2 tiles
@@ -522,7 +537,9 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
     // n_q_tiles - 1 - blk (the middle tile of an odd count pairs with an
     // empty tile past the rows); every tile index is taken exactly once
     int tile[2];
-    if (p.pair_ends) {
+    if (KSPLIT) {
+        tile[0] = tile[1] = blk;                           // one query tile, two key halves
+    } else if (p.pair_ends) {
         tile[0] = blk;
         tile[1] = p.n_q_tiles - 1 - blk > blk ? p.n_q_tiles - 1 - blk : p.n_q_tiles;
     } else {
@@ -546,6 +563,14 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         mask_from[x] = (int)max((int64_t)0, min((int64_t)N, l_first + 1));
         lo_max[x] = (int)f_last;
     }
+    if (KSPLIT) {
+        // halves kb .. mid - 1 and mid .. end - 1 (the first half holds the odd tile)
+        const int mid = kb[0] + (n_kv[0] - kb[0] + 1) / 2;
+        kb[1] = mid;
+        n_kv[0] = mid;
+    }
+    // tiles of each half (key-split mode)
+    const int n_x[2] = {n_kv[0] - kb[0], n_kv[1] - kb[1]};
     // key tiles loaded: kb0 .. n_all - 1 (the union of both tiles' ranges)
     const bool any0 = kb[0] < n_kv[0], any1 = kb[1] < n_kv[1];
     const int kb0 = any0 && any1 ? min(kb[0], kb[1]) : (any0 ? kb[0] : (any1 ? kb[1] : 0));
@@ -582,7 +607,42 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
     if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0 && n_all > kb0) {
+        if (KSPLIT && lane == 0 && n_x[0] > 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            mbar_arrive_expect_tx(q_full, C::QBYTES);
+#pragma unroll
+            for (int c = 0; c < D_QK / 64; ++c)
+                tma_load_4d(sQ + c * C::QBOX, &tmQ, q_full, c * 64, hq0, qoff + i0[0], tb);
+            // load index 2u + x for step u of half x: the K tiles of a step,
+            // then its V tiles
+            bool ok = true;
+            for (int u = 0; u < n_x[0] && ok; ++u) {
+#pragma unroll 1
+                for (int x = 0; x < 2; ++x) {
+                    if (u >= n_x[x] || !ok) continue;
+                    const int li = 2 * u + x, ks = li % KST;
+                    if (li >= KST && !(ok = mbar_wait(&k_empty[ks], ((li / KST) - 1) & 1, p.status))) break;
+                    mbar_arrive_expect_tx(&k_full[ks], C::KBYTES);
+#pragma unroll
+                    for (int c = 0; c < D_QK / 64; ++c)
+                        tma_load_4d(sK + ks * C::KBYTES + c * C::KBOX, &tmK, &k_full[ks], c * 64, hk,
+                                    koff + (kb[x] + u) * BN, tb);
+                }
+#pragma unroll 1
+                for (int x = 0; x < 2; ++x) {
+                    if (u >= n_x[x] || !ok) continue;
+                    const int li = 2 * u + x, vs = li % VST;
+                    if (li >= VST && !(ok = mbar_wait(&v_empty[vs], ((li / VST) - 1) & 1, p.status))) break;
+                    mbar_arrive_expect_tx(&v_full[vs], C::VBYTES);
+#pragma unroll
+                    for (int c = 0; c < D_V / 64; ++c)
+                        tma_load_4d(sV + vs * C::VBYTES + c * C::KBOX, &tmV, &v_full[vs], c * 64, hk,
+                                    koff + (kb[x] + u) * BN, tb);
+                }
+            }
+        } else if (!KSPLIT && lane == 0 && n_all > kb0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
@@ -611,7 +671,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         // ------------------------------------------------ MMA issuer
         // The whole warp runs the loop (waits, warp-uniform descriptors); one
         // elected lane issues the MMAs and the commits that track them.
-        if (n_all > kb0) {
+        if (KSPLIT ? n_x[0] > 0 : n_all > kb0) {
             const bool leader = tc::elect_one();
             const uint32_t idesc_qk = tc::idesc_f16(bf16, kBM, BN, false);
             const uint32_t idesc_pv = tc::idesc_f16(bf16, kBM, D_V, true);
@@ -623,10 +683,10 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             const uint64_t dV0 = tc::smem_desc(smem_addr(sV), C::KBOX, 1024);
             bool ok = mbar_wait(q_full, 0, p.status);
             auto in_range = [&](int x, int j) { return j >= kb[x] && j < n_kv[x]; };
-            // key tile j sits in stage (j - kb0) % KST / VST
-            auto issue_qk = [&](int x, int j) {
-                const uint64_t dq = dQ0 + (uint64_t)((x * C::QBYTES) >> 4);
-                const uint64_t dk = dK0 + (uint64_t)((((j - kb0) % KST) * C::KBYTES) >> 4);
+            // K tile in stage ks (key-split mode: both halves read the one Q tile)
+            auto issue_qk_s = [&](int x, int ks) {
+                const uint64_t dq = dQ0 + (uint64_t)(((KSPLIT ? 0 : x) * C::QBYTES) >> 4);
+                const uint64_t dk = dK0 + (uint64_t)((ks * C::KBYTES) >> 4);
                 const uint32_t ts = tmem + C::t_s(x);
                 if (leader) {
 #pragma unroll
@@ -639,10 +699,12 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                 }
                 __syncwarp();
             };
-            auto issue_pv = [&](int x, int j) {
-                const uint64_t dv = dV0 + (uint64_t)((((j - kb0) % VST) * C::VBYTES) >> 4);
+            // key tile j sits in stage (j - kb0) % KST / VST
+            auto issue_qk = [&](int x, int j) { issue_qk_s(x, (j - kb0) % KST); };
+            auto issue_pv_s = [&](int x, int vs, bool first) {
+                const uint64_t dv = dV0 + (uint64_t)((vs * C::VBYTES) >> 4);
                 const uint32_t to = tmem + C::t_o(x), tp = tmem + C::t_p(x);
-                const uint32_t acc0 = j > kb[x] ? 1u : 0u;
+                const uint32_t acc0 = first ? 0u : 1u;
                 if (leader) {
 #pragma unroll
                     for (int k = 0; k < BN / 16; ++k)
@@ -651,10 +713,46 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                 }
                 __syncwarp();
             };
+            auto issue_pv = [&](int x, int j) { issue_pv_s(x, (j - kb0) % VST, j == kb[x]); };
             auto commit = [&](uint64_t *bar) {
                 if (leader) tc::commit(bar);
                 __syncwarp();
             };
+            if (KSPLIT) {
+                // step u of half x: load index 2u + x (see the producer)
+                for (int x = 0; x < 2 && ok; ++x) {
+                    if (n_x[x] <= 0) continue;
+                    const int ks = x % KST;
+                    if (!(ok = mbar_wait(&k_full[ks], (x / KST) & 1, p.status))) break;
+                    tc::fence_after_sync();
+                    issue_qk_s(x, ks);
+                    commit(&k_empty[ks]);
+                }
+                for (int u = 0; u < n_x[0] && ok; ++u) {
+                    // the next scores of both halves, once S_x(u) is consumed
+#pragma unroll 1
+                    for (int x = 0; x < 2; ++x) {
+                        if (u + 1 >= n_x[x] || !ok) continue;
+                        const int li = 2 * (u + 1) + x, ks = li % KST;
+                        if (!(ok = mbar_wait(&k_full[ks], (li / KST) & 1, p.status))) break;
+                        if (!(ok = mbar_wait(&s_free[x], u & 1, p.status))) break;
+                        tc::fence_after_sync();
+                        issue_qk_s(x, ks);
+                        commit(&k_empty[ks]);
+                    }
+                    // this step's PV of both halves
+#pragma unroll 1
+                    for (int x = 0; x < 2; ++x) {
+                        if (u >= n_x[x] || !ok) continue;
+                        const int li = 2 * u + x, vs = li % VST;
+                        if (!(ok = mbar_wait(&v_full[vs], (li / VST) & 1, p.status))) break;
+                        if (!(ok = mbar_wait(&p_full[x], u & 1, p.status))) break;
+                        tc::fence_after_sync();
+                        issue_pv_s(x, vs, u == 0);
+                        commit(&v_empty[vs]);
+                    }
+                }
+            } else {
             // prologue: QK of the tiles whose range starts at the first loaded key tile
             if (ok && (ok = mbar_wait(&k_full[0], 0, p.status))) {
                 tc::fence_after_sync();
@@ -691,6 +789,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
                 }
                 if (!ok) break;
                 commit(&v_empty[vs]);
+            }
             }
         }
     } else if (warp >= 4) {
@@ -831,9 +930,11 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             tc::wait_st();
             if (p.kvcache && j == nk - 1 && j0 + BN > N) {
                 // cache rows past N_b may hold anything: zero them in the V tile
-                // (both tiles' warpgroups do it; the writes are identical)
-                const int vs = (j - kb0) % VST;
-                if (!(ok = mbar_wait(&v_full[vs], ((j - kb0) / VST) & 1, p.status))) break;
+                // (pairs: both tiles' warpgroups do it; the writes are identical;
+                // key split: only the half that holds the last tile)
+                const int li = KSPLIT ? 2 * (j - jb) + x : j - kb0;   // load index of V(j)
+                const int vs = li % VST;
+                if (!(ok = mbar_wait(&v_full[vs], (li / VST) & 1, p.status))) break;
                 uint8_t *vt = sV + vs * C::VBYTES;
                 const int first = N - j0;
                 const int n16 = (BN - first) * 8 * (D_V / 64);
@@ -869,6 +970,48 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         if (ok && nk > jb && !mbar_wait(&pv_done[x], (nk - 1 - jb) & 1, p.status)) ok = false;
         tc::fence_after_sync();
         T *orow = static_cast<T *>(p.out) + tb * p.os.b + (int64_t)(qoff + i) * p.os.s + hq * p.os.h;
+        if (KSPLIT) {
+            // exchange (max, sum) of the two key halves per row through the
+            // unused second Q buffer; both warpgroups reach the barrier once
+            float *mls = reinterpret_cast<float *>(sQ + C::QBYTES);   // [m_0 | m_1 | l_0 | l_1][128]
+            mls[x * kBM + r] = (nk > jb && l > 0.f) ? m_ref * c : -INFINITY;
+            mls[(2 + x) * kBM + r] = nk > jb ? l : 0.f;
+            tc::fence_before_sync();
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            tc::fence_after_sync();
+            const float m0 = mls[r], m1 = mls[kBM + r], l0 = mls[2 * kBM + r], l1 = mls[3 * kBM + r];
+            const float mx = fmaxf(m0, m1);
+            const float a0 = l0 > 0.f ? ex2(m0 - mx) : 0.f, a1 = l1 > 0.f ? ex2(m1 - mx) : 0.f;
+            const float lt = a0 * l0 + a1 * l1;
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            const float w0 = a0 * inv, w1 = a1 * inv;
+            // this warpgroup merges columns x d_v/2 .. (x+1) d_v/2 - 1 of both O
+            const uint32_t o_base = tmem + lane_addr;
+#pragma unroll
+            for (int h = 0; h < D_V / 64; ++h) {
+                const int col = x * (D_V / 2) + h * 32;
+                uint32_t o0[32], o1[32];
+                if (n_x[0] > 0) tc::ld32(o_base + C::t_o(0) + col, o0);
+                if (n_x[1] > 0) tc::ld32(o_base + C::t_o(1) + col, o1);
+                tc::wait_ld();
+                if (row_valid) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8) {
+                        float f[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const float v0 = n_x[0] > 0 ? __uint_as_float(o0[e + u]) * w0 : 0.f;
+                            const float v1 = n_x[1] > 0 ? __uint_as_float(o1[e + u]) * w1 : 0.f;
+                            f[u] = v0 + v1;
+                        }
+                        reinterpret_cast<uint4 *>(orow + col + e)[0] = pack8<T>(f);
+                    }
+                }
+            }
+            if (x == 0 && row_valid && p.lse)
+                p.lse[p.cu_q ? (int64_t)hq * p.total_q + qoff + i : ((int64_t)b * p.h_q + hq) * sq + i] =
+                    lt > 0.f ? (mx + log2f(lt)) * kLn2 : -INFINITY;
+        } else {
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
         for (int h = 0; h < D_V / 32; ++h) {
@@ -892,6 +1035,7 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
         }
         if (row_valid && p.lse)
             p.lse[p.cu_q ? (int64_t)hq * p.total_q + qoff + i : ((int64_t)b * p.h_q + hq) * sq + i] = l > 0.f ? (m_ref * c + log2f(l)) * kLn2 : -INFINITY;
+        }
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -901,29 +1045,36 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
     }
 }
 
+// The kernel's setmaxnreg split (128 x 64 + 256 x 216 registers) must fit in
+// what the block is launched with, or the increase never returns.
+template <typename K>
+static cudaError_t check_regs(K kernel, int *cached) {
+    if (*cached < 0) {
+        cudaFuncAttributes fa_attr;
+        const cudaError_t e = cudaFuncGetAttributes(&fa_attr, kernel);
+        if (e != cudaSuccess) return e;
+        *cached = fa_attr.numRegs;
+    }
+    return *cached * 384 < 128 * 64 + 256 * 216 ? cudaErrorInvalidConfiguration : cudaSuccess;
+}
+
 template <typename T, int D_QK, int D_V>
 static cudaError_t run_prefill(const PrefillParams &p, const CUtensorMap &tmQ, const CUtensorMap &tmK,
                                const CUtensorMap &tmV, cudaStream_t st) {
     if (p.tiles_per_cta == 2) {
         using C2 = Prefill2Cfg<D_QK, D_V>;
-        cudaError_t e = cudaFuncSetAttribute(prefill2_kernel<T, D_QK, D_V>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C2::SMEM);
+        auto kern = p.key_split ? prefill2_kernel<T, D_QK, D_V, true> : prefill2_kernel<T, D_QK, D_V, false>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C2::SMEM);
         if (e != cudaSuccess) return e;
-        // the kernel's setmaxnreg split (128 x 64 + 256 x 216 registers) must
-        // fit in what the block is launched with, or the increase never returns
-        static int launch_regs = -1;
-        if (launch_regs < 0) {
-            cudaFuncAttributes fa_attr;
-            e = cudaFuncGetAttributes(&fa_attr, prefill2_kernel<T, D_QK, D_V>);
-            if (e != cudaSuccess) return e;
-            launch_regs = fa_attr.numRegs;
-        }
-        if (launch_regs * 384 < 128 * 64 + 256 * 216) return cudaErrorInvalidConfiguration;
-        const int64_t nblk = (int64_t)((p.n_q_tiles + 1) / 2) * (p.h_q / p.pack) * p.b;
+        static int regs_pair = -1, regs_split = -1;
+        if ((e = check_regs(kern, p.key_split ? &regs_split : &regs_pair)) != cudaSuccess) return e;
+        // key split: one CTA per query tile; pairs: one per two tiles
+        const int64_t units = p.key_split ? p.n_q_tiles : (p.n_q_tiles + 1) / 2;
+        const int64_t nblk = units * (p.h_q / p.pack) * p.b;
         if (nblk > 0x7fffffff) return cudaErrorInvalidConfiguration;
         dim3 grid((unsigned)nblk);
         kernel_event(0, st);
-        prefill2_kernel<T, D_QK, D_V><<<grid, 384, C2::SMEM, st>>>(tmQ, tmK, tmV, p);
+        kern<<<grid, 384, C2::SMEM, st>>>(tmQ, tmK, tmV, p);
         e = cudaGetLastError();
         kernel_event(1, st);
         return e;

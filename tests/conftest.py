@@ -23,10 +23,12 @@ def cuda_device():
     return torch.device("cuda:0")
 
 
-@pytest.fixture(params=[1, 2], ids=["1tile", "2tiles"])
+@pytest.fixture(params=[1, 2, 3], ids=["1tile", "2tiles", "keysplit"])
 def prefill_tiles(request):
-    """Run the test with the one-tile and with the two-tile tcgen05 prefill
-    kernel (pinned through the library's test hook, released afterwards)."""
+    """Run the test with the one-tile tcgen05 prefill kernel, the two-tile
+    kernel on pairs of query tiles, and the two-tile kernel with one query
+    tile's key range split between its softmax warpgroups (pinned through
+    the library's test hook, released afterwards)."""
     import rotary_embedding_b200 as fa
     fa.fa_testing_set_prefill_tiles(request.param)
     yield request.param
