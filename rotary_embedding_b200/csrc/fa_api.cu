@@ -246,6 +246,10 @@ int run_tc_attention(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
     // tiles); with several waves the heaviest-first launch order balances
     // adjacent pairs, which keep both softmax warpgroups busy to the end.
     p.pair_ends = (causal && !varlen && p.tiles_per_cta == 2 && !p.key_split && ctas2 <= sms) ? 1 : 0;
+    // Over a cache the batch entries' key counts differ: order one-tile CTAs
+    // by their visible keys, computed on the device (chunked prefill with one
+    // long entry: 71.7 -> 63.5 us per call)
+    p.work_order = (kvcache && (p.tiles_per_cta == 1 || p.key_split) && b * p.n_q_tiles <= 256) ? 1 : 0;
     const int bn = prefill_block_n((int)d_qk, (int)d_v, p.tiles_per_cta);
     CUtensorMap tmQ, tmK, tmV;
     int rc;

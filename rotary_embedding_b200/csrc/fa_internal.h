@@ -126,6 +126,10 @@ struct PrefillParams {
     // the key range cut in two halves merged at the end (grid: one CTA per
     // query tile)
     int key_split;
+    // cache grids of one tile per CTA (one-tile kernel, key split): CTAs take
+    // (batch entry, query tile) items heaviest first by visible keys,
+    // computed on the device from cache_seqlens (b x n_q_tiles <= 256)
+    int work_order;
     int win_left, win_right;  // sliding window; -1 = unbounded
     // packed sequences (varlen): grid z = sequence s with query rows
     // cu_q[s] .. cu_q[s+1]-1 and key rows cu_k[s] .. of batch entry 0;

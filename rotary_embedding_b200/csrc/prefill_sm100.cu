@@ -63,6 +63,50 @@ __device__ __forceinline__ void grid_order(const PrefillParams &p, int &tile, in
     b = rem / nhg;
 }
 
+// Grids over a cache whose batch entries hold different numbers of keys:
+// the (batch entry, query tile) items are ordered by their visible keys,
+// heaviest first (longest processing time first, ties by index), all head
+// groups of an item adjacent, so the tiles of the longest entries start in
+// the first wave whatever their batch index.  The host uses it when the
+// items number b x n_q_tiles <= 256; every CTA ranks them in `scratch` (m + 1
+// ints of shared memory that no TMA has written yet), one block-wide pass.
+__device__ __forceinline__ void work_order(const PrefillParams &p, int *scratch, int &tile, int &hgrp, int &b) {
+    const int nhg = p.h_q / p.pack;
+    const int n_t = p.n_q_tiles, m = p.b * n_t;
+    const int rows = kBM / p.pack;
+    for (int i = threadIdx.x; i < m; i += blockDim.x) {
+        const int bb = i / n_t, t = i - bb * n_t;
+        const int L = seqlen_of(p.seqlens, p.seqlen_scalar, bb);
+        int w = 0;
+        const int i0 = t * rows;
+        if (L >= 0 && (int64_t)L + p.s_new <= p.cap && i0 < p.s_q) {
+            const int N = L + p.s_new;
+            const int i_last = min(p.s_q, i0 + rows) - 1;
+            int64_t f0, l0, f1, l1;
+            visible_keys(i0, N, p.s_q, p.causal, p.win_left, p.win_right, f0, l0);
+            visible_keys(i_last, N, p.s_q, p.causal, p.win_left, p.win_right, f1, l1);
+            w = (int)max((int64_t)0, min((int64_t)N - 1, l1) - max((int64_t)0, f0) + 1);
+        }
+        scratch[i] = w;
+    }
+    __syncthreads();
+    const int r = (int)blockIdx.x / nhg;
+    for (int i = threadIdx.x; i < m; i += blockDim.x) {
+        const int wi = scratch[i];
+        int rank = 0;
+        for (int j = 0; j < m; ++j) {
+            const int wj = scratch[j];
+            rank += (wj > wi) || (wj == wi && j < i);
+        }
+        if (rank == r) scratch[m] = i;   // ranks are a permutation: exactly one item
+    }
+    __syncthreads();
+    const int item = scratch[m];
+    b = item / n_t;
+    tile = item - b * n_t;
+    hgrp = (int)blockIdx.x % nhg;
+}
+
 template <int D_QK, int D_V>
 struct PrefillCfg {
     static constexpr int QBYTES = kBM * D_QK * 2;
@@ -108,7 +152,10 @@ __global__ void __launch_bounds__(256, 1) prefill_kernel(const __grid_constant__
     // heaviest causal tiles first across every head and batch entry: block L
     // takes tile n - 1 - L / (head groups x batch)
     int qt, hgrp, b;
-    grid_order(p, qt, hgrp, b);
+    if (p.work_order)
+        work_order(p, reinterpret_cast<int *>(sK), qt, hgrp, b);
+    else
+        grid_order(p, qt, hgrp, b);
     const int pack = p.pack;
     const int hq0 = hgrp * pack;                           // first query head of the tile
     const int hk = hq0 / p.g;
@@ -501,7 +548,10 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // heaviest causal blocks first across every head and batch entry
     int blk, hgrp, b;
-    grid_order(p, blk, hgrp, b);
+    if (KSPLIT && p.work_order)
+        work_order(p, reinterpret_cast<int *>(sK), blk, hgrp, b);
+    else
+        grid_order(p, blk, hgrp, b);
     const int pack = p.pack;
     const int hq0 = hgrp * pack;
     const int hk = hq0 / p.g;
