@@ -222,6 +222,20 @@ def test_kvcache_garbage_past_sequence(s_new, prefill_tiles, cuda_device):
         assert torch.equal(vc[b, L:L + s_new], inp["v_new"][b])
 
 
+@pytest.mark.parametrize("lens", [(0, 40, 300, 700, 700, 1500), (1500, 700, 700, 300, 40, 0)],
+                         ids=["ascending", "descending"])
+def test_kvcache_prefill_unequal_entries(lens, prefill_tiles, cuda_device):
+    """Cached prefill over entries of very different lengths, two of them
+    equal: one-tile grids take their (entry, query tile) items heaviest first
+    by visible keys, ranked on the device, with ties broken by index; every
+    row must land where it belongs whatever the rank order."""
+    w = W.Workload(name="unequal", mode="kvcache", dtype="fp16", batch=len(lens), h_q=4, h_kv=2, d_qk=128,
+                   d_v=128, s_q=200, cap=1800, seqlens=(0, 1), causal=True, rotary_dim=128, interleaved=True)
+    inp = W.make_inputs(w, seed=31)
+    inp["cache_seqlens"] = torch.tensor(lens, dtype=torch.int32)
+    check_kvcache(w, inp, run_gpu_kvcache(w, inp, cuda_device), run_oracle_kvcache(w, inp))
+
+
 # ------------------------------------------------------------------ full-size configurations
 def _slice_kv_inputs(inp, batches, heads=None):
     out = {}
