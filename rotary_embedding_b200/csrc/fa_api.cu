@@ -225,16 +225,13 @@ int run_tc_attention(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
     const int64_t ctas2 = (int64_t)((p.n_q_tiles + 1) / 2) * (h_q / pack) * b;
     const int64_t sms = sm_count();
     p.tiles_per_cta = (ctas2 >= 2 * sms || (d_qk <= 64 && 2 * ctas2 >= sms)) ? 2 : 1;
-    // Fewer pairs than two per SM, with work that differs between query tiles
-    // (a causal mask, or cached keys of different lengths), at d_qk <= 64:
-    // one query tile per CTA with its key range split between the two
-    // softmax warpgroups, so the CTA count doubles and both warpgroups work
-    // on every step.  Measured: d 64 dense causal 34.8 -> 32.8 us; at d 128
-    // (chunked prefill, 80-key tiles) it lost to the one-tile kernel
-    // (81.9 against 69.6 us), as did non-causal grids, whose pairs of tiles
-    // already have equal work.
-    p.key_split = (!varlen && (causal || kvcache) && d_qk <= 64 && ctas2 < 2 * sms) ? 1 : 0;
-    if (p.key_split) p.tiles_per_cta = 2;
+    // The key-split mode of the two-tile kernel (one query tile per CTA, its
+    // key range halved between the two softmax warpgroups) is not chosen
+    // here: on the small causal grid it measured the same as pairs of tiles
+    // (d 64 dense causal 29.4 against 29.3 us per call, ten calls per graph),
+    // and at d 128 slower than the one-tile kernel (chunked prefill 65.7
+    // against 57.3 us).  The test hook reaches it.
+    p.key_split = 0;
     // a test may pin the kernel (fa_testing_set_prefill_tiles: 3 = key split)
     if (g_forced_tiles) {
         p.tiles_per_cta = g_forced_tiles == 1 ? 1 : 2;
