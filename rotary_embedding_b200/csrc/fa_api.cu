@@ -133,7 +133,12 @@ EncodeTiledFn encode_fn() {
 // 4-D map over a [batch, rows, heads, dim] tensor, dims ordered (dim, heads,
 // rows, batch); box = (min(d, 64), box_h, box_rows, 1) with the swizzle that
 // matches the box row width.
-int make_rows_map(CUtensorMap *map, const fa_tensor *t, int box_rows, const char *name, int box_h = 1) {
+// L2 promotion: 256 B by default; the decode kernel's K/V maps take 128 B, because a
+// kv head's row there is streamed once under evict-first, and with a
+// 384-byte row (d 192) a 256-byte promotion fetches the neighbouring head's
+// 128 bytes, which are often evicted before that head's CTA reads them.
+int make_rows_map(CUtensorMap *map, const fa_tensor *t, int box_rows, const char *name, int box_h = 1,
+                  CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     const int64_t d = t->shape[3];
@@ -153,7 +158,7 @@ int make_rows_map(CUtensorMap *map, const fa_tensor *t, int box_rows, const char
     CUtensorMapDataType dt = t->dtype == FA_DTYPE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                       : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     CUresult r = fn(map, dt, 4, t->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed (%d)", name, (int)r);
     return FA_OK;
 }
@@ -637,8 +642,8 @@ int fa_kvcache_fwd_window(const fa_tensor *q, const fa_tensor *k_cache, const fa
         qr.stride[0] = a.s_q * a.h_q * a.d_qk;
         CUtensorMap tmQ, tmK, tmV;
         if ((rc = make_rows_map(&tmQ, &qr, (int)a.s_q, "q_rot", (int)(a.h_q / a.h_kv)))) return rc;
-        if ((rc = make_rows_map(&tmK, k_cache, 64, "k_cache"))) return rc;
-        if ((rc = make_rows_map(&tmV, v_cache, 64, "v_cache"))) return rc;
+        if ((rc = make_rows_map(&tmK, k_cache, 64, "k_cache", 1, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))) return rc;
+        if ((rc = make_rows_map(&tmV, v_cache, 64, "v_cache", 1, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))) return rc;
         DecodeParams p{};
         p.status = status;
         p.cs_rows = a.s_ro;
