@@ -202,3 +202,23 @@ def test_binding_rejects_host_tensors():
     lse = torch.zeros(2, 4, 3)
     with pytest.raises(ValueError, match="CUDA"):
         fa.fa_bwd(q, kc[:, :3], vc[:, :3], out, out, lse)
+
+
+def test_descriptor_cache_keys_on_every_field():
+    # the binding reuses a descriptor only for the same address, dtype, shape and strides
+    base = torch.zeros(4, 6, 2, 64, dtype=torch.float16)
+    d1 = fa.describe(base)
+    assert fa.describe(base) is d1
+    assert (d1.data, d1.ndim, list(d1.shape), list(d1.stride)) == (base.data_ptr(), 4, [4, 6, 2, 64],
+                                                                    [768, 128, 64, 1])
+    view = base[:, :3]                                   # same address, other shape
+    d2 = fa.describe(view)
+    assert d2 is not d1 and list(d2.shape) == [4, 3, 2, 64] and d2.data == d1.data
+    t = base.transpose(1, 2)                             # same address, other strides
+    d3 = fa.describe(t)
+    assert list(d3.stride) == [768, 64, 128, 1] and list(d3.shape) == [4, 2, 6, 64]
+    other = base.view(torch.bfloat16)                    # same address and layout, other dtype
+    assert fa.describe(other).dtype != d1.dtype
+    small = torch.zeros(5, 3, dtype=torch.float16)       # rank below 4 pads with zeros
+    d4 = fa.describe(small)
+    assert d4.ndim == 2 and list(d4.shape) == [5, 3, 0, 0] and list(d4.stride) == [3, 1, 0, 0]
