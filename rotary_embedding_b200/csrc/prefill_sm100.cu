@@ -36,12 +36,13 @@ namespace fa {
 // Pairs out of every 8 whose 2^x the two-tile softmax evaluates on the FMA
 // pipe (ex2_poly2) instead of the special function unit, in unmasked tiles.
 // At d_qk <= 64 a key tile's scores cost little tensor time next to their
-// exponentials and the special function unit bounds the softmax, so 3 of 8
+// exponentials and the special function unit bounds the softmax, so 2 of 8
 // pairs move; at larger d_qk that unit has room and the polynomial's extra
 // instructions only lengthen the softmax (measured: d_qk 192 3 % faster with
-// none, d_qk 64 equal or slower with fewer).
+// none; d_qk 64 with the 56 / 224 register split: 2 of 8 1.6 % faster than 3
+// on the non-causal grid and equal on the causal one, 4 of 8 slower).
 #ifndef FA_EXP2_EMU_PAIRS
-#define FA_EXP2_EMU_PAIRS 3
+#define FA_EXP2_EMU_PAIRS 2
 #endif
 template <int D_QK>
 constexpr int exp2_emu_pairs() { return D_QK <= 64 ? FA_EXP2_EMU_PAIRS : 0; }
