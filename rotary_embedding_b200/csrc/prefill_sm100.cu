@@ -940,10 +940,10 @@ __global__ void __launch_bounds__(384, 1) prefill2_kernel(const __grid_constant_
             }
             // P = 2^(s c - m c) as 16-bit pairs into the P buffer (keys
             // [2k, 2k+2) -> column k).  In tiles without masked keys and at
-            // d_qk <= 64, 3 of every 8 pairs take 2^x on the FMA pipe
-            // (ex2_poly2) and the rest on the special function unit
-            // (exp2_emu_pairs); masked tiles need exact zeros and use the
-            // special function unit throughout.  The fp32 P values overwrite S
+            // d_qk <= 64, exp2_emu_pairs() of every 8 pairs (2) take 2^x on
+            // the FMA pipe (ex2_poly2) and the rest on the special function
+            // unit; masked tiles need exact zeros and use the special
+            // function unit throughout.  The fp32 P values overwrite S
             // in registers; the row sum is taken after P has been handed to
             // the MMA warp (off the critical path).
             // one pair of scores (a, b) -> P values in place, packed 16-bit pair returned
